@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer forward pass on B200 GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--dtype bf16|f32] [--cf CF] [--impl ours|reference]
+
+One step = one whole forward pass of the layer (router -> dispatch ->
+grouped expert FFN -> combine -> statistics) over one batch of the
+workload's synthetic tokens, inputs resident in HBM.  The default workload
+is the Switch-style top-1 layer (T=4096, d=768, ff=3072, 32 experts, bf16,
+capacity factor 1.0).  L2 is flushed (a 256 MiB write) before every step,
+outside the per-step device timing.
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica of the same layer: there is no data-path collective.  The timed
+region is bracketed by a barrier and a device synchronisation on both
+sides; its device time is reduced with MAX over ranks and the value is the
+tokens processed by all ranks divided by that time.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the float64 CPU
+oracle (the correctness reference, a deliberately plain program) on a
+bounded sample of the same workload on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s on 1 B200; expert-FFN TFLOP/s as % of bf16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="switch-top1")
+    ap.add_argument("--dtype", default=None, help="bf16 or f32 (switch-top1 only; default bf16)")
+    ap.add_argument("--cf", type=float, default=None, help="capacity factor (switch-top1: 1.0 or 1.5)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget for the oracle baseline")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    return ap.parse_args(argv)
+
+
+def get_workload(args):
+    from mixture_experts_layer_45_b200 import workloads as wl
+    kw = {}
+    if args.dtype is not None:
+        kw["dtype"] = args.dtype
+    if args.cf is not None:
+        kw["cf"] = args.cf
+    return wl.workload(args.workload, **kw)
+
+
+def workload_label(w) -> str:
+    return (f"{w.name} T={w.T} d={w.d} ff={w.ff} E={w.E} k={w.k} {w.dtype} "
+            f"cf={w.capacity_factor_label()}")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region (NVML, in-process)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {  # NVML clocks-event-reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, interval_s: float = 0.005):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # NVML unavailable: report it, do not guess
+            self.error = str(e)
+        self._interval = interval_s
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
+                self.samples.append((mhz, reasons, util))
+            except Exception:
+                pass
+            time.sleep(self._interval)
+
+    def start(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def stop(self):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        reasons = set()
+        for _, r, _ in loaded:
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[0] for s in loaded]) if loaded else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# the committed ncu traffic summary for the dominant kernel (null when the
+# kernel sources changed since it was captured)
+# ---------------------------------------------------------------------------
+KERNEL_SOURCES = {
+    "ffn1": ["ffn.cuh", "common.cuh"], "ffn2": ["ffn.cuh", "common.cuh"],
+    "router": ["router.cuh", "common.cuh"], "combine": ["dispatch.cuh", "common.cuh"],
+    "gather": ["dispatch.cuh", "common.cuh"], "permute": ["dispatch.cuh", "common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        with open(os.path.join(ROOT, "mixture_experts_layer_45_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, workload_tag: str):
+    """Per-launch DRAM bytes from profiles/<kernel>_<workload_tag>.md, or None."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload_tag}.md")
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != kernel_source_hash(kernel):
+        return None
+    return float(m.group(1))
+
+
+def workload_tag(w) -> str:
+    return f"{w.name}-{w.dtype}-cf{w.capacity_factor_label()}"
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
+    except Exception:
+        return None
+
+
+def oracle_sample_inputs(w, sample_T):
+    """A bounded sample of the workload: its first sample_T tokens (the same
+    seeded draws), with the capacity recomputed for the sample's size."""
+    from mixture_experts_layer_45_b200 import workloads as wl
+    inp = wl.draw_inputs(w)
+    inp = dict(inp)
+    inp["x"] = inp["x"][:sample_T]
+    from oracle import moe_ref
+    cap = moe_ref.capacity(sample_T, w.k, w.E, w.cf)
+    return inp, cap
+
+
+def time_oracle(w, seconds: float, sample_T: int):
+    from oracle import moe_ref
+    inp, cap = oracle_sample_inputs(w, sample_T)
+    moe_ref.moe_layer(inp, w.k, cap)          # warm-up
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        moe_ref.moe_layer(inp, w.k, cap)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return n * sample_T / dt, n, dt
+
+
+def cpu_baseline(w, seconds: float):
+    sample_T = min(w.T, 1024)
+    tps, n, dt = time_oracle(w, seconds, sample_T)
+    cores = len(os.sched_getaffinity(0))
+    return {"value": tps, "unit": "tokens/s", "cores": cores, "blas_threads": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} float64 oracle passes over the first {sample_T} tokens of {workload_label(w)} "
+                      f"(capacity recomputed for the sample), {dt:.1f} s wall"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = get_workload(args)
+    from oracle import moe_ref
+    sample_T = min(w.T, 512)
+    inp, cap = oracle_sample_inputs(w, sample_T)
+    for _ in range(args.warmup):
+        moe_ref.moe_layer(inp, w.k, cap)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        moe_ref.moe_layer(inp, w.k, cap)
+    dt = time.perf_counter() - t0
+    value = args.steps * sample_T / dt
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * dt / max(args.steps, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy draws)",
+        "config": {"workload": workload_label(w), "sample_tokens_per_step": sample_T,
+                   "parallelism": "host cores (rank 0 only)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "blas_threads": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: float64 oracle over the first {sample_T} tokens"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def algorithmic_bytes(kernel, w, R, E_active, es):
+    d, ff, T, k, E = w.d, w.ff, w.T, w.k, w.E
+    if kernel == "ffn1":
+        return E_active * ff * d * es + E * ff * es + R * d * es + R * ff * es
+    if kernel == "ffn2":
+        return E_active * d * ff * es + E * d * es + R * ff * es + R * d * es + R * 4
+    if kernel == "router":
+        return T * d * es + E * d * es + T * k * 8 + E * 4
+    if kernel == "gather":
+        return 2 * R * d * es + R * 4
+    if kernel == "combine":
+        return R * d * es + T * d * es + T * k * 4
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"bench: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    from mixture_experts_layer_45_b200 import _lib
+    from mixture_experts_layer_45_b200 import build as build_mod
+    from mixture_experts_layer_45_b200.layer import MoELayer, MoEParams, dtype_code, read_stats, to_device
+    from mixture_experts_layer_45_b200 import workloads as wl
+
+    if rank == 0:
+        build_mod.build()
+    if world > 1:
+        dist.barrier()
+    _lib.load()
+
+    w = get_workload(args)
+    dt = dtype_code(w.dtype)
+    es = 2 if w.dtype == "bf16" else 4
+    inp = wl.draw_inputs(w)
+    dev = torch.device("cuda", local_rank)
+    params = MoEParams.from_arrays(inp, dt, dev)
+    cap = _lib.moe_capacity(w.T, w.k, w.E, w.cf)
+    layer = MoELayer(params, w.k, cap)
+    x = to_device(inp["x"], dt, dev)
+    out = torch.empty_like(x)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # warm-up (W >= 3 enforced)
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        layer.forward(x, out=out, stats=True)
+    if _lib.moe_get_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    st = read_stats(layer.stats_buf)
+    R = int(st["rows_kept"])
+
+    # count of experts with at least one kept row (their weights are read)
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
+    layer.forward(x, out=out, topk_idx=idx)
+    from collections import Counter
+    cnt = Counter(idx.flatten().tolist())
+    E_active = sum(1 for e in range(w.E) if cnt.get(e, 0) > 0 and cap != 0)   # experts with kept rows
+
+    sampler = ClockSampler(local_rank).start() if rank == 0 else None
+    time.sleep(0.05)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    _lib.moe_timing_enable(True)
+    _lib.moe_timing_read()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = _lib.moe_launch_count()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        layer.forward(x, out=out, stats=True)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = _lib.moe_launch_count() - n0
+    kt = _lib.moe_timing_read()
+    _lib.moe_timing_enable(False)
+    if sampler:
+        sampler.stop()
+    err = _lib.moe_get_error()
+    if err != 0:
+        raise RuntimeError(f"device error in the timed region: {_lib.status_string(err)}")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    value = world * args.steps * w.T / (total_ms / 1000.0)
+
+    # ---- end to end through the public API: pinned host in, pinned host out
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 50))
+    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_host.copy_(x.cpu())
+    out_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_dev2 = torch.empty_like(x)
+    out_dev2 = torch.empty_like(x)
+    for _ in range(3):
+        layer.forward_host(x_host, out_host, x_dev2, out_dev2)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        x_dev2.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev2, out=out_dev2)
+        out_host.copy_(out_dev2, non_blocking=True)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_value = world * e2e_steps * w.T / (float(te.item()) / 1000.0)
+    io_bytes = x.numel() * x.element_size()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    kernels = {}
+    tot_k = sum(ms for ms, n in kt.values() if n)
+    for name, (ms, n) in kt.items():
+        if n:
+            kernels[name] = {"launches": n, "ms_per_launch": ms / n, "share": ms / tot_k if tot_k else None}
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
+    ffn_ms = sum(kernels[k]["ms_per_launch"] for k in ("ffn1", "ffn2") if k in kernels)
+    ffn_flops = 4.0 * R * w.d * w.ff
+    ffn_tflops = ffn_flops / (ffn_ms / 1000.0) / 1e12 if ffn_ms else None
+    dom_bytes = algorithmic_bytes(dom, w, R, E_active, es)
+    dom_s = kernels[dom]["ms_per_launch"] / 1000.0
+    # a kernel timed inside a long run meets the power cap: use the sustained tensor peak there
+    tensor_peak = peaks["bf16_tflops"] if total_ms < 2000 else peaks["bf16_tflops_sustained"]
+    flops_dom = 2.0 * R * w.d * w.ff
+    ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if dom in ("ffn1", "ffn2") and w.dtype == "bf16" and flops_dom / max(dom_bytes, 1) > ridge:
+        achieved = flops_dom / dom_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak}
+    else:
+        achieved = dom_bytes / dom_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof.update({"kernel": dom, "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes,
+                 "traffic": committed_traffic(dom, workload_tag(w))})
+
+    clocks = sampler.summary() if sampler else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": warm, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded numpy draws of the workload's distributions; random-init weights)",
+        "config": {"workload": workload_label(w), "T": w.T, "d": w.d, "ff": w.ff, "E": w.E, "k": w.k,
+                   "capacity": cap, "rows_kept": R,
+                   "l2": "flushed before every step (256 MiB write), outside the step timing",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "ffn": {"tflops": ffn_tflops, "frac_of_bf16_peak": (ffn_tflops / peaks["bf16_tflops"]) if ffn_tflops
+                else None, "flops_per_step": ffn_flops, "ms_per_step": ffn_ms},
+        "kernels": kernels,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
+                "d2h_bytes_per_step": io_bytes, "steps": e2e_steps},
+        "clocks": clocks,
+        "gpu_launches": launches,
+        "stats": {k: st[k] for k in ("aux_loss", "imbalance", "drop_rate")},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

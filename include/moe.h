@@ -1,0 +1,238 @@
+/*
+ * moe.h -- C ABI of libmoe: the forward pass of one Mixture-of-Experts layer
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one stated in the cookbook notebook "Mixture-of-experts
+ * and expert parallelism" (llm-systems-cookbook, 05_serving/09):
+ *
+ *   router   (section "Top-k router")          logits = x W_r^T, gates =
+ *            softmax(logits), the k largest gates and their experts; the
+ *            weights are the raw probabilities (not renormalised).
+ *   dispatch (sections "Capacity factor" and "Dispatch and gather")
+ *            per-expert counts of the T*k assignments, the slot budget
+ *            int(T*k/E*cf), and the grouping of tokens by expert.
+ *   experts  (section "Dispatch and gather")    y = fc2(gelu(fc1(x))) with
+ *            biased Linear layers and the exact erf GELU.
+ *   combine  (section "Dispatch and gather")    out[t] = sum over t's kept
+ *            assignments of gate * expert output; 0 when none is kept.
+ *   stats    (sections "Capacity factor", "Switch Transformer auxiliary
+ *            loss")  imbalance, drop rate and L_aux = E * sum_e f_e p_e.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every tensor is contiguous, row-major, in DEVICE memory owned by the
+ *   caller.  The library never frees or keeps a caller pointer after the
+ *   call returns.  Tensor base pointers must be 16-byte aligned.
+ * - dtype is MOE_F32 (float) or MOE_BF16 (bfloat16 bits in uint16).  It is
+ *   the type of x, the router and expert weights and biases, the grouped
+ *   activations and the output.  Indices are int32; gates, probability sums
+ *   and statistics are float.  Accumulation is always fp32.
+ * - Sizes: T >= 0 tokens (T == 0 returns MOE_OK and launches nothing),
+ *   1 <= E <= MOE_MAX_EXPERTS experts, 1 <= k <= min(E, MOE_MAX_TOPK),
+ *   d and ff positive multiples of 8, T*k < 2^31.
+ * - Layouts: x [T,d]; w_router [E,d]; logit_bias [E] float; w1 [E,ff,d];
+ *   b1 [E,ff]; w2 [E,d,ff]; b2 [E,d]  (nn.Linear's [out,in] weight layout,
+ *   experts stacked on the leading axis).  Assignment a = t*k + j is token
+ *   t's j-th choice (j = 0 is the largest gate).
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *   legacy default stream) and never synchronises the host, except
+ *   moe_get_error and moe_timing_read.  Calls are CUDA-graph capturable.
+ * - Errors: argument and shape errors are returned synchronously, before
+ *   anything is launched (MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED,
+ *   MOE_ERR_WORKSPACE).  A failed launch returns MOE_ERR_CUDA.  Errors that
+ *   only the device can see (an expert index outside [0,E) given to
+ *   moe_dispatch, a pipeline wait that ran out of time) are recorded in a
+ *   per-device error word and reported by moe_get_error; the affected
+ *   outputs are then unspecified but every kernel still terminates.
+ * - No C++ exception crosses this interface.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define MOE_OK               0
+#define MOE_ERR_INVALID_ARG  1  /* null pointer, bad size, k > E, misaligned pointer */
+#define MOE_ERR_UNSUPPORTED  2  /* dtype, d or ff not a multiple of 8, E or k above the limits */
+#define MOE_ERR_WORKSPACE    3  /* workspace missing or smaller than the size query returns */
+#define MOE_ERR_CUDA         4  /* a CUDA runtime call or kernel launch failed */
+#define MOE_ERR_BAD_ROUTING  5  /* device: an expert index outside [0, E) */
+#define MOE_ERR_TIMEOUT      6  /* device: a bounded pipeline wait gave up */
+
+/* ---- dtypes ------------------------------------------------------------ */
+#define MOE_F32   0
+#define MOE_BF16  1
+
+#define MOE_MAX_EXPERTS 256
+#define MOE_MAX_TOPK    8
+
+/* Layer statistics, written to DEVICE memory by moe_forward / moe_layer_stats.
+ * Definitions (notebook sections "Capacity factor" and "Switch Transformer
+ * auxiliary loss"), with counts taken before any capacity drop:
+ *   aux_loss  = E * sum_e (counts_e / T) * (prob_sum_e / T)
+ *   imbalance = max_e counts_e / (T*k/E)
+ *   drop_rate = dropped / (T*k)                                         */
+typedef struct moe_stats {
+    float   aux_loss;
+    float   imbalance;
+    float   drop_rate;
+    int32_t rows_kept;   /* R = sum_e min(counts_e, capacity) */
+    int32_t max_count;   /* max_e counts_e */
+    int32_t dropped;     /* T*k - R */
+} moe_stats;
+
+/* Human-readable name of a status code (static storage). */
+MOE_API const char* moe_status_string(int status);
+
+/* ABI version of this header: major*10000 + minor*100 + patch. */
+MOE_API int moe_version(void);
+
+/* Slot budget per expert, int(T*k/E*cf) computed in double (notebook section
+ * "Capacity factor"; int() truncates).  cf <= 0 means no limit: returns -1.
+ * Returns -1 also for invalid sizes (T < 0, k < 1, E < 1). */
+MOE_API int moe_capacity(int T, int k, int E, double cf);
+
+/* Bytes of workspace moe_forward needs for these sizes (0 for invalid
+ * arguments).  The workspace holds the routing, the dispatch arrays and the
+ * grouped activations xp [T*k,d], h [T*k,ff] and yp [T*k,d]. */
+MOE_API size_t moe_workspace_size(int T, int d, int ff, int E, int k, int dtype);
+
+/* Bytes of scratch moe_dispatch needs (per-block expert histograms). */
+MOE_API size_t moe_dispatch_workspace_size(int T, int k, int E);
+
+/* ---- step 1: router (notebook section "Top-k router") ------------------
+ * logits[t,e] = sum_i x[t,i] w_router[e,i] (+ logit_bias[e]) accumulated in
+ * fp32; g = softmax over e in fp32; the k experts with the largest logits,
+ * in descending order, an exact tie going to the lower expert index.
+ *   x          [T,d] dtype           w_router [E,d] dtype
+ *   logit_bias [E] float or NULL     (added to the logits)
+ *   topk_idx   [T,k] int32 (out)     topk_gate [T,k] float (out): g at those experts
+ *   prob_sum   [E] float or NULL (out): sum over tokens of g[t,e]; it is
+ *              overwritten (zeroed on the stream first).
+ * Supports E <= MOE_MAX_EXPERTS, k <= MOE_MAX_TOPK. */
+MOE_API int moe_router_topk(const void* x, const void* w_router, const float* logit_bias,
+                    int T, int d, int E, int k, int dtype,
+                    int32_t* topk_idx, float* topk_gate, float* prob_sum,
+                    void* stream);
+
+/* ---- step 2: dispatch (notebook sections "Capacity factor", "Dispatch and
+ * gather") -----------------------------------------------------------------
+ * counts[e]  = #{a : topk_idx[a] == e}                       (before drops)
+ * kept_e     = counts[e] if capacity < 0, else min(counts[e], capacity)
+ * offsets    = exclusive prefix sum of kept; offsets[E] = R rows kept
+ * Expert e keeps its first kept_e assignments in token order; they occupy
+ * grouped rows offsets[e] .. offsets[e+1]-1 in that order:
+ *   perm[row]   = a of the assignment in that row            (rows < R)
+ *   slot_of[a]  = its row, or -1 if the assignment was dropped
+ *   drop_mask[a]= 1 if dropped, else 0
+ *   row_gate[row] = topk_gate[perm[row]]     (if topk_gate and row_gate are given)
+ *   xp[row,:]   = x[perm[row] / k, :]        (if x and xp are given)
+ * Every output is produced exactly (integer work, bit-reproducible, no
+ * dependence on thread timing).  perm, row_gate and xp are sized for T*k
+ * rows; rows >= R are left untouched.
+ *   ws/ws_bytes: scratch of at least moe_dispatch_workspace_size(T,k,E).
+ * An index outside [0,E) is dropped and raises MOE_ERR_BAD_ROUTING in the
+ * device error word. */
+MOE_API int moe_dispatch(const int32_t* topk_idx, const float* topk_gate,
+                 int T, int k, int E, int capacity,
+                 int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                 uint8_t* drop_mask, float* row_gate,
+                 const void* x, void* xp, int d, int dtype,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* ---- step 3: grouped expert FFN (notebook section "Dispatch and gather")
+ * For each expert e and each row r in offsets[e] .. offsets[e+1]-1:
+ *   h[r,:]  = gelu(xp[r,:] W1_e^T + b1_e)          (exact erf GELU)
+ *   yp[r,:] = g_r * (h[r,:] W2_e^T + b2_e),  g_r = row_gate[r] or 1 if NULL
+ * offsets is read on the device (no host synchronisation); max_rows is the
+ * number of rows xp, h and yp are allocated for (>= offsets[E], normally
+ * T*k).  h is caller-provided scratch [max_rows, ff].  bf16 runs on the
+ * tcgen05 tensor cores with fp32 accumulation in tensor memory; h and yp are
+ * rounded to bf16.  f32 runs in fp32 FMA. */
+MOE_API int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows,
+                    int E, int d, int ff,
+                    const void* w1, const void* b1, const void* w2, const void* b2,
+                    const float* row_gate, void* h, void* yp, int dtype,
+                    void* stream);
+
+/* ---- step 4: combine (notebook section "Dispatch and gather") ----------
+ * out[t,:] = sum_{j<k, slot_of[t*k+j] >= 0} w_tj * yp[slot_of[t*k+j], :]
+ * with w_tj = topk_gate[t*k+j], or 1 when topk_gate is NULL (gate already
+ * applied by moe_grouped_ffn).  Summed in fp32 in slot order j; a token
+ * whose every assignment was dropped gets 0.  out is [T,d] dtype. */
+MOE_API int moe_combine(const void* yp, const int32_t* slot_of, const float* topk_gate,
+                int T, int k, int d, int dtype, void* out, void* stream);
+
+/* ---- statistics (notebook sections "Capacity factor", "Switch
+ * Transformer auxiliary loss") ---------------------------------------------
+ * From counts [E], offsets [E+1] (moe_dispatch) and prob_sum [E]
+ * (moe_router_topk), writes one moe_stats to DEVICE memory. */
+MOE_API int moe_layer_stats(const int32_t* counts, const int32_t* offsets, const float* prob_sum,
+                    int T, int k, int E, moe_stats* stats, void* stream);
+
+/* ---- the whole layer ---------------------------------------------------
+ * Router -> dispatch -> grouped FFN -> combine (-> stats), all on `stream`,
+ * no host synchronisation.  capacity < 0 means no limit (see moe_capacity).
+ *   out           [T,d] dtype (out)
+ *   stats         one moe_stats in device memory, or NULL
+ *   topk_idx_out  [T,k] int32 or NULL: the routing, if the caller wants it
+ *   topk_gate_out [T,k] float or NULL
+ *   ws/ws_bytes   workspace of at least moe_workspace_size(T,d,ff,E,k,dtype)
+ *                 bytes, 256-byte aligned. */
+MOE_API int moe_forward(const void* x, const void* w_router, const float* logit_bias,
+                const void* w1, const void* b1, const void* w2, const void* b2,
+                int T, int d, int ff, int E, int k, int capacity, int dtype,
+                void* out, moe_stats* stats,
+                int32_t* topk_idx_out, float* topk_gate_out,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* ---- errors, counters, timing -------------------------------------------
+ * moe_get_error: synchronises `stream`, then reads and clears the current
+ * device's error word.  Returns MOE_OK, MOE_ERR_BAD_ROUTING,
+ * MOE_ERR_TIMEOUT, or MOE_ERR_CUDA if the synchronisation itself failed. */
+MOE_API int moe_get_error(void* stream);
+
+/* Number of kernels this library has launched in this process. */
+MOE_API uint64_t moe_launch_count(void);
+
+/* Kernel identifiers for moe_timing_read. */
+#define MOE_KERNEL_ROUTER   0
+#define MOE_KERNEL_COUNT    1
+#define MOE_KERNEL_SCAN     2
+#define MOE_KERNEL_PERMUTE  3
+#define MOE_KERNEL_GATHER   4
+#define MOE_KERNEL_FFN1     5
+#define MOE_KERNEL_FFN2     6
+#define MOE_KERNEL_COMBINE  7
+#define MOE_KERNEL_STATS    8
+#define MOE_NUM_KERNELS     9
+
+/* moe_timing_enable(1): from now on every kernel launch is bracketed by
+ * two CUDA events on its stream (events come from a pool created here, not
+ * per call).  moe_timing_enable(0) stops recording.  Not thread-safe
+ * against concurrent launches from several host threads. */
+MOE_API int moe_timing_enable(int enable);
+
+/* Synchronises on the recorded events and returns, per kernel identifier,
+ * the summed device time in milliseconds and the number of launches since
+ * the last read; then clears the record.  Arrays have MOE_NUM_KERNELS
+ * entries; either may be NULL. */
+MOE_API int moe_timing_read(double* ms_per_kernel, int64_t* launches_per_kernel);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,191 @@
+"""ctypes binding of libmoe (include/moe.h): the same entry points, argument
+marshalling only.  Every computation happens in the CUDA library; there is
+no Python or CPU fallback, and a missing library raises on first use.
+
+Tensors are passed as torch tensors (or None for a NULL pointer) and
+reduced to their device pointers; ``stream`` is a ``torch.cuda.Stream``, a
+raw ``cudaStream_t`` integer, or None for torch's current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_WORKSPACE = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_BAD_ROUTING = 5
+MOE_ERR_TIMEOUT = 6
+
+MOE_F32 = 0
+MOE_BF16 = 1
+MOE_MAX_EXPERTS = 256
+MOE_MAX_TOPK = 8
+
+KERNEL_NAMES = ["router", "count", "scan", "permute", "gather", "ffn1", "ffn2", "combine", "stats"]
+MOE_NUM_KERNELS = len(KERNEL_NAMES)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class MoeStats(ctypes.Structure):
+    _fields_ = [("aux_loss", ctypes.c_float), ("imbalance", ctypes.c_float), ("drop_rate", ctypes.c_float),
+                ("rows_kept", ctypes.c_int32), ("max_count", ctypes.c_int32), ("dropped", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SIGS = {
+    "moe_status_string": (ctypes.c_char_p, [_I]),
+    "moe_version": (_I, []),
+    "moe_capacity": (_I, [_I, _I, _I, ctypes.c_double]),
+    "moe_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
+    "moe_dispatch_workspace_size": (ctypes.c_size_t, [_I, _I, _I]),
+    "moe_router_topk": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P,
+                          ctypes.c_size_t, _P]),
+    "moe_grouped_ffn": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
+    "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "moe_layer_stats": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
+    "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                         ctypes.c_size_t, _P]),
+    "moe_get_error": (_I, [_P]),
+    "moe_launch_count": (ctypes.c_uint64, []),
+    "moe_timing_enable": (_I, [_I]),
+    "moe_timing_read": (_I, [_P, _P]),
+}
+EXPORTED = sorted(_SIGS)
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmoe.so (once).  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(f"libmoe.so not found at {path}; build it with "
+                                   "`python -m mixture_experts_layer_45_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+        return _lib
+
+
+def status_string(status: int) -> str:
+    return load().moe_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str):
+    if rc != MOE_OK:
+        raise MoeError(rc, where)
+
+
+# ---- entry points (names as in include/moe.h) -----------------------------
+
+def moe_version() -> int:
+    return load().moe_version()
+
+
+def moe_capacity(T: int, k: int, E: int, cf) -> int:
+    return load().moe_capacity(T, k, E, 0.0 if cf is None else float(cf))
+
+
+def moe_workspace_size(T, d, ff, E, k, dtype) -> int:
+    return load().moe_workspace_size(T, d, ff, E, k, dtype)
+
+
+def moe_dispatch_workspace_size(T, k, E) -> int:
+    return load().moe_dispatch_workspace_size(T, k, E)
+
+
+def moe_router_topk(x, w_router, logit_bias, T, d, E, k, dtype, topk_idx, topk_gate, prob_sum, stream=None):
+    _check(load().moe_router_topk(_ptr(x), _ptr(w_router), _ptr(logit_bias), T, d, E, k, dtype,
+                                  _ptr(topk_idx), _ptr(topk_gate), _ptr(prob_sum), _stream(stream)),
+           "moe_router_topk")
+
+
+def moe_dispatch(topk_idx, topk_gate, T, k, E, capacity, counts, offsets, perm, slot_of, drop_mask, row_gate,
+                 x, xp, d, dtype, ws, ws_bytes, stream=None):
+    _check(load().moe_dispatch(_ptr(topk_idx), _ptr(topk_gate), T, k, E, capacity, _ptr(counts), _ptr(offsets),
+                               _ptr(perm), _ptr(slot_of), _ptr(drop_mask), _ptr(row_gate), _ptr(x), _ptr(xp),
+                               d, dtype, _ptr(ws), ws_bytes, _stream(stream)),
+           "moe_dispatch")
+
+
+def moe_grouped_ffn(xp, offsets, max_rows, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype, stream=None):
+    _check(load().moe_grouped_ffn(_ptr(xp), _ptr(offsets), max_rows, E, d, ff, _ptr(w1), _ptr(b1), _ptr(w2),
+                                  _ptr(b2), _ptr(row_gate), _ptr(h), _ptr(yp), dtype, _stream(stream)),
+           "moe_grouped_ffn")
+
+
+def moe_combine(yp, slot_of, topk_gate, T, k, d, dtype, out, stream=None):
+    _check(load().moe_combine(_ptr(yp), _ptr(slot_of), _ptr(topk_gate), T, k, d, dtype, _ptr(out),
+                              _stream(stream)),
+           "moe_combine")
+
+
+def moe_layer_stats(counts, offsets, prob_sum, T, k, E, stats, stream=None):
+    _check(load().moe_layer_stats(_ptr(counts), _ptr(offsets), _ptr(prob_sum), T, k, E, _ptr(stats),
+                                  _stream(stream)),
+           "moe_layer_stats")
+
+
+def moe_forward(x, w_router, logit_bias, w1, b1, w2, b2, T, d, ff, E, k, capacity, dtype, out, stats,
+                topk_idx_out, topk_gate_out, ws, ws_bytes, stream=None):
+    _check(load().moe_forward(_ptr(x), _ptr(w_router), _ptr(logit_bias), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2),
+                              T, d, ff, E, k, capacity, dtype, _ptr(out), _ptr(stats), _ptr(topk_idx_out),
+                              _ptr(topk_gate_out), _ptr(ws), ws_bytes, _stream(stream)),
+           "moe_forward")
+
+
+def moe_get_error(stream=None) -> int:
+    return load().moe_get_error(_stream(stream))
+
+
+def moe_launch_count() -> int:
+    return int(load().moe_launch_count())
+
+
+def moe_timing_enable(enable: bool):
+    _check(load().moe_timing_enable(1 if enable else 0), "moe_timing_enable")
+
+
+def moe_timing_read():
+    """{kernel name: (total ms, launches)} since the last read."""
+    ms = (ctypes.c_double * MOE_NUM_KERNELS)()
+    n = (ctypes.c_int64 * MOE_NUM_KERNELS)()
+    _check(load().moe_timing_read(ctypes.cast(ms, _P), ctypes.cast(n, _P)), "moe_timing_read")
+    return {name: (ms[i], int(n[i])) for i, name in enumerate(KERNEL_NAMES)}

@@ -1,0 +1,254 @@
+// Step 2 of the layer: dispatch (cookbook notebook "Mixture-of-experts and
+// expert parallelism", sections "Capacity factor" and "Dispatch and
+// gather").  Groups the T*k assignments by expert, expert e keeping its first
+// kept_e = min(count_e, capacity) assignments in token order.
+//
+// Four launches, none of which lets thread timing decide a position:
+//   count    per-chunk expert histograms (shared-memory integer atomics;
+//            integer addition commutes, so the counts are exact)
+//   scan     per-(chunk, expert) bases, counts, capacity clamp, offsets
+//   permute  stable in-chunk ranks from warp match/ballot masks, then
+//            perm / slot_of / drop_mask / row_gate
+//   gather   xp[row] = x[token of perm[row]], one warp per row, 16-byte copies
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kDispThreads = 256;
+constexpr int kDispWarps = kDispThreads / 32;
+constexpr int kDispChunk = 2048;                       // assignments per CTA
+constexpr int kDispPerWarp = kDispChunk / kDispWarps;  // 256 = 8 rounds of 32
+
+__global__ void __launch_bounds__(kDispThreads)
+dispatch_count_kernel(const int32_t* __restrict__ idx, int A, int E, int32_t* __restrict__ hist) {
+    __shared__ int h[MOE_MAX_EXPERTS];
+    for (int e = threadIdx.x; e < E; e += kDispThreads) h[e] = 0;
+    __syncthreads();
+    const int a0 = blockIdx.x * kDispChunk;
+    for (int i = threadIdx.x; i < kDispChunk; i += kDispThreads) {
+        const int a = a0 + i;
+        if (a >= A) break;
+        const int e = idx[a];
+        if (e >= 0 && e < E)
+            atomicAdd(&h[e], 1);
+        else
+            set_error(MOE_ERR_BAD_ROUTING);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kDispThreads) hist[size_t(blockIdx.x) * E + e] = h[e];
+}
+
+// One CTA.  base[b][e] = number of expert-e assignments in chunks before b.
+__global__ void __launch_bounds__(kDispThreads)
+dispatch_scan_kernel(const int32_t* __restrict__ hist, int nblk, int E, int capacity,
+                     int32_t* __restrict__ base, int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+    __shared__ int kept[MOE_MAX_EXPERTS];
+    for (int e = threadIdx.x; e < E; e += kDispThreads) {
+        int run = 0;
+        for (int b = 0; b < nblk; ++b) {
+            base[size_t(b) * E + e] = run;
+            run += hist[size_t(b) * E + e];
+        }
+        if (counts != nullptr) counts[e] = run;
+        kept[e] = capacity < 0 ? run : min(run, capacity);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        // exclusive scan of kept over experts: lane l owns experts 8l .. 8l+7
+        const int lane = threadIdx.x;
+        int local[MOE_MAX_EXPERTS / 32];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < MOE_MAX_EXPERTS / 32; ++i) {
+            const int e = lane * (MOE_MAX_EXPERTS / 32) + i;
+            local[i] = e < E ? kept[e] : 0;
+            sum += local[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < MOE_MAX_EXPERTS / 32; ++i) {
+            const int e = lane * (MOE_MAX_EXPERTS / 32) + i;
+            if (e < E) offsets[e] = run;
+            run += local[i];
+        }
+        if (lane == 31) offsets[E] = incl;
+    }
+}
+
+__global__ void __launch_bounds__(kDispThreads)
+dispatch_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, int A, int E,
+                        const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
+                        int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, uint8_t* __restrict__ drop_mask,
+                        float* __restrict__ row_gate) {
+    __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
+    __shared__ int off_s[MOE_MAX_EXPERTS + 1];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < kDispWarps * MOE_MAX_EXPERTS; i += kDispThreads) (&wcnt[0][0])[i] = 0;
+    for (int e = tid; e <= E; e += kDispThreads) off_s[e] = offsets[e];
+    __syncthreads();
+
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int a_warp = blockIdx.x * kDispChunk + warp * kDispPerWarp;
+    constexpr int kRounds = kDispPerWarp / 32;
+    int ex[kRounds], rank[kRounds];
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+        const int a = a_warp + r * 32 + lane;
+        int e = (a < A) ? idx[a] : -1;
+        if (e >= E) e = -1;
+        if (e < -1) e = -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        const int local = __popc(peers & lt_mask);
+        rank[r] = (e >= 0) ? wcnt[warp][e] + local : 0;
+        __syncwarp();
+        if (e >= 0 && (peers & lt_mask) == 0) wcnt[warp][e] += __popc(peers);
+        __syncwarp();
+        ex[r] = e;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kDispThreads) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < kDispWarps; ++w) {
+            const int c = wcnt[w][e];
+            wcnt[w][e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+        const int a = a_warp + r * 32 + lane;
+        if (a >= A) continue;
+        const int e = ex[r];
+        int slot = -1;
+        if (e >= 0) {
+            const int g = base[size_t(blockIdx.x) * E + e] + wcnt[warp][e] + rank[r];
+            if (g < off_s[e + 1] - off_s[e]) slot = off_s[e] + g;
+        }
+        slot_of[a] = slot;
+        if (drop_mask != nullptr) drop_mask[a] = slot < 0 ? 1 : 0;
+        if (slot >= 0) {
+            perm[slot] = a;
+            if (row_gate != nullptr) row_gate[slot] = gate[a];
+        }
+    }
+}
+
+// xp[row, :] = x[perm[row] / k, :] for row < offsets[E]; row_bytes % 16 == 0
+__global__ void __launch_bounds__(256)
+dispatch_gather_kernel(const uint8_t* __restrict__ x, int row_bytes, const int32_t* __restrict__ perm,
+                       const int32_t* __restrict__ offsets, int E, int k, uint8_t* __restrict__ xp) {
+    const int R = offsets[E];
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int vecs = row_bytes >> 4;
+    for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < R; row += warps_total) {
+        const int t = perm[row] / k;
+        const uint4* src = reinterpret_cast<const uint4*>(x + size_t(t) * row_bytes);
+        uint4* dst = reinterpret_cast<uint4*>(xp + size_t(row) * row_bytes);
+        for (int i = lane; i < vecs; i += 32) dst[i] = __ldg(src + i);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Step 4: combine.  out[t] = sum over kept slots j (in slot order) of
+// w_tj * yp[slot_of[t*k+j]]; w_tj = gate or 1.  fp32 accumulation.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+    v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+}
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+    uint4 u;
+    u.x = pack_bf16x2(v[0], v[1]); u.y = pack_bf16x2(v[2], v[3]);
+    u.z = pack_bf16x2(v[4], v[5]); u.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = u;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
+               int Tn, int k, int d, T* __restrict__ out) {
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int chunks = d >> 3;
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < Tn; t += warps_total) {
+        int slot[MOE_MAX_TOPK];
+        float w[MOE_MAX_TOPK];
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+            slot[j] = (j < k) ? slot_of[size_t(t) * k + j] : -1;
+            w[j] = (j < k && gate != nullptr) ? gate[size_t(t) * k + j] : 1.f;
+        }
+        for (int c = lane; c < chunks; c += 32) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+                if (slot[j] < 0) continue;
+                float v[8];
+                load8(yp + size_t(slot[j]) * d + c * 8, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], v[i], acc[i]);
+            }
+            store8(out + size_t(t) * d + c * 8, acc);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// statistics (one CTA)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+stats_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
+             const float* __restrict__ prob_sum, int T, int k, int E, moe_stats* __restrict__ st) {
+    __shared__ float s_fp[256];
+    __shared__ int s_max[256];
+    float fp = 0.f;
+    int mx = 0;
+    const float invT = 1.0f / float(T);
+    for (int e = threadIdx.x; e < E; e += 256) {
+        fp += (float(counts[e]) * invT) * (prob_sum[e] * invT);
+        mx = max(mx, counts[e]);
+    }
+    s_fp[threadIdx.x] = fp;
+    s_max[threadIdx.x] = mx;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (threadIdx.x < o) {
+            s_fp[threadIdx.x] += s_fp[threadIdx.x + o];
+            s_max[threadIdx.x] = max(s_max[threadIdx.x], s_max[threadIdx.x + o]);
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const int A = T * k;
+        const int R = offsets[E];
+        st->aux_loss = float(E) * s_fp[0];
+        st->imbalance = float(s_max[0]) / (float(A) / float(E));
+        st->drop_rate = float(A - R) / float(A);
+        st->rows_kept = R;
+        st->max_count = s_max[0];
+        st->dropped = A - R;
+    }
+}
+
+}  // namespace moe

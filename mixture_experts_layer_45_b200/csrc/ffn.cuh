@@ -1,0 +1,393 @@
+// Step 3 of the layer: the grouped expert FFN (cookbook notebook "Mixture-
+// of-experts and expert parallelism", section "Dispatch and gather": each
+// expert is fc2(gelu(fc1(x))) on the tokens routed to it).
+//
+// Both GEMMs of an expert are C[M_e, N] = A[M_e, K] * W_e[N, K]^T with the
+// operands K-contiguous: fc1 has A = xp (K = d), W = W1_e (N = ff) and the
+// epilogue h = gelu(C + b1_e); fc2 has A = h (K = ff), W = W2_e (N = d) and
+// the epilogue y = g_row * (C + b2_e).
+//
+// The expert row ranges live only on the device (offsets), so every CTA
+// builds the same tile table from them and walks tiles t = blockIdx.x,
+// blockIdx.x + gridDim.x, ... (persistent grid, no host synchronisation).
+// Tile order: expert-major, then N tile, then M tile fastest, so CTAs that
+// run together share the same weight panel through L2.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+enum FfnMode { kFc1Gelu = 0, kFc2Gate = 1 };
+
+struct TileTable {
+    int start[MOE_MAX_EXPERTS + 1];   // first tile of each expert; start[E] = total
+    int mtiles[MOE_MAX_EXPERTS];      // M tiles of each expert
+    int off[MOE_MAX_EXPERTS + 1];     // row offsets (copy of `offsets`)
+};
+
+// Must be called by all threads of the CTA; ends with __syncthreads().
+__device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ offsets, int E, int BM, int ntiles_n,
+                                                 TileTable& tt) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) tt.off[e] = offsets[e];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        constexpr int PER = MOE_MAX_EXPERTS / 32;
+        int tl[PER];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            int mt = 0;
+            if (e < E) {
+                mt = (tt.off[e + 1] - tt.off[e] + BM - 1) / BM;
+                tt.mtiles[e] = mt;
+            }
+            tl[i] = mt * ntiles_n;
+            sum += tl[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            if (e < E) tt.start[e] = run;
+            run += tl[i];
+        }
+        if (lane == 31) tt.start[E] = incl;
+    }
+    __syncthreads();
+}
+
+struct TileCoord {
+    int e, mt, nt;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const TileTable& tt, int E, int t) {
+    int lo = 0, hi = E - 1;   // last e with start[e] <= t (experts with no tiles are skipped)
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tt.start[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    // experts without tiles have start[e] == start[e+1], so the last e with
+    // start[e] <= t is the one whose range [start[e], start[e+1]) holds t
+    TileCoord c;
+    c.e = lo;
+    const int local = t - tt.start[lo];
+    const int mt = tt.mtiles[lo];
+    c.nt = local / mt;
+    c.mt = local - c.nt * mt;
+    return c;
+}
+
+// ===========================================================================
+// fp32 path: SIMT FMA, 128 x 128 tiles, 8 x 8 outputs per thread
+// ===========================================================================
+constexpr int kSgBM = 128, kSgBN = 128, kSgBK = 8, kSgThreads = 256;
+constexpr int kSgLd = kSgBM + 4;
+
+template <int MODE>
+__global__ void __launch_bounds__(kSgThreads)
+ffn_simt_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ offsets, int E, int N, int K,
+                    const float* __restrict__ W, const float* __restrict__ bias, const float* __restrict__ row_gate,
+                    float* __restrict__ C) {
+    __shared__ TileTable tt;
+    __shared__ __align__(16) float As[2][kSgBK][kSgLd];
+    __shared__ __align__(16) float Bs[2][kSgBK][kSgLd];
+    const int ntn = (N + kSgBN - 1) / kSgBN;
+    build_tile_table(offsets, E, kSgBM, ntn, tt);
+    const int total = tt.start[E];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int lrow = tid >> 1, lk = (tid & 1) * 4;   // loader: one float4 of A and of W per thread
+
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        const TileCoord tc = decode_tile(tt, E, t);
+        const int rows = tt.off[tc.e + 1] - tt.off[tc.e];
+        const int m0 = tc.mt * kSgBM, n0 = tc.nt * kSgBN;
+        const float* Ab = A + size_t(tt.off[tc.e]) * K;
+        const float* Wb = W + size_t(tc.e) * N * K;
+
+        float acc[8][8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+        auto load_regs = [&](int k0, float4& ra, float4& rb) {
+            ra = make_float4(0.f, 0.f, 0.f, 0.f);
+            rb = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int kk = k0 + lk;
+            if (m0 + lrow < rows && kk < K) ra = *reinterpret_cast<const float4*>(Ab + size_t(m0 + lrow) * K + kk);
+            if (n0 + lrow < N && kk < K) rb = *reinterpret_cast<const float4*>(Wb + size_t(n0 + lrow) * K + kk);
+        };
+        auto store_smem = [&](int buf, const float4& ra, const float4& rb) {
+            As[buf][lk + 0][lrow] = ra.x; As[buf][lk + 1][lrow] = ra.y;
+            As[buf][lk + 2][lrow] = ra.z; As[buf][lk + 3][lrow] = ra.w;
+            Bs[buf][lk + 0][lrow] = rb.x; Bs[buf][lk + 1][lrow] = rb.y;
+            Bs[buf][lk + 2][lrow] = rb.z; Bs[buf][lk + 3][lrow] = rb.w;
+        };
+
+        float4 ra, rb;
+        load_regs(0, ra, rb);
+        __syncthreads();   // previous tile's readers are done with the buffers
+        store_smem(0, ra, rb);
+        __syncthreads();
+        int buf = 0;
+        for (int k0 = 0; k0 < K; k0 += kSgBK) {
+            const bool more = k0 + kSgBK < K;
+            if (more) load_regs(k0 + kSgBK, ra, rb);
+#pragma unroll
+            for (int kk = 0; kk < kSgBK; ++kk) {
+                const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+                const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+                const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+                const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+                const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+            }
+            if (more) {
+                store_smem(buf ^ 1, ra, rb);
+                __syncthreads();
+                buf ^= 1;
+            }
+        }
+
+        // epilogue
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+            if (r >= rows) continue;
+            const size_t grow = size_t(tt.off[tc.e]) + r;
+            const float g = (MODE == kFc2Gate && row_gate != nullptr) ? row_gate[grow] : 1.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int n = n0 + h * 64 + tx * 4;
+                if (n >= N) continue;
+                float v[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float c = acc[i][h * 4 + j] + bias[size_t(tc.e) * N + n + j];
+                    v[j] = (MODE == kFc1Gelu) ? gelu_erf(c) : g * c;
+                }
+                *reinterpret_cast<float4*>(C + grow * N + n) = make_float4(v[0], v[1], v[2], v[3]);
+            }
+        }
+    }
+}
+
+// ===========================================================================
+// bf16 path: tcgen05.mma (kind::f16) with fp32 accumulators in tensor
+// memory, operands brought to shared memory by TMA (128B swizzle).
+//
+// Warp roles (192 threads):
+//   warp 0        TMA producer (one thread)
+//   warp 1        tensor-memory allocator and MMA issuer (one thread)
+//   warps 2..5    epilogue: tcgen05.ld of their 32-lane quarter, bias,
+//                 GELU or gate, bf16 stores (row-masked to the expert)
+// Pipelines: STAGES shared-memory stages (full/empty mbarriers) and two
+// accumulators of BN columns each (tfull/tempty mbarriers), so the
+// epilogue of one tile overlaps the main loop of the next.
+// ===========================================================================
+constexpr int kTcBM = 128;
+constexpr int kTcBK = 64;            // 64 bf16 = 128 B = one swizzle row
+constexpr int kTcThreads = 192;
+
+template <int BN, int STAGES>
+struct TcCfg {
+    static constexpr uint32_t kABytes = kTcBM * kTcBK * 2;
+    static constexpr uint32_t kBBytes = BN * kTcBK * 2;
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+    static constexpr uint32_t kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                         : (2 * BN <= 256) ? 256 : 512;
+    static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;   // + alignment slack
+};
+
+template <int BN, int STAGES, int MODE>
+__global__ void __launch_bounds__(kTcThreads, 1)
+ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const int32_t* __restrict__ offsets, int E, int N, int K,
+                   const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
+                   __nv_bfloat16* __restrict__ C) {
+    using Cfg = TcCfg<BN, STAGES>;
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+    __shared__ TileTable tt;
+    __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull_bar[a], 1);
+            mbar_init(&tempty_bar[a], 4);   // one arrival per epilogue warp
+        }
+        mbar_init(&drain_bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    const int ntn = (N + BN - 1) / BN;
+    build_tile_table(offsets, E, kTcBM, ntn, tt);   // contains __syncthreads()
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+    const int total = tt.start[E];
+    const int KB = (K + kTcBK - 1) / kTcBK;
+    volatile int* abort_p = &abort_flag;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            int stage = 0;
+            uint32_t phase = 0;
+            int last_parity[STAGES];
+            for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const TileCoord tc = decode_tile(tt, E, t);
+                const int row0 = tt.off[tc.e] + tc.mt * kTcBM;
+                const int n0 = tc.nt * BN;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) { ok = false; break; }
+                    uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
+                    uint8_t* sb = sa + Cfg::kABytes;
+                    mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
+                    tma_load_2d(sa, &tmA, &full_bar[stage], kb * kTcBK, row0);
+                    tma_load_3d(sb, &tmB, &full_bar[stage], kb * kTcBK, n0, tc.e);
+                    last_parity[stage] = int(phase);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            {
+                // every load this thread issued lands before the CTA exits
+                // (immediate on the normal path, where the MMA consumed them)
+                for (int s = 0; s < STAGES; ++s) {
+                    if (last_parity[s] < 0) continue;
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(&full_bar[s], uint32_t(last_parity[s])) &&
+                           globaltimer_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            constexpr uint32_t idesc = idesc_bf16_f32(kTcBM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_p)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, abort_p)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
+                    const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sa));
+                    const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sa + Cfg::kABytes));
+#pragma unroll
+                    for (int kk = 0; kk < kTcBK / 16; ++kk)
+                        umma_f16(d_tmem, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc,
+                                 (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&empty_bar[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit(&tfull_bar[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            // every MMA this thread issued completes before TMEM is released
+            umma_commit(&drain_bar);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            const TileCoord tc = decode_tile(tt, E, t);
+            const int rows = tt.off[tc.e + 1] - tt.off[tc.e];
+            const int r_in = tc.mt * kTcBM + q * 32 + lane;
+            const bool valid = r_in < rows;
+            const size_t grow = size_t(tt.off[tc.e]) + r_in;
+            const int n0 = tc.nt * BN;
+            float g = 1.f;
+            if (MODE == kFc2Gate && row_gate != nullptr && valid) g = row_gate[grow];
+            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_p)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
+                tmem_ld_wait();
+                const int nb = n0 + c * 32;
+                if (!valid || nb >= N) continue;
+                const __nv_bfloat16* bp = bias + size_t(tc.e) * N + nb;
+                __nv_bfloat16* cp = C + grow * N + nb;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    if (nb + v * 8 >= N) break;
+                    const uint4 bb = *reinterpret_cast<const uint4*>(bp + v * 8);
+                    const float bf[8] = {bf16_lo(bb.x), bf16_hi(bb.x), bf16_lo(bb.y), bf16_hi(bb.y),
+                                         bf16_lo(bb.z), bf16_hi(bb.z), bf16_lo(bb.w), bf16_hi(bb.w)};
+                    float o[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float cval = __uint_as_float(r[v * 8 + i]) + bf[i];
+                        o[i] = (MODE == kFc1Gelu) ? gelu_erf(cval) : g * cval;
+                    }
+                    uint4 u;
+                    u.x = pack_bf16x2(o[0], o[1]);
+                    u.y = pack_bf16x2(o[2], o[3]);
+                    u.z = pack_bf16x2(o[4], o[5]);
+                    u.w = pack_bf16x2(o[6], o[7]);
+                    *reinterpret_cast<uint4*>(cp + v * 8) = u;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    }
+}
+
+}  // namespace moe

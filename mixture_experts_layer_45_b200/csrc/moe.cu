@@ -1,0 +1,551 @@
+// libmoe: host side of the C ABI declared in include/moe.h.
+//
+// Every entry point validates its arguments before touching the GPU, then
+// enqueues kernels on the caller's stream.  Nothing here synchronises the
+// host except moe_get_error and moe_timing_read, and nothing allocates
+// device memory: scratch comes from the caller's workspace.
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "ffn.cuh"
+#include "router.cuh"
+
+using namespace moe;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// launch counter and optional per-kernel event timing
+// ---------------------------------------------------------------------------
+std::atomic<uint64_t> g_launches{0};
+
+struct TimedLaunch {
+    int kernel;
+    cudaEvent_t start, stop;
+};
+
+struct TimingState {
+    std::mutex mu;
+    bool enabled = false;
+    std::vector<cudaEvent_t> free_events;
+    std::vector<TimedLaunch> pending;
+    double ms[MOE_NUM_KERNELS] = {};
+    int64_t launches[MOE_NUM_KERNELS] = {};
+};
+TimingState g_timing;
+
+constexpr int kEventPool = 4096;
+
+// caller holds g_timing.mu
+void harvest_locked(size_t upto) {
+    for (size_t i = 0; i < upto && i < g_timing.pending.size(); ++i) {
+        TimedLaunch& t = g_timing.pending[i];
+        float ms = 0.f;
+        if (cudaEventSynchronize(t.stop) == cudaSuccess && cudaEventElapsedTime(&ms, t.start, t.stop) == cudaSuccess) {
+            g_timing.ms[t.kernel] += ms;
+            g_timing.launches[t.kernel] += 1;
+        }
+        g_timing.free_events.push_back(t.start);
+        g_timing.free_events.push_back(t.stop);
+    }
+    g_timing.pending.erase(g_timing.pending.begin(),
+                           g_timing.pending.begin() + std::min(upto, g_timing.pending.size()));
+}
+
+cudaEvent_t take_event_locked() {
+    if (g_timing.free_events.empty()) harvest_locked(g_timing.pending.size() / 2 + 1);
+    if (g_timing.free_events.empty()) return nullptr;
+    cudaEvent_t e = g_timing.free_events.back();
+    g_timing.free_events.pop_back();
+    return e;
+}
+
+// Brackets one kernel launch: records the start event (when timing is on)
+// and, in finish(), checks the launch, counts it and records the stop event.
+class Launch {
+  public:
+    Launch(int kernel, cudaStream_t s) : kernel_(kernel), stream_(s) {
+        if (g_timing.enabled) {
+            std::lock_guard<std::mutex> lk(g_timing.mu);
+            start_ = take_event_locked();
+            if (start_ != nullptr) cudaEventRecord(start_, stream_);
+        }
+    }
+    int finish() {
+        const cudaError_t err = cudaGetLastError();
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if (start_ != nullptr) {
+            std::lock_guard<std::mutex> lk(g_timing.mu);
+            cudaEvent_t stop = take_event_locked();
+            if (stop != nullptr) {
+                cudaEventRecord(stop, stream_);
+                g_timing.pending.push_back({kernel_, start_, stop});
+            } else {
+                g_timing.free_events.push_back(start_);
+            }
+        }
+        if (err != cudaSuccess) {
+            std::fprintf(stderr, "libmoe: kernel %d launch failed: %s\n", kernel_, cudaGetErrorString(err));
+            return MOE_ERR_CUDA;
+        }
+        return MOE_OK;
+    }
+
+  private:
+    int kernel_;
+    cudaStream_t stream_;
+    cudaEvent_t start_ = nullptr;
+};
+
+// ---------------------------------------------------------------------------
+// helpers
+// ---------------------------------------------------------------------------
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline size_t elem_bytes(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+inline int ceil_div(long long a, long long b) { return int((a + b - 1) / b); }
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+// shared size checks: returns MOE_OK or an error code
+int check_sizes(int T, int d, int ff, int E, int k, int dtype, bool need_ff) {
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || (need_ff && ff <= 0)) return MOE_ERR_INVALID_ARG;
+    if (k > E) return MOE_ERR_INVALID_ARG;
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (d % 8 != 0 || (need_ff && ff % 8 != 0)) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+struct WsLayout {
+    size_t idx, gate, psum, counts, offsets, perm, slot_of, drop, row_gate, hist, base, xp, h, yp, total;
+};
+
+size_t dispatch_ws_bytes(int A, int E) {
+    const int nblk = std::max(1, ceil_div(A, kDispChunk));
+    return 2 * align256(size_t(nblk) * E * sizeof(int32_t));
+}
+
+WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype) {
+    WsLayout L{};
+    const size_t A = size_t(T) * k, es = elem_bytes(dtype);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t r = o;
+        o += align256(std::max<size_t>(bytes, 1));
+        return r;
+    };
+    L.idx = take(A * 4);
+    L.gate = take(A * 4);
+    L.psum = take(size_t(E) * 4);
+    L.counts = take(size_t(E) * 4);
+    L.offsets = take(size_t(E + 1) * 4);
+    L.perm = take(A * 4);
+    L.slot_of = take(A * 4);
+    L.drop = take(A);
+    L.row_gate = take(A * 4);
+    L.hist = take(dispatch_ws_bytes(int(A), E));
+    L.base = L.hist + dispatch_ws_bytes(int(A), E) / 2;
+    L.xp = take(A * d * es);
+    L.h = take(A * ff * es);
+    L.yp = take(A * d * es);
+    L.total = o;
+    return L;
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime, so the
+// library does not link libcuda directly)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// bf16 [rows, cols] row-major, box {64, box_rows}, 128B swizzle
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {uint32_t(kTcBK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [E, rows, cols], box {64, box_rows, 1}, 128B swizzle
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[3] = {cols, rows, E};
+    const cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+    const cuuint32_t box[3] = {uint32_t(kTcBK), box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename K>
+bool set_smem_attr(K kernel, size_t bytes) {
+    // cudaFuncSetAttribute is cheap and idempotent; it is per device, so set it every call
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) == cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// step launchers (arguments already validated)
+// ---------------------------------------------------------------------------
+template <typename Tin, int EP>
+int launch_router_ep(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
+                     float* gate, float* psum, cudaStream_t s) {
+    auto kern = router_topk_kernel<Tin, EP>;
+    const size_t smem = router_smem_bytes<EP>();
+    if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
+    Launch L(MOE_KERNEL_ROUTER, s);
+    kern<<<ceil_div(T, kRouterTM), kRouterThreads, smem, s>>>(static_cast<const Tin*>(x), static_cast<const Tin*>(wr),
+                                                              bias, T, d, E, k, idx, gate, psum);
+    return L.finish();
+}
+
+template <typename Tin>
+int launch_router_t(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
+                    float* gate, float* psum, cudaStream_t s) {
+    if (E <= 16) return launch_router_ep<Tin, 16>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+    if (E <= 32) return launch_router_ep<Tin, 32>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+    if (E <= 64) return launch_router_ep<Tin, 64>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+    if (E <= 128) return launch_router_ep<Tin, 128>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+    return launch_router_ep<Tin, 256>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+}
+
+int run_router(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int dtype,
+               int32_t* idx, float* gate, float* psum, cudaStream_t s) {
+    if (psum != nullptr && cudaMemsetAsync(psum, 0, size_t(E) * sizeof(float), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (dtype == MOE_BF16) return launch_router_t<__nv_bfloat16>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+    return launch_router_t<float>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+}
+
+int run_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int capacity, int32_t* counts,
+                 int32_t* offsets, int32_t* perm, int32_t* slot_of, uint8_t* drop, float* row_gate, const void* x,
+                 void* xp, int d, int dtype, void* ws, cudaStream_t s) {
+    const int A = T * k;
+    const int nblk = ceil_div(A, kDispChunk);
+    int32_t* hist = static_cast<int32_t*>(ws);
+    int32_t* base = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + dispatch_ws_bytes(A, E) / 2);
+    int rc;
+    {
+        Launch L(MOE_KERNEL_COUNT, s);
+        dispatch_count_kernel<<<nblk, kDispThreads, 0, s>>>(idx, A, E, hist);
+        if ((rc = L.finish()) != MOE_OK) return rc;
+    }
+    {
+        Launch L(MOE_KERNEL_SCAN, s);
+        dispatch_scan_kernel<<<1, kDispThreads, 0, s>>>(hist, nblk, E, capacity, base, counts, offsets);
+        if ((rc = L.finish()) != MOE_OK) return rc;
+    }
+    {
+        Launch L(MOE_KERNEL_PERMUTE, s);
+        dispatch_permute_kernel<<<nblk, kDispThreads, 0, s>>>(idx, gate, A, E, base, offsets, perm, slot_of, drop,
+                                                               row_gate);
+        if ((rc = L.finish()) != MOE_OK) return rc;
+    }
+    if (x != nullptr && xp != nullptr) {
+        const int row_bytes = int(size_t(d) * elem_bytes(dtype));
+        const int grid = std::max(1, std::min(ceil_div(A, 8), num_sms() * 8));
+        Launch L(MOE_KERNEL_GATHER, s);
+        dispatch_gather_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(x), row_bytes, perm, offsets, E, k,
+                                                    static_cast<uint8_t*>(xp));
+        if ((rc = L.finish()) != MOE_OK) return rc;
+    }
+    return MOE_OK;
+}
+
+// tile shapes of the bf16 tensor-core GEMMs
+constexpr int kFc1BN = 256, kFc1Stages = 4;
+constexpr int kFc2BN = 128, kFc2Stages = 6;
+
+template <int BN, int STAGES, int MODE>
+int launch_tc(const void* a, int a_cols, int max_rows, const void* w, int N, int E, const int32_t* offsets,
+              const void* bias, const float* row_gate, void* c, int kernel_id, cudaStream_t s) {
+    CUtensorMap tmA, tmB;
+    if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(max_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
+    if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), BN)) return MOE_ERR_UNSUPPORTED;
+    auto kern = ffn_tc_bf16_kernel<BN, STAGES, MODE>;
+    const size_t smem = TcCfg<BN, STAGES>::kSmemBytes;
+    if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
+    const long long tiles_ub = (static_cast<long long>(ceil_div(max_rows, kTcBM)) + E) * ceil_div(N, BN);
+    const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
+    Launch L(kernel_id, s);
+    kern<<<grid, kTcThreads, smem, s>>>(tmA, tmB, offsets, E, N, a_cols, static_cast<const __nv_bfloat16*>(bias),
+                                        row_gate, static_cast<__nv_bfloat16*>(c));
+    return L.finish();
+}
+
+template <int MODE>
+int launch_simt(const void* a, int K, int max_rows, const void* w, int N, int E, const int32_t* offsets,
+                const void* bias, const float* row_gate, void* c, int kernel_id, cudaStream_t s) {
+    const long long tiles_ub = (static_cast<long long>(ceil_div(max_rows, kSgBM)) + E) * ceil_div(N, kSgBN);
+    const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, 2ll * num_sms())));
+    Launch L(kernel_id, s);
+    ffn_simt_f32_kernel<MODE><<<grid, kSgThreads, 0, s>>>(static_cast<const float*>(a), offsets, E, N, K,
+                                                          static_cast<const float*>(w),
+                                                          static_cast<const float*>(bias), row_gate,
+                                                          static_cast<float*>(c));
+    return L.finish();
+}
+
+int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
+            const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp, int dtype,
+            cudaStream_t s) {
+    int rc;
+    if (dtype == MOE_BF16) {
+        rc = launch_tc<kFc1BN, kFc1Stages, kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, h,
+                                                     MOE_KERNEL_FFN1, s);
+        if (rc != MOE_OK) return rc;
+        return launch_tc<kFc2BN, kFc2Stages, kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, yp,
+                                                       MOE_KERNEL_FFN2, s);
+    }
+    rc = launch_simt<kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, h, MOE_KERNEL_FFN1, s);
+    if (rc != MOE_OK) return rc;
+    return launch_simt<kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, yp, MOE_KERNEL_FFN2, s);
+}
+
+int run_combine(const void* yp, const int32_t* slot_of, const float* gate, int T, int k, int d, int dtype, void* out,
+                cudaStream_t s) {
+    const int grid = std::max(1, std::min(ceil_div(T, 8), num_sms() * 16));
+    Launch L(MOE_KERNEL_COMBINE, s);
+    if (dtype == MOE_BF16)
+        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(yp), slot_of, gate, T,
+                                                            k, d, static_cast<__nv_bfloat16*>(out));
+    else
+        combine_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(yp), slot_of, gate, T, k, d,
+                                                   static_cast<float*>(out));
+    return L.finish();
+}
+
+int run_stats(const int32_t* counts, const int32_t* offsets, const float* psum, int T, int k, int E, moe_stats* st,
+              cudaStream_t s) {
+    Launch L(MOE_KERNEL_STATS, s);
+    stats_kernel<<<1, 256, 0, s>>>(counts, offsets, psum, T, k, E, st);
+    return L.finish();
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported dtype, shape or size";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_BAD_ROUTING: return "expert index out of range";
+        case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int moe_version(void) { return 10000; }
+
+int moe_capacity(int T, int k, int E, double cf) {
+    if (T < 0 || k < 1 || E < 1) return -1;
+    if (!(cf > 0.0)) return -1;
+    const double c = double(T) * double(k) / double(E) * cf;
+    if (c >= 2147483647.0) return 2147483647;
+    return int(c);
+}
+
+size_t moe_workspace_size(int T, int d, int ff, int E, int k, int dtype) {
+    if (check_sizes(T, d, ff, E, k, dtype, true) != MOE_OK) return 0;
+    return ws_layout(T, d, ff, E, k, dtype).total;
+}
+
+size_t moe_dispatch_workspace_size(int T, int k, int E) {
+    if (T < 0 || k < 1 || E < 1 || E > MOE_MAX_EXPERTS || static_cast<long long>(T) * k >= (1ll << 31)) return 0;
+    return dispatch_ws_bytes(T * k, E);
+}
+
+int moe_router_topk(const void* x, const void* w_router, const float* logit_bias, int T, int d, int E, int k,
+                    int dtype, int32_t* topk_idx, float* topk_gate, float* prob_sum, void* stream) {
+    int rc = check_sizes(T, d, 8, E, k, dtype, false);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) {
+        if (prob_sum != nullptr &&
+            cudaMemsetAsync(prob_sum, 0, size_t(E) * 4, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!x || !w_router || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+    return run_router(x, w_router, logit_bias, T, d, E, k, dtype, topk_idx, topk_gate, prob_sum,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int moe_dispatch(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E, int capacity,
+                 int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of, uint8_t* drop_mask,
+                 float* row_gate, const void* x, void* xp, int d, int dtype, void* ws, size_t ws_bytes,
+                 void* stream) {
+    const bool want_rows = (x != nullptr || xp != nullptr);
+    if (want_rows) {
+        if (!x || !xp) return MOE_ERR_INVALID_ARG;
+        const int rc = check_sizes(T, d, 8, E, k, dtype, false);
+        if (rc != MOE_OK) return rc;
+        if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+    } else {
+        const int rc = check_sizes(T, 8, 8, E, k, MOE_F32, false);
+        if (rc != MOE_OK) return rc;
+    }
+    if (row_gate != nullptr && topk_gate == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // no assignments: counts = 0, offsets = 0
+        if (cudaMemsetAsync(counts, 0, size_t(E) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(offsets, 0, size_t(E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!topk_idx || !perm || !slot_of) return MOE_ERR_INVALID_ARG;
+    if (ws == nullptr || ws_bytes < dispatch_ws_bytes(T * k, E)) return MOE_ERR_WORKSPACE;
+    return run_dispatch(topk_idx, topk_gate, T, k, E, capacity, counts, offsets, perm, slot_of, drop_mask, row_gate,
+                        x, xp, d, dtype, ws, s);
+}
+
+int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
+                    const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp,
+                    int dtype, void* stream) {
+    const int rc = check_sizes(max_rows, d, ff, E, 1, dtype, true);
+    if (rc != MOE_OK) return rc;
+    if (max_rows == 0) return MOE_OK;
+    if (!xp || !offsets || !w1 || !b1 || !w2 || !b2 || !h || !yp) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(w1) || !aligned16(b1) || !aligned16(w2) || !aligned16(b2) || !aligned16(h) ||
+        !aligned16(yp))
+        return MOE_ERR_INVALID_ARG;
+    return run_ffn(xp, offsets, max_rows, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype,
+                   static_cast<cudaStream_t>(stream));
+}
+
+int moe_combine(const void* yp, const int32_t* slot_of, const float* topk_gate, int T, int k, int d, int dtype,
+                void* out, void* stream) {
+    const int rc = check_sizes(T, d, 8, k, k, dtype, false);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!yp || !slot_of || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(yp) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    return run_combine(yp, slot_of, topk_gate, T, k, d, dtype, out, static_cast<cudaStream_t>(stream));
+}
+
+int moe_layer_stats(const int32_t* counts, const int32_t* offsets, const float* prob_sum, int T, int k, int E,
+                    moe_stats* stats, void* stream) {
+    const int rc = check_sizes(T, 8, 8, E, k, MOE_F32, false);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_ERR_INVALID_ARG;   // the statistics divide by T
+    if (!counts || !offsets || !prob_sum || !stats) return MOE_ERR_INVALID_ARG;
+    return run_stats(counts, offsets, prob_sum, T, k, E, stats, static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward(const void* x, const void* w_router, const float* logit_bias, const void* w1, const void* b1,
+                const void* w2, const void* b2, int T, int d, int ff, int E, int k, int capacity, int dtype,
+                void* out, moe_stats* stats, int32_t* topk_idx_out, float* topk_gate_out, void* ws,
+                size_t ws_bytes, void* stream) {
+    int rc = check_sizes(T, d, ff, E, k, dtype, true);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!x || !w_router || !w1 || !b1 || !w2 || !b2 || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w1) || !aligned16(b1) || !aligned16(w2) ||
+        !aligned16(b2) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, ff, E, k, dtype);
+    if (ws == nullptr || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(w + L.idx);
+    float* gate = topk_gate_out ? topk_gate_out : reinterpret_cast<float*>(w + L.gate);
+    float* psum = stats ? reinterpret_cast<float*>(w + L.psum) : nullptr;
+    int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
+    int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+    int32_t* perm = reinterpret_cast<int32_t*>(w + L.perm);
+    int32_t* slot_of = reinterpret_cast<int32_t*>(w + L.slot_of);
+    float* row_gate = reinterpret_cast<float*>(w + L.row_gate);
+    void* xp = w + L.xp;
+    void* h = w + L.h;
+    void* yp = w + L.yp;
+    const int A = T * k;
+
+    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, idx, gate, psum, s)) != MOE_OK) return rc;
+    if ((rc = run_dispatch(idx, gate, T, k, E, capacity, counts, offsets, perm, slot_of, nullptr, row_gate, x, xp, d,
+                           dtype, w + L.hist, s)) != MOE_OK)
+        return rc;
+    if ((rc = run_ffn(xp, offsets, A, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype, s)) != MOE_OK) return rc;
+    if ((rc = run_combine(yp, slot_of, nullptr, T, k, d, dtype, out, s)) != MOE_OK) return rc;
+    if (stats != nullptr && (rc = run_stats(counts, offsets, psum, T, k, E, stats, s)) != MOE_OK) return rc;
+    return MOE_OK;
+}
+
+int moe_get_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    const int zero = 0;
+    if (v != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    return v;
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_timing_enable(int enable) {
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    if (enable) {
+        while (g_timing.free_events.size() + 2 * g_timing.pending.size() < size_t(kEventPool)) {
+            cudaEvent_t e;
+            if (cudaEventCreate(&e) != cudaSuccess) return MOE_ERR_CUDA;
+            g_timing.free_events.push_back(e);
+        }
+    }
+    g_timing.enabled = enable != 0;
+    return MOE_OK;
+}
+
+int moe_timing_read(double* ms_per_kernel, int64_t* launches_per_kernel) {
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    harvest_locked(g_timing.pending.size());
+    for (int i = 0; i < MOE_NUM_KERNELS; ++i) {
+        if (ms_per_kernel) ms_per_kernel[i] = g_timing.ms[i];
+        if (launches_per_kernel) launches_per_kernel[i] = g_timing.launches[i];
+        g_timing.ms[i] = 0.0;
+        g_timing.launches[i] = 0;
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+"""User-facing wrapper around ``moe_forward``: device parameters, a cached
+workspace, and an end-to-end call from pinned host memory.
+
+PyTorch provides device memory and streams only; the layer's arithmetic runs
+in libmoe's CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import _lib
+
+TORCH_DTYPE = {_lib.MOE_F32: torch.float32, _lib.MOE_BF16: torch.bfloat16}
+
+
+def dtype_code(name_or_torch) -> int:
+    if name_or_torch in ("f32", torch.float32):
+        return _lib.MOE_F32
+    if name_or_torch in ("bf16", torch.bfloat16):
+        return _lib.MOE_BF16
+    raise ValueError(f"unsupported dtype {name_or_torch!r}")
+
+
+def to_device(a: np.ndarray, dtype: int, device) -> torch.Tensor:
+    """Upload a float32 array (already bf16-representable for bf16) in `dtype`."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(device=device, dtype=TORCH_DTYPE[dtype])
+
+
+@dataclass
+class MoEParams:
+    w_router: torch.Tensor
+    logit_bias: Optional[torch.Tensor]
+    w1: torch.Tensor
+    b1: torch.Tensor
+    w2: torch.Tensor
+    b2: torch.Tensor
+    dtype: int
+
+    @property
+    def E(self):
+        return self.w1.shape[0]
+
+    @property
+    def ff(self):
+        return self.w1.shape[1]
+
+    @property
+    def d(self):
+        return self.w1.shape[2]
+
+    @classmethod
+    def from_arrays(cls, inputs: Dict[str, np.ndarray], dtype: int, device="cuda") -> "MoEParams":
+        bias = inputs.get("logit_bias")
+        return cls(
+            w_router=to_device(inputs["w_router"], dtype, device),
+            logit_bias=None if bias is None else torch.from_numpy(np.asarray(bias, np.float32)).to(device),
+            w1=to_device(inputs["w1"], dtype, device), b1=to_device(inputs["b1"], dtype, device),
+            w2=to_device(inputs["w2"], dtype, device), b2=to_device(inputs["b2"], dtype, device),
+            dtype=dtype)
+
+
+def read_stats(stats_buf: torch.Tensor) -> Dict[str, float]:
+    raw = stats_buf.cpu().numpy().tobytes()
+    s = _lib.MoeStats.from_buffer_copy(raw)
+    return {f: getattr(s, f) for f, _ in _lib.MoeStats._fields_}
+
+
+class MoELayer:
+    """One MoE layer bound to device parameters; reuses its workspace."""
+
+    def __init__(self, params: MoEParams, k: int, capacity: int = -1):
+        self.p = params
+        self.k = k
+        self.capacity = capacity
+        self._ws = None
+        self._ws_T = -1
+        self.stats_buf = torch.zeros(ctypes.sizeof(_lib.MoeStats), dtype=torch.uint8,
+                                     device=params.w1.device)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        if self._ws is None or self._ws_T < T:
+            n = _lib.moe_workspace_size(T, self.p.d, self.p.ff, self.p.E, self.k, self.p.dtype)
+            if n == 0:
+                raise ValueError("invalid layer sizes")
+            self._ws = torch.empty(n, dtype=torch.uint8, device=self.p.w1.device)
+            self._ws_T = T
+        return self._ws
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stats: bool = False,
+                topk_idx: Optional[torch.Tensor] = None, topk_gate: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+        if not x.is_cuda:
+            raise ValueError("x must be a CUDA tensor")
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty_like(x)
+        ws = self.workspace(T)
+        p = self.p
+        _lib.moe_forward(x, p.w_router, p.logit_bias, p.w1, p.b1, p.w2, p.b2, T, p.d, p.ff, p.E, self.k,
+                         self.capacity, p.dtype, out, self.stats_buf if stats else None, topk_idx, topk_gate,
+                         ws, ws.numel(), stream)
+        return out
+
+    __call__ = forward
+
+    def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, x_dev: torch.Tensor,
+                     out_dev: torch.Tensor, stream=None) -> torch.Tensor:
+        """End to end from (pinned) host memory: H2D copy, forward, D2H copy,
+        all enqueued on one stream; returns out_host once the copy is done."""
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            x_dev.copy_(x_host, non_blocking=True)
+            self.forward(x_dev, out=out_dev, stream=s)
+            out_host.copy_(out_dev, non_blocking=True)
+        s.synchronize()
+        return out_host

@@ -240,26 +240,17 @@ def moe_forward(x, params, topk_idx, topk_gate, slot_of=None) -> np.ndarray:
 
 
 def moe_forward_rows(x, params, topk_idx, topk_gate, slot_of, rows) -> np.ndarray:
-    """Output rows ``rows`` of moe_forward, computed token by token.
+    """Output rows ``rows`` of moe_forward.
 
-    The FFN acts on each token independently, so a sampled row equals the
-    corresponding row of the full forward; used for full-size parity checks.
+    The expert FFN acts on each token independently, so moe_forward applied
+    to the sampled tokens (with their routing and drop flags) gives exactly
+    those rows of the full output; used for full-size parity checks.
     """
     idx = np.asarray(topk_idx)
     T, k = idx.shape
-    keep = np.asarray(slot_of).reshape(T, k) >= 0
-    g = np.asarray(topk_gate, np.float64)
-    out = np.zeros((len(rows), x.shape[1]), np.float64)
-    for r, t in enumerate(rows):
-        xt = np.asarray(x[t:t + 1], np.float64)
-        for e in sorted(set(int(v) for v in idx[t])):
-            kept_js = [j for j in range(k) if idx[t, j] == e and keep[t, j]]
-            if not kept_js:
-                continue
-            w = sum(g[t, j] for j in kept_js)
-            out[r] += w * expert_ffn(xt, params["w1"][e], params["b1"][e],
-                                     params["w2"][e], params["b2"][e])[0]
-    return out
+    rows = np.asarray(rows)
+    sub_slot = np.asarray(slot_of).reshape(T, k)[rows].reshape(-1)
+    return moe_forward(np.asarray(x)[rows], params, idx[rows], np.asarray(topk_gate)[rows], sub_slot)
 
 
 def grouped_ffn(xp, offsets, params, row_gate=None) -> np.ndarray:

@@ -1,0 +1,129 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_45_b200 import _lib
+from mixture_experts_layer_45_b200 import build as build_mod
+from oracle import moe_ref
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return _lib.load()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_surface():
+    assert header_functions() == _lib.EXPORTED
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert _lib.moe_version() == 10000
+    for code in range(7):
+        assert _lib.status_string(code) not in ("", "unknown status")
+    assert _lib.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("T,k,E,cf", [(4096, 1, 32, 1.0), (4096, 1, 32, 1.5), (16384, 1, 64, 1.25),
+                                      (1024, 2, 8, 1.0), (10, 1, 3, 1.0), (7, 3, 5, 0.7), (100, 2, 7, 2.5),
+                                      (1024, 2, 8, None), (1024, 2, 8, 0.0), (1024, 2, 8, -1.0)])
+def test_capacity_matches_oracle(lib, T, k, E, cf):
+    assert _lib.moe_capacity(T, k, E, cf) == moe_ref.capacity(T, k, E, cf)
+
+
+def test_workspace_size(lib):
+    a = _lib.moe_workspace_size(4096, 768, 3072, 32, 1, _lib.MOE_BF16)
+    b = _lib.moe_workspace_size(4096, 768, 3072, 32, 1, _lib.MOE_F32)
+    assert a > 4096 * (768 * 2 + 3072) * 2 and b > a
+    assert _lib.moe_workspace_size(4096, 12, 3072, 32, 1, _lib.MOE_BF16) == 0     # d % 8
+    assert _lib.moe_workspace_size(4096, 768, 3072, 32, 33, _lib.MOE_BF16) == 0   # k > E
+    assert _lib.moe_workspace_size(4096, 768, 3072, 300, 1, _lib.MOE_BF16) == 0   # E too large
+    assert _lib.moe_dispatch_workspace_size(4096, 1, 32) > 0
+    assert _lib.moe_dispatch_workspace_size(-1, 1, 32) == 0
+
+
+FAKE = 1 << 20          # an aligned non-null address that is never dereferenced
+MISALIGNED = FAKE + 4
+
+
+def router(lib, **kw):
+    a = dict(x=FAKE, w=FAKE, bias=None, T=64, d=64, E=8, k=2, dtype=_lib.MOE_BF16, idx=FAKE, gate=FAKE, psum=None)
+    a.update(kw)
+    return lib.moe_router_topk(a["x"], a["w"], a["bias"], a["T"], a["d"], a["E"], a["k"], a["dtype"],
+                               a["idx"], a["gate"], a["psum"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=9), _lib.MOE_ERR_INVALID_ARG),            # k > E
+    (dict(E=300, k=2), _lib.MOE_ERR_UNSUPPORTED),      # E > 256
+    (dict(E=16, k=9), _lib.MOE_ERR_UNSUPPORTED),       # k > 8
+    (dict(dtype=7), _lib.MOE_ERR_UNSUPPORTED),
+    (dict(d=12), _lib.MOE_ERR_UNSUPPORTED),
+    (dict(T=-1), _lib.MOE_ERR_INVALID_ARG),
+    (dict(x=None), _lib.MOE_ERR_INVALID_ARG),
+    (dict(idx=None), _lib.MOE_ERR_INVALID_ARG),
+    (dict(x=MISALIGNED), _lib.MOE_ERR_INVALID_ARG),
+    (dict(T=1 << 30, k=2), _lib.MOE_ERR_UNSUPPORTED),  # T*k overflows int32
+])
+def test_router_rejects_bad_arguments(lib, kw, code):
+    assert router(lib, **kw) == code
+
+
+def forward(lib, ws_bytes, ws=FAKE, **kw):
+    a = dict(T=256, d=64, ff=128, E=8, k=2, cap=-1, dtype=_lib.MOE_BF16, out=FAKE)
+    a.update(kw)
+    return lib.moe_forward(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, a["T"], a["d"], a["ff"], a["E"], a["k"],
+                           a["cap"], a["dtype"], a["out"], None, None, None, ws, ws_bytes, None)
+
+
+def test_forward_checks_workspace(lib):
+    need = _lib.moe_workspace_size(256, 64, 128, 8, 2, _lib.MOE_BF16)
+    assert forward(lib, need - 1) == _lib.MOE_ERR_WORKSPACE
+    assert forward(lib, need, ws=None) == _lib.MOE_ERR_WORKSPACE
+    assert forward(lib, need, ws=FAKE + 16) == _lib.MOE_ERR_WORKSPACE      # not 256-byte aligned
+    assert forward(lib, need, out=None) == _lib.MOE_ERR_INVALID_ARG
+    assert forward(lib, need, ff=100) == _lib.MOE_ERR_UNSUPPORTED
+    assert forward(lib, 0, T=0) == _lib.MOE_OK                              # empty batch: nothing to do
+
+
+def test_dispatch_checks(lib):
+    ws_need = _lib.moe_dispatch_workspace_size(100, 2, 8)
+    call = lambda **kw: lib.moe_dispatch(
+        kw.get("idx", FAKE), kw.get("gate", None), 100, 2, 8, -1, FAKE, FAKE, FAKE, FAKE, None,
+        kw.get("row_gate", None), kw.get("x", None), kw.get("xp", None), 64, _lib.MOE_BF16,
+        kw.get("ws", FAKE), kw.get("ws_bytes", ws_need), None)
+    assert call(ws_bytes=ws_need - 1) == _lib.MOE_ERR_WORKSPACE
+    assert call(row_gate=FAKE) == _lib.MOE_ERR_INVALID_ARG          # row_gate needs topk_gate
+    assert call(x=FAKE) == _lib.MOE_ERR_INVALID_ARG                 # x without xp
+    assert call(idx=None) == _lib.MOE_ERR_INVALID_ARG
+
+
+def test_grouped_ffn_and_combine_checks(lib):
+    assert lib.moe_grouped_ffn(FAKE, FAKE, 64, 8, 64, 128, FAKE, FAKE, FAKE, MISALIGNED, None, FAKE, FAKE,
+                               _lib.MOE_BF16, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(FAKE, FAKE, None, 64, 9, 64, _lib.MOE_BF16, FAKE, None) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_combine(None, FAKE, None, 64, 2, 64, _lib.MOE_BF16, FAKE, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_stats(FAKE, FAKE, FAKE, 0, 1, 8, FAKE, None) == _lib.MOE_ERR_INVALID_ARG
+
+
+def test_no_launch_and_timing_read_without_gpu(lib):
+    assert _lib.moe_launch_count() == 0
+    assert lib.moe_timing_enable(0) == _lib.MOE_OK
+    t = _lib.moe_timing_read()
+    assert set(t) == set(_lib.KERNEL_NAMES) and all(v == (0.0, 0) for v in t.values())
