@@ -260,6 +260,24 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# multi-rank timing aggregation (replicas: no data-path collective)
+# ---------------------------------------------------------------------------
+def reduce_max_ms(ms: float, device=None) -> float:
+    """MAX of a per-rank device time over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, steps: int, tokens_per_step: int, max_ms: float) -> float:
+    """Tokens processed by all ranks divided by the slowest rank's time."""
+    return world * steps * tokens_per_step / (max_ms / 1000.0)
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 def algorithmic_bytes(kernel, w, R, E_active, es):
@@ -361,12 +379,8 @@ def run_ours(args):
     if err != 0:
         raise RuntimeError(f"device error in the timed region: {_lib.status_string(err)}")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    value = world * args.steps * w.T / (total_ms / 1000.0)
+    total_ms = reduce_max_ms(sum(step_ms), dev)
+    value = whole_job_tokens_per_s(world, args.steps, w.T, total_ms)
 
     # ---- end to end through the public API: pinned host in, pinned host out
     e2e_steps = args.e2e_steps or max(3, min(args.steps, 50))
@@ -390,12 +404,10 @@ def run_ours(args):
         out_host.copy_(out_dev2, non_blocking=True)
         e_ends[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    e2e_ms = reduce_max_ms(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), dev)
     if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_value = world * e2e_steps * w.T / (float(te.item()) / 1000.0)
+    e2e_value = whole_job_tokens_per_s(world, e2e_steps, w.T, e2e_ms)
     io_bytes = x.numel() * x.element_size()
 
     if rank != 0:

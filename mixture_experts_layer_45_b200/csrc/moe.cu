@@ -416,24 +416,18 @@ int moe_dispatch(const int32_t* topk_idx, const float* topk_gate, int T, int k, 
                  float* row_gate, const void* x, void* xp, int d, int dtype, void* ws, size_t ws_bytes,
                  void* stream) {
     const bool want_rows = (x != nullptr || xp != nullptr);
-    if (want_rows) {
-        if (!x || !xp) return MOE_ERR_INVALID_ARG;
-        const int rc = check_sizes(T, d, 8, E, k, dtype, false);
-        if (rc != MOE_OK) return rc;
-        if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
-    } else {
-        const int rc = check_sizes(T, 8, 8, E, k, MOE_F32, false);
-        if (rc != MOE_OK) return rc;
-    }
-    if (row_gate != nullptr && topk_gate == nullptr) return MOE_ERR_INVALID_ARG;
+    const int rc = want_rows ? check_sizes(T, d, 8, E, k, dtype, false) : check_sizes(T, 8, 8, E, k, MOE_F32, false);
+    if (rc != MOE_OK) return rc;
     if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0) {
-        // no assignments: counts = 0, offsets = 0
+        // no assignments: counts = 0, offsets = 0; the other pointers may be NULL
         if (cudaMemsetAsync(counts, 0, size_t(E) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaMemsetAsync(offsets, 0, size_t(E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_OK;
     }
+    if (want_rows && (!x || !xp || !aligned16(x) || !aligned16(xp))) return MOE_ERR_INVALID_ARG;
+    if (row_gate != nullptr && topk_gate == nullptr) return MOE_ERR_INVALID_ARG;
     if (!topk_idx || !perm || !slot_of) return MOE_ERR_INVALID_ARG;
     if (ws == nullptr || ws_bytes < dispatch_ws_bytes(T * k, E)) return MOE_ERR_WORKSPACE;
     return run_dispatch(topk_idx, topk_gate, T, k, E, capacity, counts, offsets, perm, slot_of, drop_mask, row_gate,
