@@ -152,6 +152,33 @@ MOE_API int moe_dispatch(const int32_t* topk_idx, const float* topk_gate,
                  const void* x, void* xp, int d, int dtype,
                  void* ws, size_t ws_bytes, void* stream);
 
+/* ---- dispatch without a workspace -------------------------------------
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory: for example a serving runtime whose
+ * allocator has reserved the whole device up front and hands out no extra
+ * buffers, or a latency-critical path that must not call cudaMalloc (which
+ * can synchronise the device) and has no workspace to pass.
+ *
+ * Same semantics, arguments and results as moe_dispatch, minus ws/ws_bytes.
+ * Its scratch is a fixed array inside the library (1 MiB per GPU, held by
+ * every GPU that loads the library until the process exits), so it
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * Limit: T*k <= MOE_NOALLOC_MAX_ASSIGNMENTS; larger calls return
+ * MOE_ERR_WORKSPACE (and print why to stderr) before launching anything.
+ * The first call on a device looks up the array's device address for that
+ * device (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  All calls share the one array and it
+ * keeps the last call's contents (every entry a call reads is written
+ * earlier in that call, so nothing needs clearing): calls whose executions
+ * overlap on the GPU, on different streams or host threads, race on it and
+ * must be serialised by the caller. */
+#define MOE_NOALLOC_MAX_ASSIGNMENTS (1 << 20)
+MOE_API int moe_dispatch_noalloc(const int32_t* topk_idx, const float* topk_gate,
+                                 int T, int k, int E, int capacity,
+                                 int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                                 uint8_t* drop_mask, float* row_gate,
+                                 const void* x, void* xp, int d, int dtype, void* stream);
+
 /* ---- step 3: grouped expert FFN (notebook section "Dispatch and gather")
  * For each expert e and each row r in offsets[e] .. offsets[e+1]-1:
  *   h[r,:]  = gelu(xp[r,:] W1_e^T + b1_e)          (exact erf GELU)

@@ -54,6 +54,7 @@ _SIGS = {
     "moe_router_topk": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P,
                           ctypes.c_size_t, _P]),
+    "moe_dispatch_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P]),
     "moe_grouped_ffn": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "moe_layer_stats": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
@@ -143,6 +144,18 @@ def moe_dispatch(topk_idx, topk_gate, T, k, E, capacity, counts, offsets, perm, 
                                _ptr(perm), _ptr(slot_of), _ptr(drop_mask), _ptr(row_gate), _ptr(x), _ptr(xp),
                                d, dtype, _ptr(ws), ws_bytes, _stream(stream)),
            "moe_dispatch")
+
+
+MOE_NOALLOC_MAX_ASSIGNMENTS = 1 << 20
+
+
+def moe_dispatch_noalloc(topk_idx, topk_gate, T, k, E, capacity, counts, offsets, perm, slot_of, drop_mask,
+                         row_gate, x, xp, d, dtype, stream=None):
+    """moe_dispatch with the library's fixed scratch instead of a workspace."""
+    _check(load().moe_dispatch_noalloc(_ptr(topk_idx), _ptr(topk_gate), T, k, E, capacity, _ptr(counts),
+                                       _ptr(offsets), _ptr(perm), _ptr(slot_of), _ptr(drop_mask), _ptr(row_gate),
+                                       _ptr(x), _ptr(xp), d, dtype, _stream(stream)),
+           "moe_dispatch_noalloc")
 
 
 def moe_grouped_ffn(xp, offsets, max_rows, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype, stream=None):

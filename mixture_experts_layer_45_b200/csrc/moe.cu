@@ -355,6 +355,38 @@ int run_stats(const int32_t* counts, const int32_t* offsets, const float* psum, 
     return L.finish();
 }
 
+// ---------------------------------------------------------------------------
+// Fixed device scratch for moe_dispatch_noalloc.  Sized for
+// MOE_NOALLOC_MAX_ASSIGNMENTS assignments and MOE_MAX_EXPERTS experts: the
+// per-chunk histograms and bases of the dispatch kernels (1 MiB).  Every GPU
+// that loads the library holds this array until the process exits.  In host
+// code `g_dispatch_scratch` is only a host-side stand-in for the symbol;
+// its device address comes from cudaGetSymbolAddress, once per device.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoallocScratchBytes =
+    2 * ((size_t(MOE_NOALLOC_MAX_ASSIGNMENTS) / kDispChunk) * MOE_MAX_EXPERTS * sizeof(int32_t));
+static __device__ __align__(256) uint8_t g_dispatch_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_dispatch_scratch on the current device (looked up on
+// the first call for that device, with that device current).
+int noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MOE_OK;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -432,6 +464,37 @@ int moe_dispatch(const int32_t* topk_idx, const float* topk_gate, int T, int k, 
     if (ws == nullptr || ws_bytes < dispatch_ws_bytes(T * k, E)) return MOE_ERR_WORKSPACE;
     return run_dispatch(topk_idx, topk_gate, T, k, E, capacity, counts, offsets, perm, slot_of, drop_mask, row_gate,
                         x, xp, d, dtype, ws, s);
+}
+
+int moe_dispatch_noalloc(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E, int capacity,
+                         int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of, uint8_t* drop_mask,
+                         float* row_gate, const void* x, void* xp, int d, int dtype, void* stream) {
+    const bool want_rows = (x != nullptr || xp != nullptr);
+    const int rc = want_rows ? check_sizes(T, d, 8, E, k, dtype, false) : check_sizes(T, 8, 8, E, k, MOE_F32, false);
+    if (rc != MOE_OK) return rc;
+    if (static_cast<long long>(T) * k > MOE_NOALLOC_MAX_ASSIGNMENTS) {
+        std::fprintf(stderr, "libmoe: moe_dispatch_noalloc: T*k = %lld exceeds the fixed scratch limit of %d "
+                             "assignments; use moe_dispatch with a workspace\n",
+                     static_cast<long long>(T) * k, MOE_NOALLOC_MAX_ASSIGNMENTS);
+        return MOE_ERR_WORKSPACE;
+    }
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (cudaMemsetAsync(counts, 0, size_t(E) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(offsets, 0, size_t(E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (want_rows && (!x || !xp || !aligned16(x) || !aligned16(xp))) return MOE_ERR_INVALID_ARG;
+    if (row_gate != nullptr && topk_gate == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!topk_idx || !perm || !slot_of) return MOE_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    const int src = noalloc_scratch(&scratch);
+    if (src != MOE_OK) return src;
+    // every histogram and base entry the kernels read is written earlier in
+    // the same call, so nothing in the scratch needs clearing
+    return run_dispatch(topk_idx, topk_gate, T, k, E, capacity, counts, offsets, perm, slot_of, drop_mask, row_gate,
+                        x, xp, d, dtype, scratch, s);
 }
 
 int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
