@@ -112,6 +112,25 @@ MOE_API size_t moe_workspace_size(int T, int d, int ff, int E, int k, int dtype)
 /* Bytes of scratch moe_dispatch needs (per-block expert histograms). */
 MOE_API size_t moe_dispatch_workspace_size(int T, int k, int E);
 
+/* Byte offset of one of moe_forward's intermediate arrays inside its
+ * workspace, for inspection and testing (the layout may change between
+ * versions; query it, do not hard-code it).  `which` is one of the
+ * MOE_WS_* values; returns (size_t)-1 for invalid arguments.  After
+ * moe_forward completes: topk_idx/topk_gate [T,k] (when the caller passed no
+ * output for them), counts [E], offsets [E+1], perm [R], slot_of [T*k],
+ * row_gate [R], xp [R,d], h [R,ff]; yp [R,d] only when k > 1. */
+#define MOE_WS_TOPK_IDX  0
+#define MOE_WS_TOPK_GATE 1
+#define MOE_WS_COUNTS    2
+#define MOE_WS_OFFSETS   3
+#define MOE_WS_PERM      4
+#define MOE_WS_SLOT_OF   5
+#define MOE_WS_ROW_GATE  6
+#define MOE_WS_XP        7
+#define MOE_WS_H         8
+#define MOE_WS_YP        9
+MOE_API size_t moe_workspace_offset(int T, int d, int ff, int E, int k, int dtype, int which);
+
 /* ---- step 1: router (notebook section "Top-k router") ------------------
  * logits[t,e] = sum_i x[t,i] w_router[e,i] (+ logit_bias[e]) accumulated in
  * fp32; g = softmax over e in fp32; the k experts with the largest logits,

@@ -51,6 +51,7 @@ _SIGS = {
     "moe_capacity": (_I, [_I, _I, _I, ctypes.c_double]),
     "moe_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "moe_dispatch_workspace_size": (ctypes.c_size_t, [_I, _I, _I]),
+    "moe_workspace_offset": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_router_topk": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P,
                           ctypes.c_size_t, _P]),
@@ -126,6 +127,15 @@ def moe_capacity(T: int, k: int, E: int, cf) -> int:
 
 def moe_workspace_size(T, d, ff, E, k, dtype) -> int:
     return load().moe_workspace_size(T, d, ff, E, k, dtype)
+
+
+WS_VIEWS = {"topk_idx": 0, "topk_gate": 1, "counts": 2, "offsets": 3, "perm": 4, "slot_of": 5, "row_gate": 6,
+            "xp": 7, "h": 8, "yp": 9}
+
+
+def moe_workspace_offset(T, d, ff, E, k, dtype, which) -> int:
+    code = WS_VIEWS[which] if isinstance(which, str) else which
+    return load().moe_workspace_offset(T, d, ff, E, k, dtype, code)
 
 
 def moe_dispatch_workspace_size(T, k, E) -> int:

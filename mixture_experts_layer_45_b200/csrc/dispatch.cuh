@@ -160,6 +160,185 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, int row_bytes, const int32
 }
 
 // ---------------------------------------------------------------------------
+// Dispatch inside moe_forward.  The router already wrote, per chunk of
+// chunk_tokens tokens (one router CTA), the expert histogram of its chunk
+// and its per-expert probability sums; a chunk holds the chunk_tokens * k
+// consecutive assignments of its tokens.
+//   forward_scan_kernel     one CTA: bases, counts, capacity, offsets and
+//                           the layer statistics
+//   forward_permute_kernel  grid (chunks, G): stable in-chunk ranks, the
+//                           dispatch arrays (y == 0 only), and the row
+//                           gather split over the G CTAs of the chunk; for
+//                           k == 1 with a direct output it also zero-fills the
+//                           output rows of dropped tokens
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024)
+forward_scan_kernel(const int32_t* __restrict__ hist, const float* __restrict__ psum_part, int nchunk, int E,
+                    int T, int k, int capacity, int32_t* __restrict__ base, int32_t* __restrict__ counts,
+                    int32_t* __restrict__ offsets, moe_stats* __restrict__ st) {
+    __shared__ int kept[MOE_MAX_EXPERTS];
+    __shared__ int cnt[MOE_MAX_EXPERTS];
+    __shared__ float fp[MOE_MAX_EXPERTS];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        float ps = 0.f;
+        for (int b = 0; b < nchunk; ++b) {
+            base[size_t(b) * E + e] = run;
+            run += hist[size_t(b) * E + e];
+            if (psum_part != nullptr) ps += psum_part[size_t(b) * E + e];
+        }
+        counts[e] = run;
+        cnt[e] = run;
+        kept[e] = capacity < 0 ? run : min(run, capacity);
+        fp[e] = (float(run) / float(T)) * (ps / float(T));
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        constexpr int PER = MOE_MAX_EXPERTS / 32;
+        int local[PER];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            local[i] = e < E ? kept[e] : 0;
+            sum += local[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            if (e < E) offsets[e] = run;
+            run += local[i];
+        }
+        if (lane == 31) offsets[E] = incl;
+        if (st != nullptr) {
+            // statistics, in a fixed summation order
+            float f = 0.f;
+            int mx = 0;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = lane * PER + i;
+                if (e < E) {
+                    f += fp[e];
+                    mx = max(mx, cnt[e]);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                f += __shfl_xor_sync(0xffffffffu, f, o);
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            if (lane == 31) {
+                const int A = T * k;
+                const int R = incl;
+                st->aux_loss = float(E) * f;
+                st->imbalance = float(mx) / (float(A) / float(E));
+                st->drop_rate = float(A - R) / float(A);
+                st->rows_kept = R;
+                st->max_count = mx;
+                st->dropped = A - R;
+            }
+        }
+    }
+}
+
+constexpr int kFwdThreads = 256;
+constexpr int kFwdMaxChunk = 1024;   // chunk_tokens * k
+
+__global__ void __launch_bounds__(kFwdThreads)
+forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, int T, int k, int E,
+                       int chunk_tokens, const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, float* __restrict__ row_gate,
+                       const uint8_t* __restrict__ x, int row_bytes, uint8_t* __restrict__ xp,
+                       uint8_t* __restrict__ out_zero_dropped) {
+    __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
+    __shared__ int off_s[MOE_MAX_EXPERTS + 1];
+    __shared__ int slot_s[kFwdMaxChunk];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int chunk = blockIdx.x;
+    const int A = T * k;
+    const int a0 = chunk * chunk_tokens * k;
+    const int na = min(chunk_tokens * k, A - a0);
+    for (int i = tid; i < kDispWarps * MOE_MAX_EXPERTS; i += kFwdThreads) (&wcnt[0][0])[i] = 0;
+    for (int e = tid; e <= E; e += kFwdThreads) off_s[e] = offsets[e];
+    __syncthreads();
+
+    // warp w ranks the contiguous assignments [w*per, (w+1)*per) of the chunk
+    const int per = ((na + kDispWarps - 1) / kDispWarps + 31) & ~31;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    constexpr int kMaxRounds = kFwdMaxChunk / kDispWarps / 32;   // 4
+    int ex[kMaxRounds], rank[kMaxRounds];
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+        const int i = warp * per + r * 32 + lane;
+        const bool in = (r * 32 < per) && i < na;
+        int e = in ? idx[a0 + i] : -1;
+        if (e >= E || e < -1) e = -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        const int local = __popc(peers & lt_mask);
+        rank[r] = (e >= 0) ? wcnt[warp][e] + local : 0;
+        __syncwarp();
+        if (e >= 0 && (peers & lt_mask) == 0) wcnt[warp][e] += __popc(peers);
+        __syncwarp();
+        ex[r] = e;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kFwdThreads) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < kDispWarps; ++w) {
+            const int c = wcnt[w][e];
+            wcnt[w][e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    const bool writer = blockIdx.y == 0;
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+        const int i = warp * per + r * 32 + lane;
+        if (!((r * 32 < per) && i < na)) continue;
+        const int a = a0 + i;
+        const int e = ex[r];
+        int slot = -1;
+        if (e >= 0) {
+            const int g = base[size_t(chunk) * E + e] + wcnt[warp][e] + rank[r];
+            if (g < off_s[e + 1] - off_s[e]) slot = off_s[e] + g;
+        }
+        slot_s[i] = slot;
+        if (writer) {
+            slot_of[a] = slot;
+            if (slot >= 0) {
+                perm[slot] = a;
+                if (row_gate != nullptr) row_gate[slot] = gate[a];
+            }
+        }
+    }
+    __syncthreads();
+    // rows of this chunk handled by this CTA: i = blockIdx.y, blockIdx.y + gridDim.y, ...
+    const int vecs = row_bytes >> 4;
+    for (int i = blockIdx.y + int(gridDim.y) * warp; i < na; i += int(gridDim.y) * kDispWarps) {
+        const int slot = slot_s[i];
+        const int t = (a0 + i) / k;
+        if (slot >= 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(x + size_t(t) * row_bytes);
+            uint4* dst = reinterpret_cast<uint4*>(xp + size_t(slot) * row_bytes);
+            for (int v = lane; v < vecs; v += 32) dst[v] = __ldg(src + v);
+        } else if (out_zero_dropped != nullptr) {
+            uint4* dst = reinterpret_cast<uint4*>(out_zero_dropped + size_t(t) * row_bytes);
+            for (int v = lane; v < vecs; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Step 4: combine.  out[t] = sum over kept slots j (in slot order) of
 // w_tj * yp[slot_of[t*k+j]]; w_tj = gate or 1.  fp32 accumulation.
 // ---------------------------------------------------------------------------

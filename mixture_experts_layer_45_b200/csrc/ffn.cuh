@@ -96,7 +96,7 @@ template <int MODE>
 __global__ void __launch_bounds__(kSgThreads)
 ffn_simt_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ offsets, int E, int N, int K,
                     const float* __restrict__ W, const float* __restrict__ bias, const float* __restrict__ row_gate,
-                    float* __restrict__ C) {
+                    const int32_t* __restrict__ out_rows, float* __restrict__ C) {
     __shared__ TileTable tt;
     __shared__ __align__(16) float As[2][kSgBK][kSgLd];
     __shared__ __align__(16) float Bs[2][kSgBK][kSgLd];
@@ -168,6 +168,7 @@ ffn_simt_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ off
             const int r = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
             if (r >= rows) continue;
             const size_t grow = size_t(tt.off[tc.e]) + r;
+            const size_t crow = (out_rows != nullptr) ? size_t(out_rows[grow]) : grow;
             const float g = (MODE == kFc2Gate && row_gate != nullptr) ? row_gate[grow] : 1.f;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -179,7 +180,7 @@ ffn_simt_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ off
                     const float c = acc[i][h * 4 + j] + bias[size_t(tc.e) * N + n + j];
                     v[j] = (MODE == kFc1Gelu) ? gelu_erf(c) : g * c;
                 }
-                *reinterpret_cast<float4*>(C + grow * N + n) = make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<float4*>(C + crow * N + n) = make_float4(v[0], v[1], v[2], v[3]);
             }
         }
     }
@@ -189,18 +190,22 @@ ffn_simt_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ off
 // bf16 path: tcgen05.mma (kind::f16) with fp32 accumulators in tensor
 // memory, operands brought to shared memory by TMA (128B swizzle).
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0        TMA producer (one thread)
 //   warp 1        tensor-memory allocator and MMA issuer (one thread)
-//   warps 2..5    epilogue: tcgen05.ld of their 32-lane quarter, bias,
-//                 GELU or gate, bf16 stores (row-masked to the expert)
+//   warps 2..9    epilogue: warp w reads TMEM lane quarter w%4 and every
+//                 other 32-column chunk (half (w-2)/4), adds the bias
+//                 (staged once per tile in shared memory), applies GELU or
+//                 the row gate, rounds to bf16 and stores rows masked to
+//                 the expert's group
 // Pipelines: STAGES shared-memory stages (full/empty mbarriers) and two
 // accumulators of BN columns each (tfull/tempty mbarriers), so the
 // epilogue of one tile overlaps the main loop of the next.
 // ===========================================================================
 constexpr int kTcBM = 128;
 constexpr int kTcBK = 64;            // 64 bf16 = 128 B = one swizzle row
-constexpr int kTcThreads = 192;
+constexpr int kTcEpiWarps = 8;
+constexpr int kTcThreads = 64 + 32 * kTcEpiWarps;
 
 template <int BN, int STAGES>
 struct TcCfg {
@@ -217,14 +222,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const int32_t* __restrict__ offsets, int E, int N, int K,
                    const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
-                   __nv_bfloat16* __restrict__ C) {
+                   const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C) {
     using Cfg = TcCfg<BN, STAGES>;
-    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
     __shared__ TileTable tt;
     __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
     __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
+    __shared__ float sbias[BN];
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
 
@@ -236,7 +242,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], 4);   // one arrival per epilogue warp
+            mbar_init(&tempty_bar[a], kTcEpiWarps);   // one arrival per epilogue warp
         }
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
@@ -280,15 +286,13 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            {
-                // every load this thread issued lands before the CTA exits
-                // (immediate on the normal path, where the MMA consumed them)
-                for (int s = 0; s < STAGES; ++s) {
-                    if (last_parity[s] < 0) continue;
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(&full_bar[s], uint32_t(last_parity[s])) &&
-                           globaltimer_ns() - t0 < kWaitLimitNs) {
-                    }
+            // every load this thread issued lands before the CTA exits
+            // (immediate on the normal path, where the MMA consumed them)
+            for (int s = 0; s < STAGES; ++s) {
+                if (last_parity[s] < 0) continue;
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&full_bar[s], uint32_t(last_parity[s])) &&
+                       globaltimer_ns() - t0 < kWaitLimitNs) {
                 }
             }
         }
@@ -330,41 +334,52 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
-        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        // ---------------- epilogue (warps 2..9) ----------------
+        const int etid = threadIdx.x - 64;   // 0..255
+        const int q = warp & 3;              // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;    // which alternate 32-column chunks
         int acc = 0;
         uint32_t acc_phase = 0;
+        bool failed = false;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            // all epilogue warps stop together once any wait has given up, so
+            // none is left behind at a named barrier
+            if (named_bar_red_or(1, 32 * kTcEpiWarps, failed || *abort_p)) break;
             const TileCoord tc = decode_tile(tt, E, t);
             const int rows = tt.off[tc.e + 1] - tt.off[tc.e];
             const int r_in = tc.mt * kTcBM + q * 32 + lane;
             const bool valid = r_in < rows;
             const size_t grow = size_t(tt.off[tc.e]) + r_in;
+            // destination row: the grouped row, or (direct output) the row out_rows names
+            const size_t crow = (out_rows != nullptr && valid) ? size_t(out_rows[grow]) : grow;
             const int n0 = tc.nt * BN;
             float g = 1.f;
             if (MODE == kFc2Gate && row_gate != nullptr && valid) g = row_gate[grow];
-            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_p)) break;
+            // (the barrier above also ends every read of the previous tile's bias)
+            for (int i = etid; i < BN; i += 32 * kTcEpiWarps)
+                sbias[i] = (n0 + i < N) ? __bfloat162float(bias[size_t(tc.e) * N + n0 + i]) : 0.f;
+            named_bar_sync(1, 32 * kTcEpiWarps);   // this tile's bias is visible
+            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_p)) {
+                failed = true;
+                continue;
+            }
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = half; c < BN / 32; c += 2) {
                 uint32_t r[32];
                 __syncwarp();
                 tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
                 tmem_ld_wait();
                 const int nb = n0 + c * 32;
                 if (!valid || nb >= N) continue;
-                const __nv_bfloat16* bp = bias + size_t(tc.e) * N + nb;
-                __nv_bfloat16* cp = C + grow * N + nb;
+                __nv_bfloat16* cp = C + crow * N + nb;
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     if (nb + v * 8 >= N) break;
-                    const uint4 bb = *reinterpret_cast<const uint4*>(bp + v * 8);
-                    const float bf[8] = {bf16_lo(bb.x), bf16_hi(bb.x), bf16_lo(bb.y), bf16_hi(bb.y),
-                                         bf16_lo(bb.z), bf16_hi(bb.z), bf16_lo(bb.w), bf16_hi(bb.w)};
                     float o[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float cval = __uint_as_float(r[v * 8 + i]) + bf[i];
+                        const float cval = __uint_as_float(r[v * 8 + i]) + sbias[c * 32 + v * 8 + i];
                         o[i] = (MODE == kFc1Gelu) ? gelu_erf(cval) : g * cval;
                     }
                     uint4 u;

@@ -130,8 +130,12 @@ int check_sizes(int T, int d, int ff, int E, int k, int dtype, bool need_ff) {
 }
 
 struct WsLayout {
-    size_t idx, gate, psum, counts, offsets, perm, slot_of, drop, row_gate, hist, base, xp, h, yp, total;
+    size_t idx, gate, counts, offsets, perm, slot_of, row_gate, xp, h, yp;
+    size_t fhist, fbase, fpsum, total;   // per-router-chunk arrays of the fused forward dispatch
 };
+
+// tokens per router CTA (= one dispatch chunk of the forward path)
+inline int router_chunk_tokens(int dtype) { return dtype == MOE_BF16 ? kRtBM : kRouterTM; }
 
 size_t dispatch_ws_bytes(int A, int E) {
     const int nblk = std::max(1, ceil_div(A, kDispChunk));
@@ -149,18 +153,18 @@ WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype) {
     };
     L.idx = take(A * 4);
     L.gate = take(A * 4);
-    L.psum = take(size_t(E) * 4);
     L.counts = take(size_t(E) * 4);
     L.offsets = take(size_t(E + 1) * 4);
     L.perm = take(A * 4);
     L.slot_of = take(A * 4);
-    L.drop = take(A);
     L.row_gate = take(A * 4);
-    L.hist = take(dispatch_ws_bytes(int(A), E));
-    L.base = L.hist + dispatch_ws_bytes(int(A), E) / 2;
     L.xp = take(A * d * es);
     L.h = take(A * ff * es);
     L.yp = take(A * d * es);
+    const size_t nchunk = size_t(std::max(1, ceil_div(T, router_chunk_tokens(dtype))));
+    L.fhist = take(nchunk * E * 4);
+    L.fbase = take(nchunk * E * 4);
+    L.fpsum = take(nchunk * E * 4);
     L.total = o;
     return L;
 }
@@ -222,32 +226,63 @@ bool set_smem_attr(K kernel, size_t bytes) {
 // ---------------------------------------------------------------------------
 template <typename Tin, int EP>
 int launch_router_ep(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                     float* gate, float* psum, cudaStream_t s) {
+                     float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
     auto kern = router_topk_kernel<Tin, EP>;
     const size_t smem = router_smem_bytes<EP>();
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     Launch L(MOE_KERNEL_ROUTER, s);
     kern<<<ceil_div(T, kRouterTM), kRouterThreads, smem, s>>>(static_cast<const Tin*>(x), static_cast<const Tin*>(wr),
-                                                              bias, T, d, E, k, idx, gate, psum);
+                                                              bias, T, d, E, k, idx, gate, psum, psum_part, hist);
     return L.finish();
+}
+
+template <int EP, int KMAX>
+int launch_router_tc(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
+                     float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+    CUtensorMap tmX, tmW;
+    if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), kRtBM)) return MOE_ERR_UNSUPPORTED;
+    if (!make_map_2d(&tmW, wr, uint64_t(d), uint64_t(E), EP)) return MOE_ERR_UNSUPPORTED;
+    auto kern = router_tc_kernel<EP, KMAX>;
+    const size_t smem = RtCfg<EP>::kSmemBytes;
+    if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
+    Launch L(MOE_KERNEL_ROUTER, s);
+    kern<<<ceil_div(T, kRtBM), kRtThreads, smem, s>>>(tmX, tmW, bias, T, d, E, k, idx, gate, psum, psum_part, hist);
+    return L.finish();
+}
+
+template <int KMAX>
+int launch_router_tc_k(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
+                       float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    if (E <= 128) return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
 }
 
 template <typename Tin>
 int launch_router_t(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                    float* gate, float* psum, cudaStream_t s) {
-    if (E <= 16) return launch_router_ep<Tin, 16>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
-    if (E <= 32) return launch_router_ep<Tin, 32>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
-    if (E <= 64) return launch_router_ep<Tin, 64>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
-    if (E <= 128) return launch_router_ep<Tin, 128>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
-    return launch_router_ep<Tin, 256>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+                    float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+    if (E <= 16) return launch_router_ep<Tin, 16>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    if (E <= 32) return launch_router_ep<Tin, 32>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    if (E <= 64) return launch_router_ep<Tin, 64>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    if (E <= 128) return launch_router_ep<Tin, 128>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    return launch_router_ep<Tin, 256>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
 }
 
+// bf16: tcgen05 router (128-token tiles); f32: SIMT fp32 router (32-token tiles).
+// prob_sum (atomic, zeroed here) or psum_part/hist (per tile) as requested.
 int run_router(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int dtype,
-               int32_t* idx, float* gate, float* psum, cudaStream_t s) {
-    if (psum != nullptr && cudaMemsetAsync(psum, 0, size_t(E) * sizeof(float), s) != cudaSuccess)
+               int32_t* idx, float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+    if (psum != nullptr && psum_part == nullptr &&
+        cudaMemsetAsync(psum, 0, size_t(E) * sizeof(float), s) != cudaSuccess)
         return MOE_ERR_CUDA;
-    if (dtype == MOE_BF16) return launch_router_t<__nv_bfloat16>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
-    return launch_router_t<float>(x, wr, bias, T, d, E, k, idx, gate, psum, s);
+    if (dtype == MOE_BF16) {
+        if (k == 1) return launch_router_tc_k<1>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+        if (k == 2) return launch_router_tc_k<2>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+        return launch_router_tc_k<MOE_MAX_TOPK>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    }
+    return launch_router_t<float>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
 }
 
 int run_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int capacity, int32_t* counts,
@@ -285,13 +320,14 @@ int run_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int
     return MOE_OK;
 }
 
-// tile shapes of the bf16 tensor-core GEMMs
-constexpr int kFc1BN = 256, kFc1Stages = 4;
-constexpr int kFc2BN = 128, kFc2Stages = 6;
+// bf16 tensor-core GEMM tile: 128 x 256 (the widest single-CTA MMA; narrower
+// tiles measured slower on every workload: more A re-reads per FLOP)
+constexpr int kTcBN = 256, kTcStages = 4;
 
 template <int BN, int STAGES, int MODE>
 int launch_tc(const void* a, int a_cols, int max_rows, const void* w, int N, int E, const int32_t* offsets,
-              const void* bias, const float* row_gate, void* c, int kernel_id, cudaStream_t s) {
+              const void* bias, const float* row_gate, const int32_t* out_rows, void* c, int kernel_id,
+              cudaStream_t s) {
     CUtensorMap tmA, tmB;
     if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(max_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
     if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), BN)) return MOE_ERR_UNSUPPORTED;
@@ -302,37 +338,65 @@ int launch_tc(const void* a, int a_cols, int max_rows, const void* w, int N, int
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
     Launch L(kernel_id, s);
     kern<<<grid, kTcThreads, smem, s>>>(tmA, tmB, offsets, E, N, a_cols, static_cast<const __nv_bfloat16*>(bias),
-                                        row_gate, static_cast<__nv_bfloat16*>(c));
+                                        row_gate, out_rows, static_cast<__nv_bfloat16*>(c));
     return L.finish();
 }
 
 template <int MODE>
 int launch_simt(const void* a, int K, int max_rows, const void* w, int N, int E, const int32_t* offsets,
-                const void* bias, const float* row_gate, void* c, int kernel_id, cudaStream_t s) {
+                const void* bias, const float* row_gate, const int32_t* out_rows, void* c, int kernel_id,
+                cudaStream_t s) {
     const long long tiles_ub = (static_cast<long long>(ceil_div(max_rows, kSgBM)) + E) * ceil_div(N, kSgBN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, 2ll * num_sms())));
     Launch L(kernel_id, s);
     ffn_simt_f32_kernel<MODE><<<grid, kSgThreads, 0, s>>>(static_cast<const float*>(a), offsets, E, N, K,
                                                           static_cast<const float*>(w),
-                                                          static_cast<const float*>(bias), row_gate,
+                                                          static_cast<const float*>(bias), row_gate, out_rows,
                                                           static_cast<float*>(c));
     return L.finish();
 }
 
+// out_rows (nullable): fc2 writes grouped row r to row out_rows[r] of yp
+// (the direct output of a k == 1 layer, out_rows = perm)
 int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
             const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp, int dtype,
-            cudaStream_t s) {
+            const int32_t* out_rows, cudaStream_t s) {
     int rc;
     if (dtype == MOE_BF16) {
-        rc = launch_tc<kFc1BN, kFc1Stages, kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, h,
-                                                     MOE_KERNEL_FFN1, s);
+        rc = launch_tc<kTcBN, kTcStages, kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h,
+                                                   MOE_KERNEL_FFN1, s);
         if (rc != MOE_OK) return rc;
-        return launch_tc<kFc2BN, kFc2Stages, kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, yp,
-                                                       MOE_KERNEL_FFN2, s);
+        return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp,
+                                                     MOE_KERNEL_FFN2, s);
     }
-    rc = launch_simt<kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, h, MOE_KERNEL_FFN1, s);
+    rc = launch_simt<kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, MOE_KERNEL_FFN1, s);
     if (rc != MOE_OK) return rc;
-    return launch_simt<kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, yp, MOE_KERNEL_FFN2, s);
+    return launch_simt<kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, MOE_KERNEL_FFN2,
+                                 s);
+}
+
+// Dispatch of the fused forward path from the router's per-chunk histograms
+// and probability sums: one scan CTA (+ statistics), then the permute /
+// gather kernel over (chunk, G) CTAs.
+int run_forward_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int capacity, int chunk_tokens,
+                         const int32_t* fhist, const float* fpsum, int32_t* fbase, int32_t* counts, int32_t* offsets,
+                         int32_t* perm, int32_t* slot_of, float* row_gate, moe_stats* st, const void* x, void* xp,
+                         int d, int dtype, void* out_zero_dropped, cudaStream_t s) {
+    const int nchunk = ceil_div(T, chunk_tokens);
+    int rc;
+    {
+        Launch L(MOE_KERNEL_SCAN, s);
+        forward_scan_kernel<<<1, kDispThreads, 0, s>>>(fhist, fpsum, nchunk, E, T, k, capacity, fbase, counts,
+                                                       offsets, st);
+        if ((rc = L.finish()) != MOE_OK) return rc;
+    }
+    const int G = std::max(1, std::min(8, ceil_div(2 * num_sms(), nchunk)));
+    const int row_bytes = int(size_t(d) * elem_bytes(dtype));
+    Launch L(MOE_KERNEL_PERMUTE, s);
+    forward_permute_kernel<<<dim3(nchunk, G), kFwdThreads, 0, s>>>(
+        idx, gate, T, k, E, chunk_tokens, fbase, offsets, perm, slot_of, row_gate, static_cast<const uint8_t*>(x),
+        row_bytes, static_cast<uint8_t*>(xp), static_cast<uint8_t*>(out_zero_dropped));
+    return L.finish();
 }
 
 int run_combine(const void* yp, const int32_t* slot_of, const float* gate, int T, int k, int d, int dtype, void* out,
@@ -422,6 +486,24 @@ size_t moe_workspace_size(int T, int d, int ff, int E, int k, int dtype) {
     return ws_layout(T, d, ff, E, k, dtype).total;
 }
 
+size_t moe_workspace_offset(int T, int d, int ff, int E, int k, int dtype, int which) {
+    if (check_sizes(T, d, ff, E, k, dtype, true) != MOE_OK) return size_t(-1);
+    const WsLayout L = ws_layout(T, d, ff, E, k, dtype);
+    switch (which) {
+        case MOE_WS_TOPK_IDX: return L.idx;
+        case MOE_WS_TOPK_GATE: return L.gate;
+        case MOE_WS_COUNTS: return L.counts;
+        case MOE_WS_OFFSETS: return L.offsets;
+        case MOE_WS_PERM: return L.perm;
+        case MOE_WS_SLOT_OF: return L.slot_of;
+        case MOE_WS_ROW_GATE: return L.row_gate;
+        case MOE_WS_XP: return L.xp;
+        case MOE_WS_H: return L.h;
+        case MOE_WS_YP: return L.yp;
+        default: return size_t(-1);
+    }
+}
+
 size_t moe_dispatch_workspace_size(int T, int k, int E) {
     if (T < 0 || k < 1 || E < 1 || E > MOE_MAX_EXPERTS || static_cast<long long>(T) * k >= (1ll << 31)) return 0;
     return dispatch_ws_bytes(T * k, E);
@@ -439,7 +521,7 @@ int moe_router_topk(const void* x, const void* w_router, const float* logit_bias
     }
     if (!x || !w_router || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
-    return run_router(x, w_router, logit_bias, T, d, E, k, dtype, topk_idx, topk_gate, prob_sum,
+    return run_router(x, w_router, logit_bias, T, d, E, k, dtype, topk_idx, topk_gate, prob_sum, nullptr, nullptr,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -507,7 +589,7 @@ int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E,
     if (!aligned16(xp) || !aligned16(w1) || !aligned16(b1) || !aligned16(w2) || !aligned16(b2) || !aligned16(h) ||
         !aligned16(yp))
         return MOE_ERR_INVALID_ARG;
-    return run_ffn(xp, offsets, max_rows, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype,
+    return run_ffn(xp, offsets, max_rows, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype, nullptr,
                    static_cast<cudaStream_t>(stream));
 }
 
@@ -548,24 +630,32 @@ int moe_forward(const void* x, const void* w_router, const float* logit_bias, co
     uint8_t* w = static_cast<uint8_t*>(ws);
     int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(w + L.idx);
     float* gate = topk_gate_out ? topk_gate_out : reinterpret_cast<float*>(w + L.gate);
-    float* psum = stats ? reinterpret_cast<float*>(w + L.psum) : nullptr;
     int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
     int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
     int32_t* perm = reinterpret_cast<int32_t*>(w + L.perm);
     int32_t* slot_of = reinterpret_cast<int32_t*>(w + L.slot_of);
     float* row_gate = reinterpret_cast<float*>(w + L.row_gate);
+    int32_t* fhist = reinterpret_cast<int32_t*>(w + L.fhist);
+    int32_t* fbase = reinterpret_cast<int32_t*>(w + L.fbase);
+    float* fpsum = stats ? reinterpret_cast<float*>(w + L.fpsum) : nullptr;   // only the statistics need it
     void* xp = w + L.xp;
     void* h = w + L.h;
     void* yp = w + L.yp;
     const int A = T * k;
+    // top-1: every token has one assignment, so fc2 writes the output row of
+    // its token directly (rows of dropped tokens are zeroed by the dispatch)
+    const bool direct = (k == 1);
 
-    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, idx, gate, psum, s)) != MOE_OK) return rc;
-    if ((rc = run_dispatch(idx, gate, T, k, E, capacity, counts, offsets, perm, slot_of, nullptr, row_gate, x, xp, d,
-                           dtype, w + L.hist, s)) != MOE_OK)
+    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, idx, gate, nullptr, fpsum, fhist, s)) != MOE_OK)
         return rc;
-    if ((rc = run_ffn(xp, offsets, A, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype, s)) != MOE_OK) return rc;
-    if ((rc = run_combine(yp, slot_of, nullptr, T, k, d, dtype, out, s)) != MOE_OK) return rc;
-    if (stats != nullptr && (rc = run_stats(counts, offsets, psum, T, k, E, stats, s)) != MOE_OK) return rc;
+    if ((rc = run_forward_dispatch(idx, gate, T, k, E, capacity, router_chunk_tokens(dtype), fhist, fpsum, fbase,
+                                   counts, offsets, perm, slot_of, row_gate, stats, x, xp, d, dtype,
+                                   direct ? out : nullptr, s)) != MOE_OK)
+        return rc;
+    if ((rc = run_ffn(xp, offsets, A, E, d, ff, w1, b1, w2, b2, row_gate, h, direct ? out : yp, dtype,
+                      direct ? perm : nullptr, s)) != MOE_OK)
+        return rc;
+    if (!direct && (rc = run_combine(yp, slot_of, nullptr, T, k, d, dtype, out, s)) != MOE_OK) return rc;
     return MOE_OK;
 }
 

@@ -1,11 +1,17 @@
 // Step 1 of the layer: the top-k softmax router (cookbook notebook "Mixture-
 // of-experts and expert parallelism", section "Top-k router").
 //
-// One CTA owns kRouterTM tokens.  The logits tile [tokens x experts] is an
-// fp32 register-tiled product over K chunks staged in shared memory; then
-// one warp per token does the max-subtracted softmax, the k-round warp
-// argmax (ties -> lower expert index) and the per-expert probability sums
-// used by the Switch auxiliary loss.
+// Two kernels compute the same thing:
+//  * router_tc_kernel (bf16): the logits tile [128 tokens x E] is one
+//    tcgen05.mma chain into tensor memory; each epilogue thread then owns one
+//    token's logits row (online softmax, register top-k).
+//  * router_topk_kernel (fp32 and the fallback-free fp32 path): fp32
+//    register-tiled logits over K chunks staged in shared memory, one warp
+//    per token for softmax and a k-round warp argmax.
+// Both select by logit, largest first, an exact tie going to the lower
+// expert index, and both can emit, per token tile, the expert histogram of
+// the chosen experts and the per-expert probability sums (used by the
+// dispatch scan and the Switch auxiliary loss) without atomics on floats.
 #pragma once
 
 #include "common.cuh"
@@ -31,11 +37,14 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
 }
 
 // EP: expert count padded to a multiple of 16 (16..256)
+// prob_sum:  [E], accumulated with one atomicAdd per CTA and expert (caller zeroes it), or
+// psum_part: [gridDim.x][E] per-CTA sums (deterministic), and
+// hist:      [gridDim.x][E] per-CTA counts of the chosen experts; each may be null.
 template <typename Tin, int EP>
 __global__ void __launch_bounds__(kRouterThreads)
 router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const float* __restrict__ bias,
                    int T, int d, int E, int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
-                   float* __restrict__ prob_sum) {
+                   float* __restrict__ prob_sum, float* __restrict__ psum_part, int32_t* __restrict__ hist) {
     constexpr int EPT = EP / 16;          // experts per thread
     constexpr int NV = (EP + 31) / 32;    // expert values per lane in the softmax
     extern __shared__ __align__(16) float smem[];
@@ -43,6 +52,8 @@ router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const 
     float* ws = xs + kRouterTM * kRouterLd;             // [EP][Ld]
     float* lg = ws + EP * kRouterLd;                    // [TM][EP+1]
     float* red = lg + kRouterTM * (EP + 1);             // [8][EP]
+    __shared__ int s_hist[EP];
+    for (int e = threadIdx.x; e < EP; e += kRouterThreads) s_hist[e] = 0;
 
     const int tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
@@ -158,23 +169,253 @@ router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const 
             if (lane == 0) {
                 topk_idx[size_t(t) * k + j] = be;
                 topk_gate[size_t(t) * k + j] = expf(bv - m) * inv;
+                atomicAdd(&s_hist[be], 1);
             }
         }
     }
 
-    if (prob_sum != nullptr) {
 #pragma unroll
-        for (int c = 0; c < NV; ++c) {
-            const int e = lane + 32 * c;
-            if (e < EP) red[warp * EP + e] = psum[c];
-        }
-        __syncthreads();
-        for (int e = tid; e < E; e += kRouterThreads) {
-            float tot = 0.f;
+    for (int c = 0; c < NV; ++c) {
+        const int e = lane + 32 * c;
+        if (e < EP) red[warp * EP + e] = psum[c];
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kRouterThreads) {
+        float tot = 0.f;
 #pragma unroll
-            for (int w = 0; w < kRouterThreads / 32; ++w) tot += red[w * EP + e];
-            atomicAdd(prob_sum + e, tot);
+        for (int w = 0; w < kRouterThreads / 32; ++w) tot += red[w * EP + e];
+        if (psum_part != nullptr) psum_part[size_t(blockIdx.x) * E + e] = tot;
+        else if (prob_sum != nullptr) atomicAdd(prob_sum + e, tot);
+        if (hist != nullptr) hist[size_t(blockIdx.x) * E + e] = s_hist[e];
+    }
+}
+
+// ===========================================================================
+// bf16 router on the tensor cores.  One CTA per 128-token tile, 192 threads:
+//   warp 0      TMA producer: x tile rows [t0, t0+128) and W_r, 64 columns of
+//               K per stage (128B swizzle; rows past T and experts past E
+//               are zero-filled by the tensor maps)
+//   warp 1      TMEM allocator and MMA issuer: logits[128 x EP] in fp32
+//   warps 2..5  epilogue, thread = token: +bias, online max/sum over 32-column
+//               TMEM loads, register top-k (ties to the lower index), gates,
+//               then the per-expert probability column sums (shared-memory
+//               transpose, fixed summation order) and the expert histogram
+// ===========================================================================
+constexpr int kRtBM = 128;
+constexpr int kRtThreads = 192;
+
+template <int EP>
+struct RtCfg {
+    static constexpr uint32_t kABytes = kRtBM * 64 * 2;
+    static constexpr uint32_t kBBytes = EP * 64 * 2;
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = (EP <= 64) ? 8 : (EP <= 128 ? 6 : 4);
+    static constexpr uint32_t kTmemCols = EP < 32 ? 32 : EP;
+    static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024;
+};
+
+template <int EP, int KMAX>
+__global__ void __launch_bounds__(kRtThreads, 1)
+router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                 const float* __restrict__ bias, int T, int d, int E, int k, int32_t* __restrict__ topk_idx,
+                 float* __restrict__ topk_gate, float* __restrict__ prob_sum, float* __restrict__ psum_part,
+                 int32_t* __restrict__ hist) {
+    using Cfg = RtCfg<EP>;
+    constexpr int S = Cfg::kStages;
+    constexpr int NCH = (EP + 31) / 32;   // 32-column TMEM chunks
+    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], done_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+    __shared__ int s_hist[EP];
+    __shared__ float s_col[4][NCH * 32];     // per-warp column sums of the probabilities
+    __shared__ float s_tr[4][32][33];        // per-warp 32 x 32 transpose
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full_bar[i], 1);
+            mbar_init(&empty_bar[i], 1);
         }
+        mbar_init(&done_bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW);
+    }
+    for (int e = threadIdx.x; e < EP; e += kRtThreads) s_hist[e] = 0;
+    for (int i = threadIdx.x; i < 4 * NCH * 32; i += kRtThreads) (&s_col[0][0])[i] = 0.f;
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+    const int KB = (d + 63) / 64;
+    const int t0 = blockIdx.x * kRtBM;
+    volatile int* abort_p = &abort_flag;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int last_parity[S];
+            for (int i = 0; i < S; ++i) last_parity[i] = -1;
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) break;
+                uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
+                mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
+                tma_load_2d(sa, &tmX, &full_bar[stage], kb * 64, t0);
+                tma_load_2d(sa + Cfg::kABytes, &tmW, &full_bar[stage], kb * 64, 0);
+                last_parity[stage] = int(phase);
+                if (++stage == S) { stage = 0; phase ^= 1u; }
+            }
+            for (int i = 0; i < S; ++i) {
+                if (last_parity[i] < 0) continue;
+                const uint64_t w0 = globaltimer_ns();
+                while (!mbar_try_wait(&full_bar[i], uint32_t(last_parity[i])) && globaltimer_ns() - w0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kRtBM, EP);
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(&full_bar[stage], phase, abort_p)) break;
+                tc_fence_after();
+                const uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
+                const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sa));
+                const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sa + Cfg::kABytes));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem_base, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc,
+                             (kb > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&empty_bar[stage]);
+                if (++stage == S) { stage = 0; phase ^= 1u; }
+            }
+            umma_commit(&done_bar);   // tracks every MMA issued above
+            // TMEM is released only after those MMAs complete (bounded wait)
+            const uint64_t w0 = globaltimer_ns();
+            while (!mbar_try_wait(&done_bar, 0) && globaltimer_ns() - w0 < kWaitLimitNs) {
+            }
+        }
+    } else {
+        const int ew = warp - 2;      // 0..3
+        const int q = warp & 3;       // TMEM lane quarter
+        const int row = q * 32 + lane;
+        const int t = t0 + row;
+        const bool valid = t < T;
+        const bool ok = mbar_wait(&done_bar, 0, abort_p);
+        tc_fence_after();
+        float m = -INFINITY, ssum = 0.f;
+        float tv[KMAX];
+        int ti[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            tv[j] = -INFINITY;
+            ti[j] = 0x7fffffff;
+        }
+        // pass 1: online softmax statistics and top-k over the logits row
+#pragma unroll 1
+        for (int c = 0; c < NCH; ++c) {
+            uint32_t r[32];
+            __syncwarp();
+            tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
+            tmem_ld_wait();
+            float l[32];
+            float cm = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int e = c * 32 + i;
+                float v = (e < E && ok) ? __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f) : -INFINITY;
+                if (v != v) v = -INFINITY;
+                l[i] = v;
+                cm = fmaxf(cm, v);
+            }
+            const float mn = fmaxf(m, cm);
+            if (mn != -INFINITY) {
+                float acc = (m == -INFINITY) ? 0.f : ssum * expf(m - mn);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc += (l[i] == -INFINITY) ? 0.f : expf(l[i] - mn);
+                ssum = acc;
+                m = mn;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                float v = l[i];
+                int ix = c * 32 + i;
+                if (v == -INFINITY || !(v > tv[KMAX - 1])) continue;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    if (v > tv[j]) {
+                        const float tf = tv[j];
+                        tv[j] = v;
+                        v = tf;
+                        const int tix = ti[j];
+                        ti[j] = ix;
+                        ix = tix;
+                    }
+                }
+            }
+        }
+        const float inv = 1.0f / ssum;
+        if (valid && ok) {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < k) {
+                    // fewer than k finite logits cannot happen for k <= E with finite inputs;
+                    // guard so an all-NaN row still yields valid, distinct indices
+                    int e = ti[j];
+                    if (e >= E) e = j;
+                    topk_idx[size_t(t) * k + j] = e;
+                    topk_gate[size_t(t) * k + j] = (tv[j] == -INFINITY) ? 0.f : expf(tv[j] - m) * inv;
+                    atomicAdd(&s_hist[e], 1);
+                }
+            }
+        }
+        // pass 2: per-expert sums of this tile's probabilities (fixed order)
+        if (prob_sum != nullptr || psum_part != nullptr) {
+#pragma unroll 1
+            for (int c = 0; c < NCH; ++c) {
+                uint32_t r[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int e = c * 32 + i;
+                    float p = 0.f;
+                    if (valid && ok && e < E) {
+                        float v = __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f);
+                        p = (v != v) ? 0.f : expf(v - m) * inv;
+                    }
+                    s_tr[ew][lane][i] = p;
+                }
+                __syncwarp();
+                float cs = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) cs += s_tr[ew][i][lane];
+                s_col[q][c * 32 + lane] = cs;
+                __syncwarp();
+            }
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kRtThreads) {
+        const float tot = ((s_col[0][e] + s_col[1][e]) + s_col[2][e]) + s_col[3][e];
+        if (psum_part != nullptr) psum_part[size_t(blockIdx.x) * E + e] = tot;
+        else if (prob_sum != nullptr) atomicAdd(prob_sum + e, tot);
+        if (hist != nullptr) hist[size_t(blockIdx.x) * E + e] = s_hist[e];
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::kTmemCols);
     }
 }
 

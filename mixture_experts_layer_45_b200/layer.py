@@ -109,6 +109,14 @@ class MoELayer:
 
     __call__ = forward
 
+    def workspace_view(self, T: int, which: str, dtype, count: int) -> torch.Tensor:
+        """A view of one of moe_forward's intermediate arrays in the workspace
+        (valid after a forward call on T tokens; for inspection and tests)."""
+        off = _lib.moe_workspace_offset(T, self.p.d, self.p.ff, self.p.E, self.k, self.p.dtype, which)
+        ws = self.workspace(T)
+        nbytes = count * torch.tensor([], dtype=dtype).element_size()
+        return ws[off:off + nbytes].view(dtype)
+
     def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, x_dev: torch.Tensor,
                      out_dev: torch.Tensor, stream=None) -> torch.Tensor:
         """End to end from (pinned) host memory: H2D copy, forward, D2H copy,
