@@ -31,6 +31,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: every kernel is launched allowed to start
+// before the previous kernel on the stream has finished.  It calls
+// pdl_wait() before it reads anything an earlier kernel wrote (the wait
+// returns once the previous grid has completed and its memory is visible;
+// immediately when launched normally), and pdl_release() to let the next
+// kernel launch its own prologue early.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -23,6 +23,8 @@ constexpr int kDispPerWarp = kDispChunk / kDispWarps;  // 256 = 8 rounds of 32
 
 __global__ void __launch_bounds__(kDispThreads)
 dispatch_count_kernel(const int32_t* __restrict__ idx, int A, int E, int32_t* __restrict__ hist) {
+    pdl_wait();
+    pdl_release();
     __shared__ int h[MOE_MAX_EXPERTS];
     for (int e = threadIdx.x; e < E; e += kDispThreads) h[e] = 0;
     __syncthreads();
@@ -44,6 +46,8 @@ dispatch_count_kernel(const int32_t* __restrict__ idx, int A, int E, int32_t* __
 __global__ void __launch_bounds__(kDispThreads)
 dispatch_scan_kernel(const int32_t* __restrict__ hist, int nblk, int E, int capacity,
                      int32_t* __restrict__ base, int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+    pdl_wait();
+    pdl_release();
     __shared__ int kept[MOE_MAX_EXPERTS];
     for (int e = threadIdx.x; e < E; e += kDispThreads) {
         int run = 0;
@@ -88,6 +92,8 @@ dispatch_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict
                         const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
                         int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, uint8_t* __restrict__ drop_mask,
                         float* __restrict__ row_gate) {
+    pdl_wait();
+    pdl_release();
     __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
     __shared__ int off_s[MOE_MAX_EXPERTS + 1];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -147,6 +153,8 @@ dispatch_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict
 __global__ void __launch_bounds__(256)
 dispatch_gather_kernel(const uint8_t* __restrict__ x, int row_bytes, const int32_t* __restrict__ perm,
                        const int32_t* __restrict__ offsets, int E, int k, uint8_t* __restrict__ xp) {
+    pdl_wait();
+    pdl_release();
     const int R = offsets[E];
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -172,29 +180,47 @@ dispatch_gather_kernel(const uint8_t* __restrict__ x, int row_bytes, const int32
 //                           k == 1 with a direct output it also zero-fills the
 //                           output rows of dropped tokens
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024)
+constexpr int kFwdScanThreads = 1024;
+
+// One CTA; warp w scans experts w, w+32, ...: 32 chunks per step, each lane
+// one chunk, a warp prefix sum and a carried total (sums in fixed order).
+__global__ void __launch_bounds__(kFwdScanThreads)
 forward_scan_kernel(const int32_t* __restrict__ hist, const float* __restrict__ psum_part, int nchunk, int E,
                     int T, int k, int capacity, int32_t* __restrict__ base, int32_t* __restrict__ counts,
                     int32_t* __restrict__ offsets, moe_stats* __restrict__ st) {
+    pdl_wait();
+    pdl_release();
     __shared__ int kept[MOE_MAX_EXPERTS];
     __shared__ int cnt[MOE_MAX_EXPERTS];
     __shared__ float fp[MOE_MAX_EXPERTS];
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = warp; e < E; e += kFwdScanThreads / 32) {
+        int carry = 0;
         float ps = 0.f;
-        for (int b = 0; b < nchunk; ++b) {
-            base[size_t(b) * E + e] = run;
-            run += hist[size_t(b) * E + e];
-            if (psum_part != nullptr) ps += psum_part[size_t(b) * E + e];
+        for (int b0 = 0; b0 < nchunk; b0 += 32) {
+            const int b = b0 + lane;
+            const int h = b < nchunk ? hist[size_t(b) * E + e] : 0;
+            if (psum_part != nullptr && b < nchunk) ps += psum_part[size_t(b) * E + e];
+            int incl = h;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (b < nchunk) base[size_t(b) * E + e] = carry + incl - h;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        counts[e] = run;
-        cnt[e] = run;
-        kept[e] = capacity < 0 ? run : min(run, capacity);
-        fp[e] = (float(run) / float(T)) * (ps / float(T));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        if (lane == 0) {
+            counts[e] = carry;
+            cnt[e] = carry;
+            kept[e] = capacity < 0 ? carry : min(carry, capacity);
+            fp[e] = (float(carry) / float(T)) * (ps / float(T));
+        }
     }
     __syncthreads();
     if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
         constexpr int PER = MOE_MAX_EXPERTS / 32;
         int local[PER];
         int sum = 0;
@@ -258,6 +284,8 @@ forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict_
                        int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, float* __restrict__ row_gate,
                        const uint8_t* __restrict__ x, int row_bytes, uint8_t* __restrict__ xp,
                        uint8_t* __restrict__ out_zero_dropped) {
+    pdl_wait();
+    pdl_release();
     __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
     __shared__ int off_s[MOE_MAX_EXPERTS + 1];
     __shared__ int slot_s[kFwdMaxChunk];
@@ -367,6 +395,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
                int Tn, int k, int d, T* __restrict__ out) {
+    pdl_wait();
+    pdl_release();
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int lane = threadIdx.x & 31;
     const int chunks = d >> 3;
@@ -399,6 +429,8 @@ combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, co
 __global__ void __launch_bounds__(256)
 stats_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
              const float* __restrict__ prob_sum, int T, int k, int E, moe_stats* __restrict__ st) {
+    pdl_wait();
+    pdl_release();
     __shared__ float s_fp[256];
     __shared__ int s_max[256];
     float fp = 0.f;

@@ -29,6 +29,8 @@ struct TileTable {
 // Must be called by all threads of the CTA; ends with __syncthreads().
 __device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ offsets, int E, int BM, int ntiles_n,
                                                  TileTable& tt) {
+    pdl_wait();
+    pdl_release();
     for (int e = threadIdx.x; e <= E; e += blockDim.x) tt.off[e] = offsets[e];
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -224,7 +226,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                    const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
                    const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C) {
     using Cfg = TcCfg<BN, STAGES>;
-    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN: whole 32-column epilogue chunks, MMA N <= 256");
     __shared__ TileTable tt;
     __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
     __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;

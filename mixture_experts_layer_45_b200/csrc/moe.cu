@@ -77,8 +77,9 @@ class Launch {
             if (start_ != nullptr) cudaEventRecord(start_, stream_);
         }
     }
-    int finish() {
-        const cudaError_t err = cudaGetLastError();
+    int finish(cudaError_t launch_err = cudaSuccess) {
+        const cudaError_t last = cudaGetLastError();
+        const cudaError_t err = launch_err != cudaSuccess ? launch_err : last;
         g_launches.fetch_add(1, std::memory_order_relaxed);
         if (start_ != nullptr) {
             std::lock_guard<std::mutex> lk(g_timing.mu);
@@ -102,6 +103,24 @@ class Launch {
     cudaStream_t stream_;
     cudaEvent_t start_ = nullptr;
 };
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream drains; the kernels order their own
+// global reads with griddepcontrol.wait.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------------------
 // helpers
@@ -131,8 +150,12 @@ int check_sizes(int T, int d, int ff, int E, int k, int dtype, bool need_ff) {
 
 struct WsLayout {
     size_t idx, gate, counts, offsets, perm, slot_of, row_gate, xp, h, yp;
-    size_t fhist, fbase, fpsum, total;   // per-router-chunk arrays of the fused forward dispatch
+    size_t fhist, fbase, fpsum, rpart, total;   // per-router-chunk arrays of the fused forward path
 };
+
+// expert count padded for the router tile (16, 32, 64, 128 or 256)
+inline int router_ep(int E) { return E <= 16 ? 16 : E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256; }
+constexpr int kMaxRouterSplit = 4;
 
 // tokens per router CTA (= one dispatch chunk of the forward path)
 inline int router_chunk_tokens(int dtype) { return dtype == MOE_BF16 ? kRtBM : kRouterTM; }
@@ -165,6 +188,8 @@ WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype) {
     L.fhist = take(nchunk * E * 4);
     L.fbase = take(nchunk * E * 4);
     L.fpsum = take(nchunk * E * 4);
+    // split-K router partial logits: up to kMaxRouterSplit x [T, EP] fp32 (bf16 path only)
+    L.rpart = take(dtype == MOE_BF16 ? size_t(kMaxRouterSplit) * T * router_ep(E) * 4 : 0);
     L.total = o;
     return L;
 }
@@ -231,33 +256,62 @@ int launch_router_ep(const void* x, const void* wr, const float* bias, int T, in
     const size_t smem = router_smem_bytes<EP>();
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     Launch L(MOE_KERNEL_ROUTER, s);
-    kern<<<ceil_div(T, kRouterTM), kRouterThreads, smem, s>>>(static_cast<const Tin*>(x), static_cast<const Tin*>(wr),
+    cudaError_t launch_err;
+    launch_err = launch_pdl(kern, dim3(ceil_div(T, kRouterTM)), dim3(kRouterThreads), smem, s, static_cast<const Tin*>(x), static_cast<const Tin*>(wr),
                                                               bias, T, d, E, k, idx, gate, psum, psum_part, hist);
-    return L.finish();
+    return L.finish(launch_err);
+}
+
+// K split of the tensor-core router: enough CTAs to stream x from most
+// SMs (each CTA keeps only ~8 TMA boxes in flight), at most kMaxRouterSplit,
+// at least two K blocks per slice; 1 when the tiles alone fill the GPU or
+// there is no workspace for partial logits.
+int router_split(int T, int d, bool have_part) {
+    if (!have_part) return 1;
+    const int tiles = ceil_div(T, kRtBM);
+    const int kblocks = ceil_div(d, 64);
+    if (4 * tiles >= 3 * num_sms()) return 1;
+    int split = ceil_div(num_sms(), tiles);
+    split = std::min(split, kMaxRouterSplit);
+    split = std::min(split, std::max(1, kblocks / 2));
+    return std::max(1, split);
 }
 
 template <int EP, int KMAX>
 int launch_router_tc(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                     float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+                     float* gate, float* psum, float* psum_part, int32_t* hist, float* part, cudaStream_t s) {
     CUtensorMap tmX, tmW;
     if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), kRtBM)) return MOE_ERR_UNSUPPORTED;
     if (!make_map_2d(&tmW, wr, uint64_t(d), uint64_t(E), EP)) return MOE_ERR_UNSUPPORTED;
     auto kern = router_tc_kernel<EP, KMAX>;
     const size_t smem = RtCfg<EP>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
-    Launch L(MOE_KERNEL_ROUTER, s);
-    kern<<<ceil_div(T, kRtBM), kRtThreads, smem, s>>>(tmX, tmW, bias, T, d, E, k, idx, gate, psum, psum_part, hist);
-    return L.finish();
+    const int tiles = ceil_div(T, kRtBM);
+    const int split = router_split(T, d, part != nullptr);
+    int rc;
+    {
+        Launch L(MOE_KERNEL_ROUTER, s);
+        cudaError_t launch_err;
+        launch_err = launch_pdl(kern, dim3(tiles, split), dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k, idx,
+                                gate, psum, psum_part, hist, split > 1 ? part : static_cast<float*>(nullptr));
+        if ((rc = L.finish(launch_err)) != MOE_OK || split == 1) return rc;
+    }
+    Launch L(MOE_KERNEL_SELECT, s);
+    cudaError_t launch_err;
+    launch_err = launch_pdl(router_select_kernel<EP, KMAX>, dim3(tiles), dim3(kRtBM), 0, s,
+                            static_cast<const float*>(part), split, bias, T, E, k, idx, gate, psum_part, hist);
+    return L.finish(launch_err);
 }
 
 template <int KMAX>
 int launch_router_tc_k(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                       float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
-    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 128) return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+                       float* gate, float* psum, float* psum_part, int32_t* hist, float* part, cudaStream_t s) {
+    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
+    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
+    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
+    if (E <= 128)
+        return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
+    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
 }
 
 template <typename Tin>
@@ -270,17 +324,20 @@ int launch_router_t(const void* x, const void* wr, const float* bias, int T, int
     return launch_router_ep<Tin, 256>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
 }
 
-// bf16: tcgen05 router (128-token tiles); f32: SIMT fp32 router (32-token tiles).
-// prob_sum (atomic, zeroed here) or psum_part/hist (per tile) as requested.
+// bf16: tcgen05 router (128-token tiles, split over K when the tiles are
+// too few and `part` offers room for partial logits); f32: SIMT fp32 router
+// (32-token tiles).  prob_sum (atomic, zeroed here) or psum_part/hist (per
+// tile) as requested.
 int run_router(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int dtype,
-               int32_t* idx, float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+               int32_t* idx, float* gate, float* psum, float* psum_part, int32_t* hist, float* part, cudaStream_t s) {
     if (psum != nullptr && psum_part == nullptr &&
         cudaMemsetAsync(psum, 0, size_t(E) * sizeof(float), s) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (dtype == MOE_BF16) {
-        if (k == 1) return launch_router_tc_k<1>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-        if (k == 2) return launch_router_tc_k<2>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-        return launch_router_tc_k<MOE_MAX_TOPK>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+        if (k == 1) return launch_router_tc_k<1>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
+        if (k == 2) return launch_router_tc_k<2>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
+        return launch_router_tc_k<MOE_MAX_TOPK>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part,
+                                                s);
     }
     return launch_router_t<float>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
 }
@@ -295,27 +352,31 @@ int run_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int
     int rc;
     {
         Launch L(MOE_KERNEL_COUNT, s);
-        dispatch_count_kernel<<<nblk, kDispThreads, 0, s>>>(idx, A, E, hist);
-        if ((rc = L.finish()) != MOE_OK) return rc;
+        cudaError_t launch_err;
+        launch_err = launch_pdl(dispatch_count_kernel, dim3(nblk), dim3(kDispThreads), 0, s, idx, A, E, hist);
+        if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
     }
     {
         Launch L(MOE_KERNEL_SCAN, s);
-        dispatch_scan_kernel<<<1, kDispThreads, 0, s>>>(hist, nblk, E, capacity, base, counts, offsets);
-        if ((rc = L.finish()) != MOE_OK) return rc;
+        cudaError_t launch_err;
+        launch_err = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(kDispThreads), 0, s, hist, nblk, E, capacity, base, counts, offsets);
+        if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
     }
     {
         Launch L(MOE_KERNEL_PERMUTE, s);
-        dispatch_permute_kernel<<<nblk, kDispThreads, 0, s>>>(idx, gate, A, E, base, offsets, perm, slot_of, drop,
+        cudaError_t launch_err;
+        launch_err = launch_pdl(dispatch_permute_kernel, dim3(nblk), dim3(kDispThreads), 0, s, idx, gate, A, E, base, offsets, perm, slot_of, drop,
                                                                row_gate);
-        if ((rc = L.finish()) != MOE_OK) return rc;
+        if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
     }
     if (x != nullptr && xp != nullptr) {
         const int row_bytes = int(size_t(d) * elem_bytes(dtype));
         const int grid = std::max(1, std::min(ceil_div(A, 8), num_sms() * 8));
         Launch L(MOE_KERNEL_GATHER, s);
-        dispatch_gather_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(x), row_bytes, perm, offsets, E, k,
+        cudaError_t launch_err;
+        launch_err = launch_pdl(dispatch_gather_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint8_t*>(x), row_bytes, perm, offsets, E, k,
                                                     static_cast<uint8_t*>(xp));
-        if ((rc = L.finish()) != MOE_OK) return rc;
+        if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
     }
     return MOE_OK;
 }
@@ -337,9 +398,10 @@ int launch_tc(const void* a, int a_cols, int max_rows, const void* w, int N, int
     const long long tiles_ub = (static_cast<long long>(ceil_div(max_rows, kTcBM)) + E) * ceil_div(N, BN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
     Launch L(kernel_id, s);
-    kern<<<grid, kTcThreads, smem, s>>>(tmA, tmB, offsets, E, N, a_cols, static_cast<const __nv_bfloat16*>(bias),
+    cudaError_t launch_err;
+    launch_err = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, s, tmA, tmB, offsets, E, N, a_cols, static_cast<const __nv_bfloat16*>(bias),
                                         row_gate, out_rows, static_cast<__nv_bfloat16*>(c));
-    return L.finish();
+    return L.finish(launch_err);
 }
 
 template <int MODE>
@@ -349,11 +411,12 @@ int launch_simt(const void* a, int K, int max_rows, const void* w, int N, int E,
     const long long tiles_ub = (static_cast<long long>(ceil_div(max_rows, kSgBM)) + E) * ceil_div(N, kSgBN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, 2ll * num_sms())));
     Launch L(kernel_id, s);
-    ffn_simt_f32_kernel<MODE><<<grid, kSgThreads, 0, s>>>(static_cast<const float*>(a), offsets, E, N, K,
+    cudaError_t launch_err;
+    launch_err = launch_pdl(ffn_simt_f32_kernel<MODE>, dim3(grid), dim3(kSgThreads), 0, s, static_cast<const float*>(a), offsets, E, N, K,
                                                           static_cast<const float*>(w),
                                                           static_cast<const float*>(bias), row_gate, out_rows,
                                                           static_cast<float*>(c));
-    return L.finish();
+    return L.finish(launch_err);
 }
 
 // out_rows (nullable): fc2 writes grouped row r to row out_rows[r] of yp
@@ -386,37 +449,41 @@ int run_forward_dispatch(const int32_t* idx, const float* gate, int T, int k, in
     int rc;
     {
         Launch L(MOE_KERNEL_SCAN, s);
-        forward_scan_kernel<<<1, kDispThreads, 0, s>>>(fhist, fpsum, nchunk, E, T, k, capacity, fbase, counts,
+        cudaError_t launch_err;
+        launch_err = launch_pdl(forward_scan_kernel, dim3(1), dim3(kFwdScanThreads), 0, s, fhist, fpsum, nchunk, E, T, k, capacity, fbase, counts,
                                                        offsets, st);
-        if ((rc = L.finish()) != MOE_OK) return rc;
+        if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
     }
     const int G = std::max(1, std::min(8, ceil_div(2 * num_sms(), nchunk)));
     const int row_bytes = int(size_t(d) * elem_bytes(dtype));
     Launch L(MOE_KERNEL_PERMUTE, s);
-    forward_permute_kernel<<<dim3(nchunk, G), kFwdThreads, 0, s>>>(
+    cudaError_t launch_err;
+    launch_err = launch_pdl(forward_permute_kernel, dim3(dim3(nchunk, G)), dim3(kFwdThreads), 0, s, 
         idx, gate, T, k, E, chunk_tokens, fbase, offsets, perm, slot_of, row_gate, static_cast<const uint8_t*>(x),
         row_bytes, static_cast<uint8_t*>(xp), static_cast<uint8_t*>(out_zero_dropped));
-    return L.finish();
+    return L.finish(launch_err);
 }
 
 int run_combine(const void* yp, const int32_t* slot_of, const float* gate, int T, int k, int d, int dtype, void* out,
                 cudaStream_t s) {
     const int grid = std::max(1, std::min(ceil_div(T, 8), num_sms() * 16));
     Launch L(MOE_KERNEL_COMBINE, s);
+    cudaError_t launch_err;
     if (dtype == MOE_BF16)
-        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(yp), slot_of, gate, T,
+        launch_err = launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(yp), slot_of, gate, T,
                                                             k, d, static_cast<__nv_bfloat16*>(out));
     else
-        combine_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(yp), slot_of, gate, T, k, d,
+        launch_err = launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, static_cast<const float*>(yp), slot_of, gate, T, k, d,
                                                    static_cast<float*>(out));
-    return L.finish();
+    return L.finish(launch_err);
 }
 
 int run_stats(const int32_t* counts, const int32_t* offsets, const float* psum, int T, int k, int E, moe_stats* st,
               cudaStream_t s) {
     Launch L(MOE_KERNEL_STATS, s);
-    stats_kernel<<<1, 256, 0, s>>>(counts, offsets, psum, T, k, E, st);
-    return L.finish();
+    cudaError_t launch_err;
+    launch_err = launch_pdl(stats_kernel, dim3(1), dim3(256), 0, s, counts, offsets, psum, T, k, E, st);
+    return L.finish(launch_err);
 }
 
 // ---------------------------------------------------------------------------
@@ -522,7 +589,7 @@ int moe_router_topk(const void* x, const void* w_router, const float* logit_bias
     if (!x || !w_router || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
     return run_router(x, w_router, logit_bias, T, d, E, k, dtype, topk_idx, topk_gate, prob_sum, nullptr, nullptr,
-                      static_cast<cudaStream_t>(stream));
+                      nullptr, static_cast<cudaStream_t>(stream));
 }
 
 int moe_dispatch(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E, int capacity,
@@ -646,7 +713,9 @@ int moe_forward(const void* x, const void* w_router, const float* logit_bias, co
     // its token directly (rows of dropped tokens are zeroed by the dispatch)
     const bool direct = (k == 1);
 
-    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, idx, gate, nullptr, fpsum, fhist, s)) != MOE_OK)
+    float* rpart = dtype == MOE_BF16 ? reinterpret_cast<float*>(w + L.rpart) : nullptr;
+    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, idx, gate, nullptr, fpsum, fhist, rpart, s)) !=
+        MOE_OK)
         return rc;
     if ((rc = run_forward_dispatch(idx, gate, T, k, E, capacity, router_chunk_tokens(dtype), fhist, fpsum, fbase,
                                    counts, offsets, perm, slot_of, row_gate, stats, x, xp, d, dtype,

@@ -128,3 +128,57 @@ class MoELayer:
             out_host.copy_(out_dev, non_blocking=True)
         s.synchronize()
         return out_host
+
+
+class HostPipeline:
+    """End-to-end forward passes from pinned host memory, pipelined.
+
+    Each step copies its tokens host -> device, runs the layer and copies
+    the output device -> host.  The three run on their own streams with
+    `depth` device buffers, so the input copy of step i+1 and the output
+    copy of step i-1 overlap the layer of step i (PCIe is full duplex).
+    Every step's copies are still issued and completed.
+    """
+
+    def __init__(self, layer: MoELayer, T: int, depth: int = 2):
+        dev = layer.p.w1.device
+        dt = TORCH_DTYPE[layer.p.dtype]
+        self.layer = layer
+        self.depth = depth
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_run = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        self.x_dev = [torch.empty((T, layer.p.d), dtype=dt, device=dev) for _ in range(depth)]
+        self.out_dev = [torch.empty((T, layer.p.d), dtype=dt, device=dev) for _ in range(depth)]
+        self.in_done = [torch.cuda.Event() for _ in range(depth)]
+        self.run_done = [torch.cuda.Event() for _ in range(depth)]
+        self.out_done = [torch.cuda.Event() for _ in range(depth)]
+
+    def run(self, x_hosts, out_hosts, start_event=None, end_event=None):
+        """x_hosts[i] (pinned) -> layer -> out_hosts[i] (pinned), for every i."""
+        if start_event is not None:
+            start_event.record(self.s_in)
+            self.s_run.wait_event(start_event)
+            self.s_out.wait_event(start_event)
+        for i, (xh, oh) in enumerate(zip(x_hosts, out_hosts)):
+            b = i % self.depth
+            self.s_in.wait_event(self.run_done[b])          # x_dev[b] no longer read
+            with torch.cuda.stream(self.s_in):
+                self.x_dev[b].copy_(xh, non_blocking=True)
+            self.in_done[b].record(self.s_in)
+            self.s_run.wait_event(self.in_done[b])
+            self.s_run.wait_event(self.out_done[b])         # out_dev[b] already copied out
+            self.layer.forward(self.x_dev[b], out=self.out_dev[b], stream=self.s_run)
+            self.run_done[b].record(self.s_run)
+            self.s_out.wait_event(self.run_done[b])
+            with torch.cuda.stream(self.s_out):
+                oh.copy_(self.out_dev[b], non_blocking=True)
+            self.out_done[b].record(self.s_out)
+        if end_event is not None:
+            self.s_run.wait_stream(self.s_out)
+            self.s_in.wait_stream(self.s_out)
+            end_event.record(self.s_out)
+        self.s_out.synchronize()
+        self.s_in.synchronize()
+        self.s_run.synchronize()
+
