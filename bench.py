@@ -435,7 +435,8 @@ def run_ours(args):
     for name, (ms, n) in kt.items():
         if n:
             kernels[name] = {"launches": n, "ms_per_launch": ms / n, "share": ms / tot_k if tot_k else None}
-    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
+    modelled = [kn for kn in kernels if algorithmic_bytes(kn, w, R, E_active, es) is not None]
+    dom = max(modelled, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
     ffn_ms = sum(kernels[k]["ms_per_launch"] for k in ("ffn1", "ffn2") if k in kernels)
     ffn_flops = 4.0 * R * w.d * w.ff
     ffn_tflops = ffn_flops / (ffn_ms / 1000.0) / 1e12 if ffn_ms else None

@@ -263,8 +263,7 @@ MOE_API uint64_t moe_launch_count(void);
 #define MOE_KERNEL_FFN2     6
 #define MOE_KERNEL_COMBINE  7
 #define MOE_KERNEL_STATS    8
-#define MOE_KERNEL_SELECT   9   /* second half of a split-K router */
-#define MOE_NUM_KERNELS     10
+#define MOE_NUM_KERNELS     9
 
 /* moe_timing_enable(1): from now on every kernel launch is bracketed by
  * two CUDA events on its stream (events come from a pool created here, not

@@ -28,7 +28,7 @@ MOE_BF16 = 1
 MOE_MAX_EXPERTS = 256
 MOE_MAX_TOPK = 8
 
-KERNEL_NAMES = ["router", "count", "scan", "permute", "gather", "ffn1", "ffn2", "combine", "stats", "select"]
+KERNEL_NAMES = ["router", "count", "scan", "permute", "gather", "ffn1", "ffn2", "combine", "stats"]
 MOE_NUM_KERNELS = len(KERNEL_NAMES)
 
 

@@ -149,21 +149,47 @@ dispatch_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict
     }
 }
 
-// xp[row, :] = x[perm[row] / k, :] for row < offsets[E]; row_bytes % 16 == 0
+// xp[row, :] = x[perm[row] / k, :] for row < offsets[E]; row_bytes % 16 == 0.
+// With zero_out (top-1 direct output), also zero_out[t, :] = 0 for every token
+// t whose assignment was dropped (slot_of[t] < 0).  Flattened over 16-byte
+// pieces, eight independent loads in flight per thread.
 __global__ void __launch_bounds__(256)
 dispatch_gather_kernel(const uint8_t* __restrict__ x, int row_bytes, const int32_t* __restrict__ perm,
-                       const int32_t* __restrict__ offsets, int E, int k, uint8_t* __restrict__ xp) {
+                       const int32_t* __restrict__ offsets, int E, int k, uint8_t* __restrict__ xp,
+                       const int32_t* __restrict__ slot_of, int T, uint8_t* __restrict__ zero_out) {
     pdl_wait();
     pdl_release();
-    const int R = offsets[E];
-    const int warps_total = gridDim.x * (blockDim.x >> 5);
-    const int lane = threadIdx.x & 31;
+    const long long R = offsets[E];
     const int vecs = row_bytes >> 4;
-    for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < R; row += warps_total) {
-        const int t = perm[row] / k;
-        const uint4* src = reinterpret_cast<const uint4*>(x + size_t(t) * row_bytes);
-        uint4* dst = reinterpret_cast<uint4*>(xp + size_t(row) * row_bytes);
-        for (int i = lane; i < vecs; i += 32) dst[i] = __ldg(src + i);
+    const long long copy_pieces = R * vecs;
+    const long long pieces = copy_pieces + (zero_out != nullptr ? (long long)T * vecs : 0);
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    constexpr int U = 8;
+    for (long long p0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; p0 < pieces; p0 += stride * U) {
+        uint4 val[U];
+        uint4* dst[U];
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            const long long pc = p0 + j * stride;
+            dst[j] = nullptr;
+            if (pc < copy_pieces) {
+                const long long row = pc / vecs;
+                const int v = int(pc - row * vecs);
+                const int t = perm[row] / k;
+                val[j] = __ldg(reinterpret_cast<const uint4*>(x + size_t(t) * row_bytes) + v);
+                dst[j] = reinterpret_cast<uint4*>(xp) + pc;
+            } else if (pc < pieces) {
+                const long long q = pc - copy_pieces;
+                const long long t = q / vecs;
+                if (slot_of[t] < 0) {
+                    val[j] = make_uint4(0u, 0u, 0u, 0u);
+                    dst[j] = reinterpret_cast<uint4*>(zero_out) + q;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < U; ++j)
+            if (dst[j] != nullptr) *dst[j] = val[j];
     }
 }
 
@@ -350,18 +376,44 @@ forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict_
         }
     }
     __syncthreads();
-    // rows of this chunk handled by this CTA: i = blockIdx.y, blockIdx.y + gridDim.y, ...
+    // rows of this chunk handled by this CTA: i = blockIdx.y, blockIdx.y + gridDim.y, ...,
+    // flattened into 16-byte pieces with eight independent loads in flight per thread
     const int vecs = row_bytes >> 4;
-    for (int i = blockIdx.y + int(gridDim.y) * warp; i < na; i += int(gridDim.y) * kDispWarps) {
-        const int slot = slot_s[i];
-        const int t = (a0 + i) / k;
-        if (slot >= 0) {
-            const uint4* src = reinterpret_cast<const uint4*>(x + size_t(t) * row_bytes);
-            uint4* dst = reinterpret_cast<uint4*>(xp + size_t(slot) * row_bytes);
-            for (int v = lane; v < vecs; v += 32) dst[v] = __ldg(src + v);
-        } else if (out_zero_dropped != nullptr) {
-            uint4* dst = reinterpret_cast<uint4*>(out_zero_dropped + size_t(t) * row_bytes);
-            for (int v = lane; v < vecs; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+    const int Y = int(gridDim.y), y = int(blockIdx.y);
+    const int my_rows = (na - y + Y - 1) / Y;
+    const int pieces = my_rows * vecs;
+    constexpr int U = 8;
+    for (int p0 = tid; p0 < pieces; p0 += kFwdThreads * U) {
+        uint4 val[U];
+        int row[U], vv[U], kind[U];   // kind 1: xp row, 2: zeroed output row of a dropped token
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            const int pc = p0 + j * kFwdThreads;
+            kind[j] = 0;
+            row[j] = 0;
+            vv[j] = 0;
+            if (pc < pieces) {
+                const int il = pc / vecs;
+                vv[j] = pc - il * vecs;
+                const int i = y + Y * il;
+                const int slot = slot_s[i];
+                const int t = (a0 + i) / k;
+                if (slot >= 0) {
+                    val[j] = __ldg(reinterpret_cast<const uint4*>(x + size_t(t) * row_bytes) + vv[j]);
+                    row[j] = slot;
+                    kind[j] = 1;
+                } else if (out_zero_dropped != nullptr) {
+                    val[j] = make_uint4(0u, 0u, 0u, 0u);
+                    row[j] = t;
+                    kind[j] = 2;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            if (kind[j] == 1) reinterpret_cast<uint4*>(xp + size_t(row[j]) * row_bytes)[vv[j]] = val[j];
+            else if (kind[j] == 2)
+                reinterpret_cast<uint4*>(out_zero_dropped + size_t(row[j]) * row_bytes)[vv[j]] = val[j];
         }
     }
 }
@@ -391,15 +443,19 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
     *reinterpret_cast<uint4*>(p) = u;
 }
 
+// One warp per token; each lane handles 16-byte pieces of the row, four at a
+// time, so 4 * k independent loads are in flight before the adds.
 template <typename T>
 __global__ void __launch_bounds__(256)
 combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
                int Tn, int k, int d, T* __restrict__ out) {
     pdl_wait();
     pdl_release();
+    constexpr int EPV = 16 / sizeof(T);   // elements per 16-byte piece
+    constexpr int U = 4;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int lane = threadIdx.x & 31;
-    const int chunks = d >> 3;
+    const int pieces = d / EPV;
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < Tn; t += warps_total) {
         int slot[MOE_MAX_TOPK];
         float w[MOE_MAX_TOPK];
@@ -408,17 +464,53 @@ combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, co
             slot[j] = (j < k) ? slot_of[size_t(t) * k + j] : -1;
             w[j] = (j < k && gate != nullptr) ? gate[size_t(t) * k + j] : 1.f;
         }
-        for (int c = lane; c < chunks; c += 32) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c0 = lane; c0 < pieces; c0 += 32 * U) {
+            float acc[U][EPV];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int i = 0; i < EPV; ++i) acc[u][i] = 0.f;
 #pragma unroll
             for (int j = 0; j < MOE_MAX_TOPK; ++j) {
                 if (slot[j] < 0) continue;
-                float v[8];
-                load8(yp + size_t(slot[j]) * d + c * 8, v);
+                uint4 raw[U];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w[j], v[i], acc[i]);
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * 32;
+                    raw[u] = (c < pieces) ? __ldg(reinterpret_cast<const uint4*>(yp + size_t(slot[j]) * d) + c)
+                                          : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    float v[8];
+                    if constexpr (sizeof(T) == 2) {
+                        v[0] = bf16_lo(raw[u].x); v[1] = bf16_hi(raw[u].x); v[2] = bf16_lo(raw[u].y);
+                        v[3] = bf16_hi(raw[u].y); v[4] = bf16_lo(raw[u].z); v[5] = bf16_hi(raw[u].z);
+                        v[6] = bf16_lo(raw[u].w); v[7] = bf16_hi(raw[u].w);
+                    } else {
+                        v[0] = __uint_as_float(raw[u].x); v[1] = __uint_as_float(raw[u].y);
+                        v[2] = __uint_as_float(raw[u].z); v[3] = __uint_as_float(raw[u].w);
+                    }
+#pragma unroll
+                    for (int i = 0; i < EPV; ++i) acc[u][i] = fmaf(w[j], v[i], acc[u][i]);
+                }
             }
-            store8(out + size_t(t) * d + c * 8, acc);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32;
+                if (c >= pieces) continue;
+                uint4 o;
+                if constexpr (sizeof(T) == 2) {
+                    o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+                    o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+                    o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+                    o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+                } else {
+                    o = make_uint4(__float_as_uint(acc[u][0]), __float_as_uint(acc[u][1]),
+                                   __float_as_uint(acc[u][2]), __float_as_uint(acc[u][3]));
+                }
+                reinterpret_cast<uint4*>(out + size_t(t) * d)[c] = o;
+            }
         }
     }
 }

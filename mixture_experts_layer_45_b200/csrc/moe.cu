@@ -150,12 +150,8 @@ int check_sizes(int T, int d, int ff, int E, int k, int dtype, bool need_ff) {
 
 struct WsLayout {
     size_t idx, gate, counts, offsets, perm, slot_of, row_gate, xp, h, yp;
-    size_t fhist, fbase, fpsum, rpart, total;   // per-router-chunk arrays of the fused forward path
+    size_t fhist, fbase, fpsum, total;   // per-router-chunk arrays of the forward path
 };
-
-// expert count padded for the router tile (16, 32, 64, 128 or 256)
-inline int router_ep(int E) { return E <= 16 ? 16 : E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256; }
-constexpr int kMaxRouterSplit = 4;
 
 // tokens per router CTA (= one dispatch chunk of the forward path)
 inline int router_chunk_tokens(int dtype) { return dtype == MOE_BF16 ? kRtBM : kRouterTM; }
@@ -188,8 +184,6 @@ WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype) {
     L.fhist = take(nchunk * E * 4);
     L.fbase = take(nchunk * E * 4);
     L.fpsum = take(nchunk * E * 4);
-    // split-K router partial logits: up to kMaxRouterSplit x [T, EP] fp32 (bf16 path only)
-    L.rpart = take(dtype == MOE_BF16 ? size_t(kMaxRouterSplit) * T * router_ep(E) * 4 : 0);
     L.total = o;
     return L;
 }
@@ -262,56 +256,31 @@ int launch_router_ep(const void* x, const void* wr, const float* bias, int T, in
     return L.finish(launch_err);
 }
 
-// K split of the tensor-core router: enough CTAs to stream x from most
-// SMs (each CTA keeps only ~8 TMA boxes in flight), at most kMaxRouterSplit,
-// at least two K blocks per slice; 1 when the tiles alone fill the GPU or
-// there is no workspace for partial logits.
-int router_split(int T, int d, bool have_part) {
-    if (!have_part) return 1;
-    const int tiles = ceil_div(T, kRtBM);
-    const int kblocks = ceil_div(d, 64);
-    if (4 * tiles >= 3 * num_sms()) return 1;
-    int split = ceil_div(num_sms(), tiles);
-    split = std::min(split, kMaxRouterSplit);
-    split = std::min(split, std::max(1, kblocks / 2));
-    return std::max(1, split);
-}
-
 template <int EP, int KMAX>
 int launch_router_tc(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                     float* gate, float* psum, float* psum_part, int32_t* hist, float* part, cudaStream_t s) {
+                     float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
     CUtensorMap tmX, tmW;
     if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), kRtBM)) return MOE_ERR_UNSUPPORTED;
     if (!make_map_2d(&tmW, wr, uint64_t(d), uint64_t(E), EP)) return MOE_ERR_UNSUPPORTED;
     auto kern = router_tc_kernel<EP, KMAX>;
     const size_t smem = RtCfg<EP>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
-    const int tiles = ceil_div(T, kRtBM);
-    const int split = router_split(T, d, part != nullptr);
-    int rc;
-    {
-        Launch L(MOE_KERNEL_ROUTER, s);
-        cudaError_t launch_err;
-        launch_err = launch_pdl(kern, dim3(tiles, split), dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k, idx,
-                                gate, psum, psum_part, hist, split > 1 ? part : static_cast<float*>(nullptr));
-        if ((rc = L.finish(launch_err)) != MOE_OK || split == 1) return rc;
-    }
-    Launch L(MOE_KERNEL_SELECT, s);
+    Launch L(MOE_KERNEL_ROUTER, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(router_select_kernel<EP, KMAX>, dim3(tiles), dim3(kRtBM), 0, s,
-                            static_cast<const float*>(part), split, bias, T, E, k, idx, gate, psum_part, hist);
+    launch_err = launch_pdl(kern, dim3(ceil_div(T, kRtBM)), dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k,
+                            idx, gate, psum, psum_part, hist);
     return L.finish(launch_err);
 }
 
 template <int KMAX>
 int launch_router_tc_k(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                       float* gate, float* psum, float* psum_part, int32_t* hist, float* part, cudaStream_t s) {
-    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
-    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
-    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
+                       float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
     if (E <= 128)
-        return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
-    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
+        return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
 }
 
 template <typename Tin>
@@ -324,20 +293,17 @@ int launch_router_t(const void* x, const void* wr, const float* bias, int T, int
     return launch_router_ep<Tin, 256>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
 }
 
-// bf16: tcgen05 router (128-token tiles, split over K when the tiles are
-// too few and `part` offers room for partial logits); f32: SIMT fp32 router
-// (32-token tiles).  prob_sum (atomic, zeroed here) or psum_part/hist (per
+// bf16: tcgen05 router (128-token tiles); f32: SIMT fp32 router (32-token tiles).  prob_sum (atomic, zeroed here) or psum_part/hist (per
 // tile) as requested.
 int run_router(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int dtype,
-               int32_t* idx, float* gate, float* psum, float* psum_part, int32_t* hist, float* part, cudaStream_t s) {
+               int32_t* idx, float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
     if (psum != nullptr && psum_part == nullptr &&
         cudaMemsetAsync(psum, 0, size_t(E) * sizeof(float), s) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (dtype == MOE_BF16) {
-        if (k == 1) return launch_router_tc_k<1>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
-        if (k == 2) return launch_router_tc_k<2>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part, s);
-        return launch_router_tc_k<MOE_MAX_TOPK>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, part,
-                                                s);
+        if (k == 1) return launch_router_tc_k<1>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+        if (k == 2) return launch_router_tc_k<2>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+        return launch_router_tc_k<MOE_MAX_TOPK>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
     }
     return launch_router_t<float>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
 }
@@ -375,7 +341,7 @@ int run_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int
         Launch L(MOE_KERNEL_GATHER, s);
         cudaError_t launch_err;
         launch_err = launch_pdl(dispatch_gather_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint8_t*>(x), row_bytes, perm, offsets, E, k,
-                                                    static_cast<uint8_t*>(xp));
+                                                    static_cast<uint8_t*>(xp), static_cast<const int32_t*>(nullptr), 0, static_cast<uint8_t*>(nullptr));
         if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
     }
     return MOE_OK;
@@ -589,7 +555,7 @@ int moe_router_topk(const void* x, const void* w_router, const float* logit_bias
     if (!x || !w_router || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
     return run_router(x, w_router, logit_bias, T, d, E, k, dtype, topk_idx, topk_gate, prob_sum, nullptr, nullptr,
-                      nullptr, static_cast<cudaStream_t>(stream));
+                      static_cast<cudaStream_t>(stream));
 }
 
 int moe_dispatch(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E, int capacity,
@@ -713,9 +679,7 @@ int moe_forward(const void* x, const void* w_router, const float* logit_bias, co
     // its token directly (rows of dropped tokens are zeroed by the dispatch)
     const bool direct = (k == 1);
 
-    float* rpart = dtype == MOE_BF16 ? reinterpret_cast<float*>(w + L.rpart) : nullptr;
-    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, idx, gate, nullptr, fpsum, fhist, rpart, s)) !=
-        MOE_OK)
+    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, idx, gate, nullptr, fpsum, fhist, s)) != MOE_OK)
         return rc;
     if ((rc = run_forward_dispatch(idx, gate, T, k, E, capacity, router_chunk_tokens(dtype), fhist, fpsum, fbase,
                                    counts, offsets, perm, slot_of, row_gate, stats, x, xp, d, dtype,

@@ -216,15 +216,12 @@ struct RtCfg {
     static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024;
 };
 
-// Split-K mode (gridDim.y > 1): CTA (tile, r) multiplies the r-th slice of
-// the K blocks and writes its raw partial logits to part[r][T][EP] (fp32,
-// no bias); router_select_kernel then finishes the tile.
 template <int EP, int KMAX>
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ bias, int T, int d, int E, int k, int32_t* __restrict__ topk_idx,
                  float* __restrict__ topk_gate, float* __restrict__ prob_sum, float* __restrict__ psum_part,
-                 int32_t* __restrict__ hist, float* __restrict__ part) {
+                 int32_t* __restrict__ hist) {
     using Cfg = RtCfg<EP>;
     constexpr int S = Cfg::kStages;
     constexpr int NCH = (EP + 31) / 32;   // 32-column TMEM chunks
@@ -261,11 +258,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     pdl_wait();
     pdl_release();
     const uint32_t tmem_base = tmem_slot;
-    const int KB_all = (d + 63) / 64;
-    const int split = gridDim.y, r_split = blockIdx.y;
-    const int kb_lo = int((long long)KB_all * r_split / split);
-    const int kb_hi = int((long long)KB_all * (r_split + 1) / split);
-    const int KB = kb_hi - kb_lo;
+    const int KB = (d + 63) / 64;
     const int t0 = blockIdx.x * kRtBM;
     volatile int* abort_p = &abort_flag;
 
@@ -279,8 +272,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) break;
                 uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
                 mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
-                tma_load_2d(sa, &tmX, &full_bar[stage], (kb_lo + kb) * 64, t0);
-                tma_load_2d(sa + Cfg::kABytes, &tmW, &full_bar[stage], (kb_lo + kb) * 64, 0);
+                tma_load_2d(sa, &tmX, &full_bar[stage], kb * 64, t0);
+                tma_load_2d(sa + Cfg::kABytes, &tmW, &full_bar[stage], kb * 64, 0);
                 last_parity[stage] = int(phase);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
@@ -323,27 +316,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const bool valid = t < T;
         const bool ok = mbar_wait(&done_bar, 0, abort_p);
         tc_fence_after();
-        if (part != nullptr) {
-            // split-K: hand the raw partial logits to router_select_kernel
-            float* dst = part + (size_t(r_split) * T + size_t(t)) * EP;
-#pragma unroll 1
-            for (int c = 0; c < NCH; ++c) {
-                uint32_t r[32];
-                __syncwarp();
-                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
-                tmem_ld_wait();
-                if (valid && ok) {
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        if (c * 32 + v * 4 < EP)
-                            *reinterpret_cast<float4*>(dst + c * 32 + v * 4) =
-                                make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                            __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-                    }
-                }
-            }
-            tc_fence_before();
-        } else {
         float m = -INFINITY, ssum = 0.f;
         float tv[KMAX];
         int ti[KMAX];
@@ -437,10 +409,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
         }
         tc_fence_before();
-        }   // full (non-split) mode
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E && part == nullptr; e += kRtThreads) {
+    for (int e = threadIdx.x; e < E; e += kRtThreads) {
         const float tot = ((s_col[0][e] + s_col[1][e]) + s_col[2][e]) + s_col[3][e];
         if (psum_part != nullptr) psum_part[size_t(blockIdx.x) * E + e] = tot;
         else if (prob_sum != nullptr) atomicAdd(prob_sum + e, tot);
@@ -449,117 +420,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);
-    }
-}
-
-// Finishes a split-K router tile: thread = token; sums the split partial
-// logits in split order, adds the bias, then the same online softmax,
-// register top-k, gates, expert histogram and probability column sums as
-// the full tensor-core epilogue.  One CTA per 128-token tile.
-template <int EP, int KMAX>
-__global__ void __launch_bounds__(kRtBM)
-router_select_kernel(const float* __restrict__ part, int split, const float* __restrict__ bias, int T, int E, int k,
-                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, float* __restrict__ psum_part,
-                     int32_t* __restrict__ hist) {
-    pdl_wait();
-    pdl_release();
-    constexpr int NCH = (EP + 31) / 32;
-    __shared__ int s_hist[EP];
-    __shared__ float s_col[4][NCH * 32];
-    __shared__ float s_tr[4][32][33];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int e = threadIdx.x; e < EP; e += kRtBM) s_hist[e] = 0;
-    __syncthreads();
-    const int t = blockIdx.x * kRtBM + threadIdx.x;
-    const bool valid = t < T;
-    auto load_chunk = [&](int c, float (&l)[32]) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) l[i] = 0.f;
-        if (!valid) return;
-        for (int r = 0; r < split; ++r) {
-            const float* src = part + (size_t(r) * T + size_t(t)) * EP + c * 32;
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                if (c * 32 + v * 4 < EP) {
-                    const float4 f = *reinterpret_cast<const float4*>(src + v * 4);
-                    l[4 * v] += f.x; l[4 * v + 1] += f.y; l[4 * v + 2] += f.z; l[4 * v + 3] += f.w;
-                }
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int e = c * 32 + i;
-            float v = (e < E) ? l[i] + (bias != nullptr ? bias[e] : 0.f) : -INFINITY;
-            l[i] = (v != v) ? -INFINITY : v;
-        }
-    };
-    float m = -INFINITY, ssum = 0.f;
-    float tv[KMAX];
-    int ti[KMAX];
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) { tv[j] = -INFINITY; ti[j] = 0x7fffffff; }
-#pragma unroll 1
-    for (int c = 0; c < NCH; ++c) {
-        float l[32];
-        load_chunk(c, l);
-        float cm = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) cm = fmaxf(cm, l[i]);
-        const float mn = fmaxf(m, cm);
-        if (mn != -INFINITY) {
-            float acc = (m == -INFINITY) ? 0.f : ssum * expf(m - mn);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc += (l[i] == -INFINITY) ? 0.f : expf(l[i] - mn);
-            ssum = acc;
-            m = mn;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            float v = l[i];
-            int ix = c * 32 + i;
-            if (v == -INFINITY || !(v > tv[KMAX - 1])) continue;
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                if (v > tv[j]) {
-                    const float tf = tv[j]; tv[j] = v; v = tf;
-                    const int tix = ti[j]; ti[j] = ix; ix = tix;
-                }
-            }
-        }
-    }
-    const float inv = 1.0f / ssum;
-    if (valid) {
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (j < k) {
-                int e = ti[j];
-                if (e >= E) e = j;
-                topk_idx[size_t(t) * k + j] = e;
-                topk_gate[size_t(t) * k + j] = (tv[j] == -INFINITY) ? 0.f : expf(tv[j] - m) * inv;
-                atomicAdd(&s_hist[e], 1);
-            }
-        }
-    }
-    if (psum_part != nullptr) {
-#pragma unroll 1
-        for (int c = 0; c < NCH; ++c) {
-            float l[32];
-            load_chunk(c, l);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s_tr[warp][lane][i] = (valid && l[i] != -INFINITY) ? expf(l[i] - m) * inv : 0.f;
-            __syncwarp();
-            float cs = 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) cs += s_tr[warp][i][lane];
-            s_col[warp][c * 32 + lane] = cs;
-            __syncwarp();
-        }
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kRtBM) {
-        if (psum_part != nullptr)
-            psum_part[size_t(blockIdx.x) * E + e] = ((s_col[0][e] + s_col[1][e]) + s_col[2][e]) + s_col[3][e];
-        if (hist != nullptr) hist[size_t(blockIdx.x) * E + e] = s_hist[e];
     }
 }
 

@@ -316,7 +316,8 @@ def test_forward_matches_oracle(w):
     (500, 64, 64, 8, 2, 0),          # capacity 0: every assignment dropped
     (2000, 128, 256, 16, 2, 60),     # capacity drops on a top-2 layer
     (1, 64, 64, 8, 2, -1),           # one token
-    (1000, 520, 256, 40, 3, 700),    # split-K router (bf16): uneven K slices, ragged last tile, k = 3
+    (1000, 520, 256, 40, 3, 700),    # ragged last router tile, K tail (520 = 8 * 64 + 8), k = 3
+    (600, 64, 64, 256, 8, -1),       # the most experts and slots: 256 experts, top-8
 ])
 def test_forward_edge_cases(dtype, T, d, ff, E, k, cap):
     inp = wl.draw_custom(5, T=T, d=d, ff=ff, E=E, dtype=dtype, router_std=0.5)
