@@ -250,6 +250,12 @@ MOE_API int moe_forward(const void* x, const void* w_router, const float* logit_
  * MOE_ERR_TIMEOUT, or MOE_ERR_CUDA if the synchronisation itself failed. */
 MOE_API int moe_get_error(void* stream);
 
+/* Device GELU forms, for testing: y[i] = GELU(x[i]) (x, y device float[n]).
+ * variant 0: 0.5 x (1 + erff(x / sqrt 2)), the fp32 path's form;
+ * variant 1: the same with erf by Abramowitz & Stegun eq. 7.1.26 (|error|
+ * <= 1.5e-7), the bf16 tensor-core epilogue's form. */
+MOE_API int moe_debug_gelu(const float* x, float* y, int n, int variant, void* stream);
+
 /* Number of kernels this library has launched in this process. */
 MOE_API uint64_t moe_launch_count(void);
 

@@ -62,6 +62,7 @@ _SIGS = {
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                          ctypes.c_size_t, _P]),
     "moe_get_error": (_I, [_P]),
+    "moe_debug_gelu": (_I, [_P, _P, _I, _I, _P]),
     "moe_launch_count": (ctypes.c_uint64, []),
     "moe_timing_enable": (_I, [_I]),
     "moe_timing_read": (_I, [_P, _P]),
@@ -196,6 +197,10 @@ def moe_forward(x, w_router, logit_bias, w1, b1, w2, b2, T, d, ff, E, k, capacit
 
 def moe_get_error(stream=None) -> int:
     return load().moe_get_error(_stream(stream))
+
+
+def moe_debug_gelu(x, y, n, variant, stream=None):
+    _check(load().moe_debug_gelu(_ptr(x), _ptr(y), n, variant, _stream(stream)), "moe_debug_gelu")
 
 
 def moe_launch_count() -> int:

@@ -71,9 +71,30 @@ template <> struct Elem<__nv_bfloat16> {
     }
 };
 
-// exact GELU, 0.5 v (1 + erf(v / sqrt 2)), with CUDA's erff
+// exact GELU, 0.5 v (1 + erf(v / sqrt 2)), with CUDA's erff (fp32 path)
 __device__ __forceinline__ float gelu_erf(float v) {
     return 0.5f * v * (1.0f + erff(v * 0.70710678118654752440f));
+}
+
+// erf(z) by Abramowitz & Stegun, Handbook of Mathematical Functions, eq.
+// 7.1.26: erf(a) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-a^2),
+// t = 1 / (1 + p a), a >= 0, |error| <= 1.5e-7; odd in z.  Branch-free, one
+// exponential and one reciprocal: used where the result is rounded to bf16.
+__device__ __forceinline__ float erf_as7126(float z) {
+    const float a = fabsf(z);
+    const float t = __fdividef(1.0f, fmaf(0.3275911f, a, 1.0f));
+    float poly = fmaf(1.061405429f, t, -1.453152027f);
+    poly = fmaf(poly, t, 1.421413741f);
+    poly = fmaf(poly, t, -0.284496736f);
+    poly = fmaf(poly, t, 0.254829592f);
+    poly *= t;
+    const float r = fmaf(-poly, __expf(-a * a), 1.0f);
+    return copysignf(r, z);
+}
+
+// GELU with the A&S erf (bf16 tensor-core epilogue)
+__device__ __forceinline__ float gelu_as(float v) {
+    return 0.5f * v * (1.0f + erf_as7126(v * 0.70710678118654752440f));
 }
 
 // ---------------------------------------------------------------------------

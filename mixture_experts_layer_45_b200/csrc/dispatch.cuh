@@ -515,6 +515,13 @@ combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, co
     }
 }
 
+// y[i] = GELU(x[i]) with the form the fp32 path uses (variant 0, erff) or the
+// bf16 tensor-core epilogue uses (variant 1, A&S 7.1.26); for testing.
+__global__ void gelu_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int variant) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        y[i] = variant == 0 ? gelu_erf(x[i]) : gelu_as(x[i]);
+}
+
 // ---------------------------------------------------------------------------
 // statistics (one CTA)
 // ---------------------------------------------------------------------------

@@ -382,7 +382,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const float cval = __uint_as_float(r[v * 8 + i]) + sbias[c * 32 + v * 8 + i];
-                        o[i] = (MODE == kFc1Gelu) ? gelu_erf(cval) : g * cval;
+                        o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
                     }
                     uint4 u;
                     u.x = pack_bf16x2(o[0], o[1]);

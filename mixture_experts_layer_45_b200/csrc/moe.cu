@@ -701,6 +701,15 @@ int moe_get_error(void* stream) {
     return v;
 }
 
+int moe_debug_gelu(const float* x, float* y, int n, int variant, void* stream) {
+    if (n < 0 || (variant != 0 && variant != 1)) return MOE_ERR_INVALID_ARG;
+    if (n == 0) return MOE_OK;
+    if (!x || !y) return MOE_ERR_INVALID_ARG;
+    gelu_probe_kernel<<<std::min(ceil_div(n, 256), 1024), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n,
+                                                                                                     variant);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int moe_timing_enable(int enable) {

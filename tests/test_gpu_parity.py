@@ -240,6 +240,24 @@ def test_grouped_ffn_tile_edges(dtype, sizes, d, ff):
     assert np.isnan(yp[R:]).all()          # rows past R are not written
 
 
+def test_device_gelu_forms_match_erf():
+    """Both device GELU forms against CUDA's erff form and the float64 definition:
+    the A&S 7.1.26 erf is within its published bound (1.5e-7) plus fp32 rounding."""
+    xs = np.concatenate([np.linspace(-12, 12, 200001), [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0]]).astype(np.float32)
+    x = torch.from_numpy(xs).to(DEV)
+    y0 = torch.empty_like(x)
+    y1 = torch.empty_like(x)
+    _lib.moe_debug_gelu(x, y0, x.numel(), 0)
+    _lib.moe_debug_gelu(x, y1, x.numel(), 1)
+    y0, y1 = y0.cpu().double().numpy(), y1.cpu().double().numpy()
+    ref = moe_ref.gelu(xs.astype(np.float64))
+    scale = np.maximum(np.abs(xs.astype(np.float64)), 1.0)
+    assert np.max(np.abs(y0 - ref) / scale) <= 2e-7
+    assert np.max(np.abs(y1 - ref) / scale) <= 0.5 * 1.5e-7 + 4e-7
+    assert np.max(np.abs(y1 - y0) / scale) <= 6e-7
+    assert y1[np.argmin(np.abs(xs))] == 0.0
+
+
 # ---------------------------------------------------------------------------
 # the whole layer (and step 4, combine)
 # ---------------------------------------------------------------------------
@@ -318,6 +336,8 @@ def test_forward_matches_oracle(w):
     (1, 64, 64, 8, 2, -1),           # one token
     (1000, 520, 256, 40, 3, 700),    # ragged last router tile, K tail (520 = 8 * 64 + 8), k = 3
     (600, 64, 64, 256, 8, -1),       # the most experts and slots: 256 experts, top-8
+    (2000, 256, 4096, 8, 1, -1),     # few tiles, long fc2 K, ragged rows
+    (1500, 256, 2048, 6, 2, 300),    # k = 2 with capacity drops, long fc2 K
 ])
 def test_forward_edge_cases(dtype, T, d, ff, E, k, cap):
     inp = wl.draw_custom(5, T=T, d=d, ff=ff, E=E, dtype=dtype, router_std=0.5)
