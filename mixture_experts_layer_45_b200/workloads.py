@@ -56,13 +56,15 @@ class Workload:
     seq_len: int = 0           # tokens per sequence for "seq_shift"
     seq_shift_std: float = 0.0
     zipf_bias: bool = False
+    shared: int = 0            # shared always-on experts (same shapes and init as the routed ones)
 
     def capacity_factor_label(self) -> str:
         return "none" if self.cf is None else f"{self.cf:g}"
 
     def describe(self) -> str:
         return (f"{self.name}: T={self.T} d={self.d} ff={self.ff} E={self.E} "
-                f"k={self.k} {self.dtype} cf={self.capacity_factor_label()}")
+                f"k={self.k} {self.dtype} cf={self.capacity_factor_label()}"
+                + (f" shared={self.shared}" if self.shared else ""))
 
 
 _BASE = {
@@ -188,35 +190,46 @@ def draw_inputs(w: Workload, T: Optional[int] = None) -> Dict[str, np.ndarray]:
 
     Keys: x [T,d], w_router [E,d], logit_bias [E] or None, w1 [E,ff,d],
     b1 [E,ff], w2 [E,d,ff], b2 [E,d] -- float32 (bf16-rounded for bf16).
+    With ``w.shared`` = S > 0 also shared_w1 [S,ff,d], shared_b1 [S,ff],
+    shared_w2 [S,d,ff], shared_b2 [S,d], drawn after the routed experts (so
+    the routed draws do not depend on S) with the same recipe.
     ``T`` overrides the token count (a prefix-independent redraw, used for
     ragged-size tests).
     """
     rng = np.random.Generator(np.random.PCG64(w.seed))
     out = _draw_router(rng, w, T)
-    E, d, ff = w.E, w.d, w.ff
+    w1, b1, w2, b2 = _draw_experts(rng, w, w.E)
+    out.update(w1=w1, b1=b1, w2=w2, b2=b2)
+    if w.shared > 0:
+        sw1, sb1, sw2, sb2 = _draw_experts(rng, w, w.shared)
+        out.update(shared_w1=sw1, shared_b1=sb1, shared_w2=sw2, shared_b2=sb2)
+    return out
+
+
+def _draw_experts(rng, w: Workload, n: int):
+    d, ff = w.d, w.ff
     if w.expert_init == "uniform":
-        w1 = _uniform(rng, (E, ff, d), d)
-        b1 = _uniform(rng, (E, ff), d)
-        w2 = _uniform(rng, (E, d, ff), ff)
-        b2 = _uniform(rng, (E, d), ff)
+        w1 = _uniform(rng, (n, ff, d), d)
+        b1 = _uniform(rng, (n, ff), d)
+        w2 = _uniform(rng, (n, d, ff), ff)
+        b2 = _uniform(rng, (n, d), ff)
     elif w.expert_init == "normal002":
-        w1 = _normal(rng, (E, ff, d), 0.02)
-        b1 = np.zeros((E, ff), np.float32)
-        w2 = _normal(rng, (E, d, ff), 0.02)
-        b2 = np.zeros((E, d), np.float32)
+        w1 = _normal(rng, (n, ff, d), 0.02)
+        b1 = np.zeros((n, ff), np.float32)
+        w2 = _normal(rng, (n, d, ff), 0.02)
+        b2 = np.zeros((n, d), np.float32)
     else:
         raise ValueError(w.expert_init)
     if w.dtype == "bf16":
         w1, b1, w2, b2 = (round_to_bf16(a) for a in (w1, b1, w2, b2))
-    out.update(w1=w1, b1=b1, w2=w2, b2=b2)
-    return out
+    return w1, b1, w2, b2
 
 
 def draw_custom(seed: int, T: int, d: int, ff: int, E: int, dtype: str,
-                router_std: float = 0.1, x_scale: float = 1.0) -> Dict[str, np.ndarray]:
+                router_std: float = 0.1, x_scale: float = 1.0, shared: int = 0) -> Dict[str, np.ndarray]:
     """Small arbitrary-shape inputs for edge-case and brute-force tests."""
     w = Workload(name="custom", T=T, d=d, ff=ff, E=E, k=1, dtype=dtype, cf=None,
-                 seed=seed, router_std=router_std, expert_init="uniform")
+                 seed=seed, router_std=router_std, expert_init="uniform", shared=shared)
     out = draw_inputs(w)
     if x_scale != 1.0:
         x = out["x"] * np.float32(x_scale)

@@ -38,6 +38,15 @@ notes of the repository):
   ascending order.
 * softmax is evaluated with the row maximum subtracted (the same function).
 
+Shared always-on experts (notebook section "Exercises", item 3: DeepSeek-V2
+keeps a small set of experts that every token uses beside the routed ones;
+the exercise asks to extend the forward with them).  Readings: every token
+passes through every shared expert and its output is added with weight 1
+(no gate); shared experts have the routed experts' form and shapes
+(fc2(gelu(fc1(x))), d -> ff -> d, biased); they are outside the router, the
+capacity limit and the statistics, so a token whose routed assignments are
+all dropped still receives the shared experts' sum.
+
 Every function below works in float64 on whatever values it is given; bf16
 workloads pass the bf16-rounded values the GPU also receives.
 
@@ -284,6 +293,36 @@ def combine(yp, slot_of, T: int, k: int, topk_gate=None) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Shared always-on experts (notebook section "Exercises", item 3)
+# ---------------------------------------------------------------------------
+
+def has_shared(params) -> bool:
+    return params.get("shared_w1") is not None and np.asarray(params["shared_w1"]).shape[0] > 0
+
+
+def shared_expert_outputs(x, params) -> np.ndarray:
+    """Ys[s] = shared expert s applied to every token: [S, T, d]."""
+    x = np.asarray(x, np.float64)
+    S = np.asarray(params["shared_w1"]).shape[0]
+    return np.stack([expert_ffn(x, params["shared_w1"][s], params["shared_b1"][s],
+                                params["shared_w2"][s], params["shared_b2"][s]) for s in range(S)])
+
+
+def shared_experts(x, params) -> np.ndarray:
+    """Sum over the shared experts of their outputs, weight 1, every token: [T, d]."""
+    return shared_expert_outputs(x, params).sum(axis=0)
+
+
+def moe_forward_rows_shared(x, params, topk_idx, topk_gate, slot_of, rows) -> np.ndarray:
+    """Output rows ``rows`` of the layer with shared experts (routed part
+    from moe_forward_rows; the shared experts act on each token alone)."""
+    out = moe_forward_rows(x, params, topk_idx, topk_gate, slot_of, rows)
+    if has_shared(params):
+        out = out + shared_experts(np.asarray(x)[np.asarray(rows)], params)
+    return out
+
+
+# ---------------------------------------------------------------------------
 # Switch auxiliary loss and the layer's statistics
 # (notebook sections "Switch Transformer auxiliary loss" and "Capacity factor")
 # ---------------------------------------------------------------------------
@@ -320,11 +359,19 @@ def layer_stats(topk_idx, gates, E: int, cap: int) -> Dict[str, float]:
 # ---------------------------------------------------------------------------
 
 def moe_layer(inputs, k: int, cap: int) -> Dict[str, np.ndarray]:
-    """Router -> dispatch -> expert FFN -> combine, all in float64."""
+    """Router -> dispatch -> expert FFN -> combine, all in float64.
+
+    With shared experts in ``inputs`` (keys shared_w1 [S,ff,d], shared_b1
+    [S,ff], shared_w2 [S,d,ff], shared_b2 [S,d]) their ungated sum over all
+    tokens is added to the routed output; routing and statistics are those
+    of the routed experts alone.
+    """
     r = route(inputs["x"], inputs["w_router"], k, inputs.get("logit_bias"))
     E = inputs["w_router"].shape[0]
     dsp = dispatch(r["topk_idx"], E, cap)
     out = moe_forward(inputs["x"], inputs, r["topk_idx"], r["topk_gate"], dsp["slot_of"])
+    if has_shared(inputs):
+        out = out + shared_experts(inputs["x"], inputs)
     r.update(dsp)
     r["out"] = out
     r["stats"] = layer_stats(r["topk_idx"], r["gates"], E, cap)

@@ -241,6 +241,84 @@ def test_forward_bf16_rounded_inputs_brute_force():
 
 
 # ---------------------------------------------------------------------------
+# shared always-on experts (notebook section "Exercises", item 3)
+# ---------------------------------------------------------------------------
+
+def _torch_mlp(x, w1, b1, w2, b2):
+    """fc2(gelu(fc1(x))) with torch's float64 Linear and exact GELU."""
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))
+    h = F.gelu(F.linear(t(x), t(w1), t(b1)))
+    return F.linear(h, t(w2), t(b2)).numpy()
+
+
+def _routed_only(inp):
+    return {key: v for key, v in inp.items() if not key.startswith("shared_")}
+
+
+def check_shared_experts_added_ungated(inp, k, cap):
+    """With shared experts the output gains, on every token (dropped or not),
+    the plain sum of the shared MLPs; routing, dispatch and statistics are
+    those of the routed layer alone."""
+    res = moe_ref.moe_layer(inp, k=k, cap=cap)
+    base = moe_ref.moe_layer(_routed_only(inp), k=k, cap=cap)
+    S = inp["shared_w1"].shape[0]
+    ref = sum(_torch_mlp(inp["x"], inp["shared_w1"][s], inp["shared_b1"][s],
+                         inp["shared_w2"][s], inp["shared_b2"][s]) for s in range(S))
+    np.testing.assert_allclose(res["out"] - base["out"], ref, rtol=0, atol=1e-12)
+    for key in ("topk_idx", "topk_gate", "perm", "slot_of", "offsets", "counts"):
+        assert np.array_equal(res[key], base[key]), key
+    assert res["stats"] == base["stats"]
+    # per-expert outputs, in order
+    ys = moe_ref.shared_expert_outputs(inp["x"], inp)
+    assert ys.shape == (S,) + inp["x"].shape
+    for s in range(S):
+        np.testing.assert_allclose(ys[s], _torch_mlp(inp["x"], inp["shared_w1"][s], inp["shared_b1"][s],
+                                                     inp["shared_w2"][s], inp["shared_b2"][s]),
+                                   rtol=0, atol=1e-12)
+    return res, ref
+
+
+@pytest.mark.parametrize("k,cap,S", [(1, -1, 1), (2, -1, 2), (2, 5, 2), (1, 4, 3)])
+def test_shared_experts_add_plain_mlps(k, cap, S):
+    inp = wl.draw_custom(30 + S, T=48, d=24, ff=40, E=6, dtype="f32", router_std=0.3, shared=S)
+    res, ref = check_shared_experts_added_ungated(inp, k, cap)
+    if cap >= 0:
+        dropped_all = (res["slot_of"].reshape(-1, k) < 0).all(1)
+        assert dropped_all.any()
+        # a token with every assignment dropped receives exactly the shared sum
+        np.testing.assert_allclose(res["out"][dropped_all], ref[dropped_all], rtol=0, atol=1e-12)
+
+
+def test_shared_experts_with_zero_capacity_is_shared_sum():
+    inp = wl.draw_custom(41, T=20, d=16, ff=24, E=4, dtype="bf16", router_std=0.3, shared=2)
+    res = moe_ref.moe_layer(inp, k=2, cap=0)
+    assert (res["slot_of"] < 0).all()
+    np.testing.assert_allclose(res["out"], moe_ref.shared_experts(inp["x"], inp), rtol=0, atol=0)
+    check_shared_experts_added_ungated(inp, 2, 0)
+
+
+def test_shared_expert_equals_routed_single_expert_layer():
+    """A shared expert is the E = 1, k = 1 routed layer (gate softmax over one
+    expert = 1, no capacity) with the same weights."""
+    inp = wl.draw_custom(43, T=32, d=16, ff=24, E=3, dtype="f32", router_std=0.3, shared=2)
+    for s in range(2):
+        single = {"x": inp["x"], "w_router": inp["w_router"][:1], "logit_bias": None,
+                  "w1": inp["shared_w1"][s:s + 1], "b1": inp["shared_b1"][s:s + 1],
+                  "w2": inp["shared_w2"][s:s + 1], "b2": inp["shared_b2"][s:s + 1]}
+        np.testing.assert_allclose(moe_ref.shared_expert_outputs(inp["x"], inp)[s],
+                                   moe_ref.moe_layer(single, k=1, cap=-1)["out"], rtol=0, atol=1e-12)
+
+
+def test_shared_rows_match_full_layer():
+    inp = wl.draw_custom(44, T=40, d=16, ff=24, E=5, dtype="f32", router_std=0.3, shared=2)
+    res = moe_ref.moe_layer(inp, k=2, cap=6)
+    rows = np.array([0, 7, 39])
+    np.testing.assert_allclose(
+        moe_ref.moe_forward_rows_shared(inp["x"], inp, res["topk_idx"], res["topk_gate"], res["slot_of"], rows),
+        res["out"][rows], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
 # Switch auxiliary loss
 # ---------------------------------------------------------------------------
 
@@ -348,9 +426,20 @@ def _transposed_w1(x_e, w1_e, b1_e):
     return moe_ref.gelu(np.asarray(x_e, np.float64) @ w.T + np.asarray(b1_e)[None, :])
 
 
+def _shared_mean_not_sum(x, params):
+    return moe_ref.shared_expert_outputs(x, params).mean(axis=0)
+
+
+def _shared_without_fc2_bias(x, params):
+    p = dict(params)
+    p["shared_b2"] = np.zeros_like(np.asarray(params["shared_b2"]))
+    return _ORIG_SHARED_OUT(x, p)
+
+
 _ORIG_ROUTE = moe_ref.route
 _ORIG_DISPATCH = moe_ref.dispatch
 _ORIG_AUX = moe_ref.switch_aux_loss
+_ORIG_SHARED_OUT = moe_ref.shared_expert_outputs
 
 MUTATIONS = {
     "tanh-gelu": ("gelu", _tanh_gelu, lambda: check_gelu(moe_ref.gelu)),
@@ -365,6 +454,13 @@ MUTATIONS = {
                             lambda: check_softmax_vs_library(np.random.default_rng(0).normal(size=(5, 4)))),
     "aux-loss-missing-E": ("switch_aux_loss", _aux_without_E, lambda: check_aux_balanced_closed_form(64, 2, 8)),
     "w1-transposed": ("fc1_gelu", _transposed_w1, lambda: check_single_expert_is_mlp(_tiny(5, E=1))),
+    "shared-averaged": ("shared_experts", _shared_mean_not_sum,
+                        lambda: check_shared_experts_added_ungated(
+                            wl.draw_custom(32, T=24, d=16, ff=24, E=4, dtype="f32", router_std=0.3, shared=2), 2, 5)),
+    "shared-fc2-bias-dropped": ("shared_expert_outputs", _shared_without_fc2_bias,
+                                lambda: check_shared_experts_added_ungated(
+                                    wl.draw_custom(33, T=24, d=16, ff=24, E=4, dtype="f32", router_std=0.3,
+                                                   shared=1), 1, -1)),
 }
 
 

@@ -56,3 +56,19 @@ def test_workload_table():
     assert len(names) == 8
     with pytest.raises(KeyError):
         wl.workload("nope")
+
+
+def test_shared_expert_draws_follow_the_routed_ones():
+    """Adding shared experts leaves every routed draw unchanged and gives the
+    shared experts the routed experts' shapes and bf16 rounding."""
+    base = wl.draw_inputs(wl.workload("switch-top1"), T=64)
+    w = wl.workload("switch-top1", shared=2)
+    got = wl.draw_inputs(w, T=64)
+    for key, v in base.items():
+        if v is not None:
+            assert np.array_equal(got[key], v), key
+    assert got["shared_w1"].shape == (2, w.ff, w.d) and got["shared_b1"].shape == (2, w.ff)
+    assert got["shared_w2"].shape == (2, w.d, w.ff) and got["shared_b2"].shape == (2, w.d)
+    for key in ("shared_w1", "shared_b1", "shared_w2", "shared_b2"):
+        assert np.array_equal(wl.round_to_bf16(got[key]), got[key])
+    assert not np.array_equal(got["shared_w1"][0], got["w1"][0])
