@@ -183,6 +183,83 @@ def dispatch(topk_idx, E: int, cap: int) -> Dict[str, np.ndarray]:
 
 
 # ---------------------------------------------------------------------------
+# Overflow rerouting instead of dropping (the blog "MoE Parallelism for
+# Inference", section "Common Bottlenecks", item 1, on sending rejected
+# tokens to less busy experts; the cookbook notebook, section "What": the
+# overflow is dropped or sent to a fallback path)
+# ---------------------------------------------------------------------------
+
+def reroute_offers(ranked_idx, served, k: int, r: int):
+    """Round r's offers, in the order experts see them (token order): for each
+    token with an unserved slot, (t, its first unserved slot j, its (k+r)-th
+    expert)."""
+    offers = []
+    for t in range(served.shape[0]):
+        waiting = [j for j in range(k) if not served[t, j]]
+        if waiting:
+            offers.append((t, waiting[0], int(ranked_idx[t, k + r - 1])))
+    return offers
+
+
+def dispatch_reroute(ranked_idx, ranked_gate, k: int, E: int, cap: int, rounds: int) -> Dict[str, np.ndarray]:
+    """Dispatch with up to ``rounds`` rerouting rounds for dropped assignments.
+
+    ranked_idx / ranked_gate [T, k + rounds]: each token's experts in the
+    router's order (largest logit first) and their softmax gates; the first
+    k are the token's assignments, the rest its fallback experts.
+
+    Readings (the pages name the idea, not the rule): first the plain
+    dispatch (each expert keeps its first ``cap`` assignments in token
+    order).  Then in round r = 1 .. rounds, every token that still has a
+    dropped assignment offers its first such slot j to its (k+r)-th expert
+    c = ranked_idx[t, k+r-1]; each expert accepts offers in token order while
+    it holds fewer than ``cap`` rows.  An accepted slot is served by c with
+    gate ranked_gate[t, k+r-1].  Expert e's rows are its own kept
+    assignments in token order, then those it accepted in round 1 (token
+    order), round 2, and so on.  A token never gets an expert twice: the
+    fallbacks differ from its first k experts and from each other.
+
+    Returns the keys of ``dispatch`` (counts are the router's choices before
+    any drop; kept and offsets are final) plus
+      final_idx / final_gate [T, k]  the expert and gate serving each slot
+      kept_primary [E]               rows each expert kept from its own choices
+      rerouted                       assignments served by a fallback expert
+    """
+    ranked_idx = np.asarray(ranked_idx)
+    ranked_gate = np.asarray(ranked_gate, np.float64)
+    T = ranked_idx.shape[0]
+    if ranked_idx.shape[1] < k + rounds:
+        raise ValueError("ranked_idx needs k + rounds columns")
+    idx = ranked_idx[:, :k]
+    base = dispatch(idx, E, cap)
+    final_idx = idx.copy()
+    final_gate = ranked_gate[:, :k].copy()
+    served = (base["slot_of"].reshape(T, k) >= 0)
+    # members[e]: assignments served by e, in row order
+    members = [[a for a in base["perm"][base["offsets"][e]:base["offsets"][e + 1]]] for e in range(E)]
+    load = np.array([len(m) for m in members], dtype=np.int64)
+    rerouted = 0
+    if cap >= 0:
+        for r in range(1, rounds + 1):
+            for t, j, c in reroute_offers(ranked_idx, served, k, r):
+                if load[c] < cap:
+                    load[c] += 1
+                    members[c].append(t * k + j)
+                    served[t, j] = True
+                    final_idx[t, j] = c
+                    final_gate[t, j] = ranked_gate[t, k + r - 1]
+                    rerouted += 1
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(load)
+    perm = np.array([a for e in range(E) for a in members[e]], dtype=np.int64)
+    slot_of = np.full(T * k, -1, dtype=np.int64)
+    slot_of[perm] = np.arange(len(perm))
+    return {"counts": base["counts"], "kept": load, "kept_primary": base["kept"], "offsets": offsets,
+            "perm": perm, "slot_of": slot_of, "drop_mask": (slot_of < 0).astype(np.uint8),
+            "final_idx": final_idx, "final_gate": final_gate, "rerouted": rerouted}
+
+
+# ---------------------------------------------------------------------------
 # Expert FFN and gated combine (notebook section "Dispatch and gather")
 # ---------------------------------------------------------------------------
 
@@ -338,19 +415,24 @@ def switch_aux_loss(topk_idx, gates, E: int) -> float:
     return float(E * (f * p).sum())
 
 
-def layer_stats(topk_idx, gates, E: int, cap: int) -> Dict[str, float]:
-    """The layer's reported statistics from its routing."""
+def layer_stats(topk_idx, gates, E: int, cap: int, slot_of=None) -> Dict[str, float]:
+    """The layer's reported statistics from its routing (the router's own
+    choices).  With ``slot_of`` from a rerouting dispatch, rows_kept,
+    dropped and drop_rate count the assignments served after rerouting and
+    ``rerouted`` those served by a fallback expert."""
     idx = np.asarray(topk_idx)
     T, k = idx.shape
     counts = token_count_per_expert(idx, E)
     kept = counts if cap < 0 else np.minimum(counts, cap)
+    served = int(kept.sum()) if slot_of is None else int((np.asarray(slot_of) >= 0).sum())
     return {
         "aux_loss": switch_aux_loss(idx, gates, E),
         "imbalance": imbalance(counts, T, k, E),
-        "drop_rate": drop_rate(counts, cap),
-        "rows_kept": int(kept.sum()),
+        "drop_rate": (T * k - served) / (T * k) if T * k else 0.0,
+        "rows_kept": served,
         "max_count": int(counts.max()),
-        "dropped": int((counts - kept).sum()),
+        "dropped": T * k - served,
+        "rerouted": served - int(kept.sum()),
     }
 
 
@@ -358,21 +440,30 @@ def layer_stats(topk_idx, gates, E: int, cap: int) -> Dict[str, float]:
 # Whole layer
 # ---------------------------------------------------------------------------
 
-def moe_layer(inputs, k: int, cap: int) -> Dict[str, np.ndarray]:
+def moe_layer(inputs, k: int, cap: int, reroute: int = 0) -> Dict[str, np.ndarray]:
     """Router -> dispatch -> expert FFN -> combine, all in float64.
 
     With shared experts in ``inputs`` (keys shared_w1 [S,ff,d], shared_b1
     [S,ff], shared_w2 [S,d,ff], shared_b2 [S,d]) their ungated sum over all
     tokens is added to the routed output; routing and statistics are those
-    of the routed experts alone.
+    of the routed experts alone.  ``reroute`` > 0 gives dropped assignments
+    that many rounds of fallback experts (dispatch_reroute).
     """
-    r = route(inputs["x"], inputs["w_router"], k, inputs.get("logit_bias"))
     E = inputs["w_router"].shape[0]
-    dsp = dispatch(r["topk_idx"], E, cap)
-    out = moe_forward(inputs["x"], inputs, r["topk_idx"], r["topk_gate"], dsp["slot_of"])
+    if reroute <= 0:
+        r = route(inputs["x"], inputs["w_router"], k, inputs.get("logit_bias"))
+        dsp = dispatch(r["topk_idx"], E, cap)
+        out = moe_forward(inputs["x"], inputs, r["topk_idx"], r["topk_gate"], dsp["slot_of"])
+    else:
+        r = route(inputs["x"], inputs["w_router"], k + reroute, inputs.get("logit_bias"))
+        ranked_idx, ranked_gate = r["topk_idx"], r["topk_gate"]
+        r["ranked_idx"], r["ranked_gate"] = ranked_idx, ranked_gate
+        r["topk_idx"], r["topk_gate"] = ranked_idx[:, :k], ranked_gate[:, :k]
+        dsp = dispatch_reroute(ranked_idx, ranked_gate, k, E, cap, reroute)
+        out = moe_forward(inputs["x"], inputs, dsp["final_idx"], dsp["final_gate"], dsp["slot_of"])
     if has_shared(inputs):
         out = out + shared_experts(inputs["x"], inputs)
     r.update(dsp)
     r["out"] = out
-    r["stats"] = layer_stats(r["topk_idx"], r["gates"], E, cap)
+    r["stats"] = layer_stats(r["topk_idx"], r["gates"], E, cap, slot_of=dsp["slot_of"])
     return r

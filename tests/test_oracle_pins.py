@@ -319,6 +319,157 @@ def test_shared_rows_match_full_layer():
 
 
 # ---------------------------------------------------------------------------
+# overflow rerouting (dispatch_reroute)
+# ---------------------------------------------------------------------------
+
+def _ranked(rows):
+    idx = np.array(rows, dtype=np.int64)
+    gate = (idx + 1) / 100.0 + np.arange(idx.shape[0])[:, None] / 1000.0   # distinct, traceable gates
+    return idx, gate
+
+
+def check_reroute_hand_example_top1():
+    """Worked by hand.  E = 4, k = 1, cap = 2, two rounds.
+    Own choices: tokens 0-4 pick expert 0, token 5 expert 1, token 6 expert 2.
+    Expert 0 keeps tokens 0, 1 and drops 2, 3, 4 (loads 2, 1, 1, 0).
+    Round 1 offers (second choices): t2 -> 1 (accepted, load 2), t3 -> 1
+    (full), t4 -> 2 (accepted, load 2).  Round 2: t3 -> its third choice 3
+    (accepted).  Rows: e0 [t0 t1], e1 [t5 t2], e2 [t6 t4], e3 [t3]."""
+    idx, gate = _ranked([[0, 1, 2], [0, 1, 2], [0, 1, 2], [0, 1, 3], [0, 2, 1], [1, 0, 2], [2, 0, 1]])
+    res = moe_ref.dispatch_reroute(idx, gate, 1, 4, 2, 2)
+    np.testing.assert_array_equal(res["perm"], [0, 1, 5, 2, 6, 4, 3])
+    np.testing.assert_array_equal(res["offsets"], [0, 2, 4, 6, 7])
+    np.testing.assert_array_equal(res["slot_of"], [0, 1, 3, 6, 5, 2, 4])
+    np.testing.assert_array_equal(res["final_idx"][:, 0], [0, 0, 1, 3, 2, 1, 2])
+    np.testing.assert_array_equal(res["final_gate"][:, 0],
+                                  [gate[0, 0], gate[1, 0], gate[2, 1], gate[3, 2], gate[4, 1], gate[5, 0], gate[6, 0]])
+    np.testing.assert_array_equal(res["counts"], [5, 1, 1, 0])
+    np.testing.assert_array_equal(res["kept_primary"], [2, 1, 1, 0])
+    assert res["rerouted"] == 3 and res["drop_mask"].sum() == 0
+    # one round only: token 3 stays dropped
+    one = moe_ref.dispatch_reroute(idx, gate, 1, 4, 2, 1)
+    np.testing.assert_array_equal(one["slot_of"], [0, 1, 3, -1, 5, 2, 4])
+    assert one["rerouted"] == 2
+
+
+def check_reroute_hand_example_top2():
+    """Worked by hand.  E = 4, k = 2, cap = 1, two rounds.  Tokens 0 and 1
+    choose (0, 1) with fallbacks (2, 3); token 2 chooses (1, 0), fallbacks
+    (3, 2).  Kept: a0 = (t0, slot 0) at expert 0, a1 = (t0, 1) at expert 1.
+    Round 1: t1 offers its first dropped slot (slot 0) to expert 2
+    (accepted); t2 offers slot 0 to expert 3 (accepted).  Round 2: t1 offers
+    slot 1 to expert 3, t2 slot 1 to expert 2: both full."""
+    idx, gate = _ranked([[0, 1, 2, 3], [0, 1, 2, 3], [1, 0, 3, 2]])
+    res = moe_ref.dispatch_reroute(idx, gate, 2, 4, 1, 2)
+    np.testing.assert_array_equal(res["perm"], [0, 1, 2, 4])
+    np.testing.assert_array_equal(res["offsets"], [0, 1, 2, 3, 4])
+    np.testing.assert_array_equal(res["slot_of"], [0, 1, 2, -1, 3, -1])
+    np.testing.assert_array_equal(res["final_idx"], [[0, 1], [2, 1], [3, 0]])
+    assert res["final_gate"][1, 0] == gate[1, 2] and res["final_gate"][2, 0] == gate[2, 2]
+    assert res["rerouted"] == 2
+
+
+def test_reroute_hand_worked_examples():
+    check_reroute_hand_example_top1()
+    check_reroute_hand_example_top2()
+
+
+def _random_ranked(seed, T, E, kk):
+    rng = np.random.default_rng(seed)
+    p = rng.dirichlet(np.ones(E) * 0.4)
+    idx = np.stack([rng.choice(E, size=kk, replace=False, p=p) for _ in range(T)])
+    return idx, rng.random((T, kk))
+
+
+@pytest.mark.parametrize("T,E,k,cap,rounds,seed", [(200, 8, 1, 20, 1, 0), (300, 6, 2, 70, 3, 1),
+                                                   (150, 16, 1, 3, 4, 2), (100, 5, 3, 40, 2, 3),
+                                                   (64, 4, 1, 0, 2, 4)])
+def test_reroute_invariants(T, E, k, cap, rounds, seed):
+    idx, gate = _random_ranked(seed, T, E, k + rounds)
+    res = moe_ref.dispatch_reroute(idx, gate, k, E, cap, rounds)
+    base = moe_ref.dispatch(idx[:, :k], E, cap)
+    # the router's choices are dispatched as before; rerouting only adds rows
+    np.testing.assert_array_equal(res["counts"], base["counts"])
+    np.testing.assert_array_equal(res["kept_primary"], base["kept"])
+    assert np.all(res["kept"] <= cap) and np.all(res["kept"] >= base["kept"])
+    np.testing.assert_array_equal(np.diff(res["offsets"]), res["kept"])
+    served = res["slot_of"] >= 0
+    assert np.all(served[base["slot_of"] >= 0])
+    assert res["rerouted"] == int(served.sum() - (base["slot_of"] >= 0).sum())
+    assert sorted(res["perm"]) == sorted(np.nonzero(served)[0])
+    fi = res["final_idx"]
+    for t in range(T):
+        used = [fi[t, j] for j in range(k) if served[t * k + j]]
+        assert len(set(used)) == len(used)            # never the same expert twice
+    # each row belongs to its expert; within an expert: own rows in token
+    # order first, then rerouted rows by (round, token)
+    for e in range(E):
+        rows = res["perm"][res["offsets"][e]:res["offsets"][e + 1]]
+        keys = []
+        for a in rows:
+            t, j = divmod(int(a), k)
+            assert fi[t, j] == e
+            pos = list(idx[t]).index(e)
+            rnd = 0 if pos < k else pos - k + 1
+            assert rnd == 0 or res["final_gate"][t, j] == gate[t, pos]
+            keys.append((rnd, t))
+        assert keys == sorted(keys)
+    # an offer is refused only when the expert is full by the end of its round
+    if cap == 0:
+        assert res["rerouted"] == 0 and not served.any()
+
+
+def test_reroute_one_round_top1_closed_form():
+    """k = 1, one round: expert c takes, in token order, the first
+    cap - kept_c dropped tokens whose second choice is c (a stable sort)."""
+    T, E, cap = 500, 10, 35
+    idx, gate = _random_ranked(7, T, E, 2)
+    res = moe_ref.dispatch_reroute(idx, gate, 1, E, cap, 1)
+    base = moe_ref.dispatch(idx[:, :1], E, cap)
+    dropped = np.nonzero(base["slot_of"] < 0)[0]
+    second = idx[dropped, 1]
+    order = np.argsort(second, kind="stable")
+    expect = np.zeros(T, bool)
+    for c in range(E):
+        mine = dropped[order][second[order] == c]
+        expect[mine[:cap - base["kept"][c]]] = True
+    np.testing.assert_array_equal((res["slot_of"] >= 0) & (base["slot_of"] < 0), expect)
+
+
+def test_reroute_degenerate_cases():
+    idx, gate = _random_ranked(9, 120, 6, 4)
+    base = moe_ref.dispatch(idx[:, :2], 6, 25)
+    zero = moe_ref.dispatch_reroute(idx, gate, 2, 6, 25, 0)
+    for key in ("counts", "offsets", "perm", "slot_of", "drop_mask"):
+        np.testing.assert_array_equal(zero[key], base[key])
+    unlimited = moe_ref.dispatch_reroute(idx, gate, 2, 6, -1, 2)
+    plain = moe_ref.dispatch(idx[:, :2], 6, -1)
+    np.testing.assert_array_equal(unlimited["perm"], plain["perm"])
+    assert unlimited["rerouted"] == 0
+
+
+def check_reroute_forward_vs_brute_force(inp, k, cap, rounds):
+    res = moe_ref.moe_layer(inp, k=k, cap=cap, reroute=rounds)
+    ref = brute_force_dense(inp, res["final_idx"], res["final_gate"], res["slot_of"])
+    np.testing.assert_allclose(res["out"], ref, rtol=0, atol=1e-12)
+    # the router's full softmax gives the fallback gates
+    np.testing.assert_allclose(res["final_gate"], np.take_along_axis(res["gates"], res["final_idx"], 1),
+                               rtol=0, atol=0)
+    st = res["stats"]
+    assert st["rows_kept"] == int((res["slot_of"] >= 0).sum()) and st["rerouted"] == res["rerouted"]
+    plain = moe_ref.moe_layer(inp, k=k, cap=cap)
+    assert st["dropped"] <= plain["stats"]["dropped"]
+    assert st["aux_loss"] == plain["stats"]["aux_loss"] and st["imbalance"] == plain["stats"]["imbalance"]
+    return res
+
+
+@pytest.mark.parametrize("k,cap,rounds", [(1, 7, 1), (2, 14, 2), (1, 6, 3)])
+def test_reroute_forward_matches_brute_force(k, cap, rounds):
+    res = check_reroute_forward_vs_brute_force(_tiny(50 + k), k, cap, rounds)
+    assert res["rerouted"] > 0
+
+
+# ---------------------------------------------------------------------------
 # Switch auxiliary loss
 # ---------------------------------------------------------------------------
 
@@ -436,10 +587,19 @@ def _shared_without_fc2_bias(x, params):
     return _ORIG_SHARED_OUT(x, p)
 
 
+def _offers_reverse_token_order(ranked_idx, served, k, r):
+    return _ORIG_OFFERS(ranked_idx, served, k, r)[::-1]
+
+
+def _offers_always_first_fallback(ranked_idx, served, k, r):
+    return _ORIG_OFFERS(ranked_idx, served, k, 1)
+
+
 _ORIG_ROUTE = moe_ref.route
 _ORIG_DISPATCH = moe_ref.dispatch
 _ORIG_AUX = moe_ref.switch_aux_loss
 _ORIG_SHARED_OUT = moe_ref.shared_expert_outputs
+_ORIG_OFFERS = moe_ref.reroute_offers
 
 MUTATIONS = {
     "tanh-gelu": ("gelu", _tanh_gelu, lambda: check_gelu(moe_ref.gelu)),
@@ -461,6 +621,9 @@ MUTATIONS = {
                                 lambda: check_shared_experts_added_ungated(
                                     wl.draw_custom(33, T=24, d=16, ff=24, E=4, dtype="f32", router_std=0.3,
                                                    shared=1), 1, -1)),
+    "reroute-offers-reversed": ("reroute_offers", _offers_reverse_token_order, check_reroute_hand_example_top1),
+    "reroute-no-deeper-fallback": ("reroute_offers", _offers_always_first_fallback,
+                                   check_reroute_hand_example_top1),
 }
 
 
