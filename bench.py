@@ -51,6 +51,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="switch-top1")
     ap.add_argument("--dtype", default=None, help="bf16 or f32 (switch-top1 only; default bf16)")
     ap.add_argument("--cf", type=float, default=None, help="capacity factor (switch-top1: 1.0 or 1.5)")
+    ap.add_argument("--shared", type=int, default=0, help="shared always-on experts added to the workload")
+    ap.add_argument("--reroute", type=int, default=0,
+                    help="rounds of overflow rerouting for assignments dropped at capacity (0: drop)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget for the oracle baseline")
     ap.add_argument("--e2e-steps", type=int, default=None)
@@ -64,12 +67,15 @@ def get_workload(args):
         kw["dtype"] = args.dtype
     if args.cf is not None:
         kw["cf"] = args.cf
+    if args.shared:
+        kw["shared"] = args.shared
     return wl.workload(args.workload, **kw)
 
 
-def workload_label(w) -> str:
+def workload_label(w, reroute: int = 0) -> str:
     return (f"{w.name} T={w.T} d={w.d} ff={w.ff} E={w.E} k={w.k} {w.dtype} "
-            f"cf={w.capacity_factor_label()}")
+            f"cf={w.capacity_factor_label()}" + (f" shared={w.shared}" if w.shared else "")
+            + (f" reroute={reroute}" if reroute else ""))
 
 
 def load_peaks():
@@ -176,7 +182,7 @@ def committed_traffic(kernel: str, workload_tag: str):
 
 
 def workload_tag(w) -> str:
-    return f"{w.name}-{w.dtype}-cf{w.capacity_factor_label()}"
+    return f"{w.name}-{w.dtype}-cf{w.capacity_factor_label()}" + (f"-shared{w.shared}" if w.shared else "")
 
 
 # ---------------------------------------------------------------------------
@@ -281,17 +287,22 @@ def whole_job_tokens_per_s(world: int, steps: int, tokens_per_step: int, max_ms:
 # our arm
 # ---------------------------------------------------------------------------
 def algorithmic_bytes(kernel, w, R, E_active, es):
-    d, ff, T, k, E = w.d, w.ff, w.T, w.k, w.E
+    """Bytes one launch must move at least: every operand read once, every
+    result written once.  S shared experts add S weight panels and S*T rows
+    to both FFN GEMMs (they read x once) and S*T rows to the combine."""
+    d, ff, T, k, E, S = w.d, w.ff, w.T, w.k, w.E, w.shared
     if kernel == "ffn1":
-        return E_active * ff * d * es + E * ff * es + R * d * es + R * ff * es
+        return ((E_active + S) * ff * d * es + (E + S) * ff * es + R * d * es + (T * d * es if S else 0)
+                + (R + S * T) * ff * es)
     if kernel == "ffn2":
-        return E_active * d * ff * es + E * d * es + R * ff * es + R * d * es + R * 4
+        return ((E_active + S) * d * ff * es + (E + S) * d * es + (R + S * T) * ff * es + (R + S * T) * d * es
+                + R * 4)
     if kernel == "router":
         return T * d * es + E * d * es + T * k * 8 + E * 4
     if kernel == "gather":
         return 2 * R * d * es + R * 4
     if kernel == "combine":
-        return R * d * es + T * d * es + T * k * 4
+        return (R + S * T) * d * es + T * d * es + T * k * 4
     return None
 
 
@@ -330,7 +341,7 @@ def run_ours(args):
     dev = torch.device("cuda", local_rank)
     params = MoEParams.from_arrays(inp, dt, dev)
     cap = _lib.moe_capacity(w.T, w.k, w.E, w.cf)
-    layer = MoELayer(params, w.k, cap)
+    layer = MoELayer(params, w.k, cap, reroute=args.reroute)
     x = to_device(inp["x"], dt, dev)
     out = torch.empty_like(x)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -345,12 +356,10 @@ def run_ours(args):
     st = read_stats(layer.stats_buf)
     R = int(st["rows_kept"])
 
-    # count of experts with at least one kept row (their weights are read)
-    idx = torch.empty((w.T, w.k), dtype=torch.int32, device=dev)
-    layer.forward(x, out=out, topk_idx=idx)
-    from collections import Counter
-    cnt = Counter(idx.flatten().tolist())
-    E_active = sum(1 for e in range(w.E) if cnt.get(e, 0) > 0 and cap != 0)   # experts with kept rows
+    # experts with at least one grouped row (their weights are read), from
+    # the dispatch's offsets after the warm-up forward
+    offs = layer.workspace_view(w.T, "offsets", torch.int32, w.E + 1).cpu().numpy()
+    E_active = int((offs[1:] > offs[:-1]).sum())
 
     sampler = ClockSampler(local_rank).start() if rank == 0 else None
     time.sleep(0.05)
@@ -438,13 +447,14 @@ def run_ours(args):
     modelled = [kn for kn in kernels if algorithmic_bytes(kn, w, R, E_active, es) is not None]
     dom = max(modelled, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
     ffn_ms = sum(kernels[k]["ms_per_launch"] for k in ("ffn1", "ffn2") if k in kernels)
-    ffn_flops = 4.0 * R * w.d * w.ff
+    ffn_rows = R + w.shared * w.T                 # routed rows kept + shared-expert rows
+    ffn_flops = 4.0 * ffn_rows * w.d * w.ff
     ffn_tflops = ffn_flops / (ffn_ms / 1000.0) / 1e12 if ffn_ms else None
     dom_bytes = algorithmic_bytes(dom, w, R, E_active, es)
     dom_s = kernels[dom]["ms_per_launch"] / 1000.0
     # a kernel timed inside a long run meets the power cap: use the sustained tensor peak there
     tensor_peak = peaks["bf16_tflops"] if total_ms < 2000 else peaks["bf16_tflops_sustained"]
-    flops_dom = 2.0 * R * w.d * w.ff
+    flops_dom = 2.0 * ffn_rows * w.d * w.ff
     ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if dom in ("ffn1", "ffn2") and w.dtype == "bf16" and flops_dom / max(dom_bytes, 1) > ridge:
         achieved = flops_dom / dom_s / 1e12
@@ -463,8 +473,8 @@ def run_ours(args):
         "warmup": warm, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded numpy draws of the workload's distributions; random-init weights)",
-        "config": {"workload": workload_label(w), "T": w.T, "d": w.d, "ff": w.ff, "E": w.E, "k": w.k,
-                   "capacity": cap, "rows_kept": R,
+        "config": {"workload": workload_label(w, args.reroute), "T": w.T, "d": w.d, "ff": w.ff, "E": w.E, "k": w.k,
+                   "shared_experts": w.shared, "reroute_rounds": args.reroute, "capacity": cap, "rows_kept": R,
                    "l2": "flushed before every step (256 MiB write), outside the step timing",
                    "kernel_timing": "second pass of the same steps with CUDA events around each launch",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
@@ -477,7 +487,7 @@ def run_ours(args):
                 "mode": "pinned host buffers; H2D, layer and D2H of consecutive steps overlap on three streams"},
         "clocks": clocks,
         "gpu_launches": launches,
-        "stats": {k: st[k] for k in ("aux_loss", "imbalance", "drop_rate")},
+        "stats": {k: st[k] for k in ("aux_loss", "imbalance", "drop_rate", "rerouted")},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)

@@ -77,13 +77,16 @@ extern "C" {
 
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK    8
+#define MOE_MAX_SHARED  8   /* shared always-on experts (moe_forward_ex) */
 
 /* Layer statistics, written to DEVICE memory by moe_forward / moe_layer_stats.
  * Definitions (notebook sections "Capacity factor" and "Switch Transformer
  * auxiliary loss"), with counts taken before any capacity drop:
  *   aux_loss  = E * sum_e (counts_e / T) * (prob_sum_e / T)
  *   imbalance = max_e counts_e / (T*k/E)
- *   drop_rate = dropped / (T*k)                                         */
+ *   drop_rate = dropped / (T*k)
+ * With overflow rerouting (moe_forward_ex), rows_kept, dropped and
+ * drop_rate count the assignments served after rerouting.              */
 typedef struct moe_stats {
     float   aux_loss;
     float   imbalance;
@@ -91,6 +94,8 @@ typedef struct moe_stats {
     int32_t rows_kept;   /* R = sum_e min(counts_e, capacity) */
     int32_t max_count;   /* max_e counts_e */
     int32_t dropped;     /* T*k - R */
+    int32_t rerouted;    /* assignments served by a fallback expert (moe_forward_ex
+                            with overflow rerouting; 0 otherwise) */
 } moe_stats;
 
 /* Human-readable name of a status code (static storage). */
@@ -129,6 +134,8 @@ MOE_API size_t moe_dispatch_workspace_size(int T, int k, int E);
 #define MOE_WS_XP        7
 #define MOE_WS_H         8
 #define MOE_WS_YP        9
+#define MOE_WS_FALLBACK_IDX  10  /* [T,F] moe_forward_ex with F > 0 rerouting rounds */
+#define MOE_WS_FALLBACK_GATE 11  /* [T,F] */
 MOE_API size_t moe_workspace_offset(int T, int d, int ff, int E, int k, int dtype, int which);
 
 /* ---- step 1: router (notebook section "Top-k router") ------------------
@@ -244,6 +251,99 @@ MOE_API int moe_forward(const void* x, const void* w_router, const float* logit_
                 int32_t* topk_idx_out, float* topk_gate_out,
                 void* ws, size_t ws_bytes, void* stream);
 
+/* ---- extensions: shared experts and overflow rerouting ------------------
+ *
+ * Shared always-on experts (notebook section "Exercises", item 3): experts
+ * that every token passes through beside its routed ones (the DeepSeek-V2
+ * arrangement the exercise names).  S in [0, MOE_MAX_SHARED] shared experts
+ * of the routed experts' form and shapes, in dtype:
+ *   w1s [S,ff,d], b1s [S,ff], w2s [S,d,ff], b2s [S,d]
+ *   shared_s(x) = fc2_s(gelu(fc1_s(x)))          (exact erf GELU)
+ * Their outputs are added with weight 1 (no gate) to every token, also to
+ * tokens whose routed assignments were all dropped.  Routing, dispatch,
+ * capacity and the statistics concern the routed experts only.
+ * Limits: T*(k+S) < 2^31.  S > MOE_MAX_SHARED returns MOE_ERR_UNSUPPORTED.
+ *
+ * Overflow rerouting (the blog "MoE Parallelism for Inference", section
+ * "Common Bottlenecks", item 1: rejected tokens sent to less busy experts;
+ * the cookbook notebook, section "What": overflow dropped or sent to a
+ * fallback path).  With F >= 1 rounds and a capacity >= 0, the router also
+ * ranks each token's next F experts (its fallbacks, by logit, ties to the
+ * lower index).  After the plain dispatch, in round r = 1..F every token
+ * that still has a dropped assignment offers its first dropped slot j to
+ * its r-th fallback expert c; c accepts offers in token order while it
+ * holds fewer than `capacity` rows.  An accepted slot is served by c with
+ * gate softmax(logits)[c].  Expert e's grouped rows: its own kept
+ * assignments in token order, then those it accepted in round 1 (token
+ * order), round 2, ...  A token never uses one expert twice.  Needs
+ * k + F <= min(E, MOE_MAX_TOPK); F = 0 (or capacity < 0) is the plain
+ * dispatch.  Integer work: exact and independent of thread timing. */
+
+/* Workspace of moe_forward_ex (S = F = 0: moe_workspace_size); 0 if the
+ * sizes are invalid. */
+MOE_API size_t moe_forward_ex_workspace_size(int T, int d, int ff, int E, int k, int S, int F, int dtype);
+
+/* Byte offset of one moe_forward_ex intermediate (MOE_WS_*) in its
+ * workspace.  With S > 0 the h and yp regions hold T*k routed rows, then
+ * S*T shared rows (shared expert s, token t at row T*k + s*T + t). */
+MOE_API size_t moe_forward_ex_workspace_offset(int T, int d, int ff, int E, int k, int S, int F, int dtype,
+                                               int which);
+
+/* The whole layer with shared experts and overflow rerouting:
+ *   out[t,:] = sum over t's served slots j of g_tj * expert_{e_tj}(x[t,:])
+ *              + sum_{s<S} shared_s(x[t,:])
+ * where e_tj / g_tj are the slot's own expert and gate, or its fallback
+ * expert and that expert's gate when rerouting served it.  S = 0 and
+ * reroute_rounds = 0 is exactly moe_forward.  The shared experts run as S
+ * extra row groups (T rows each) inside the same two grouped-FFN launches as
+ * the routed experts; the combine adds their rows in fp32 after the routed
+ * slots.  Rerouting adds 2 * F small launches to the dispatch.  stats, when
+ * given, also reports `rerouted`.  ws: moe_forward_ex_workspace_size(T, d,
+ * ff, E, k, S, reroute_rounds, dtype) bytes, 256-byte aligned.  Other
+ * arguments as moe_forward. */
+MOE_API int moe_forward_ex(const void* x, const void* w_router, const float* logit_bias,
+                   const void* w1, const void* b1, const void* w2, const void* b2,
+                   int S, const void* w1s, const void* b1s, const void* w2s, const void* b2s,
+                   int reroute_rounds,
+                   int T, int d, int ff, int E, int k, int capacity, int dtype,
+                   void* out, moe_stats* stats,
+                   int32_t* topk_idx_out, float* topk_gate_out,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* Step form of overflow rerouting: moe_dispatch with F rounds.
+ *   ranked_idx [T, k+F] int32: each token's experts in router order (the
+ *     first k are its assignments, the rest its fallbacks; distinct per
+ *     row), e.g. moe_router_topk called with k+F;
+ *   ranked_gate [T, k+F] float or NULL: their gates.
+ * Outputs as moe_dispatch, for the assignments a = t*k + j: counts are the
+ * own choices before any drop, offsets / perm / slot_of / drop_mask the
+ * final grouped rows, row_gate[row] the gate of the expert that serves the
+ * row (so combine with topk_gate = NULL after a gated grouped FFN).
+ *   ws/ws_bytes: moe_dispatch_reroute_workspace_size(T, k, F, E) bytes,
+ *   256-byte aligned.
+ * An own choice outside [0,E) is dropped and raises MOE_ERR_BAD_ROUTING in
+ * the device error word; a fallback outside [0,E) is never offered. */
+MOE_API size_t moe_dispatch_reroute_workspace_size(int T, int k, int F, int E);
+MOE_API int moe_dispatch_reroute(const int32_t* ranked_idx, const float* ranked_gate,
+                         int T, int k, int F, int E, int capacity,
+                         int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                         uint8_t* drop_mask, float* row_gate,
+                         const void* x, void* xp, int d, int dtype,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Step form of the shared experts: ys[s*T + t, :] = shared_s(x[t, :]) for
+ * s < S, t < T.  h is caller scratch [S*T, ff]; ys is [S*T, d]; both dtype.
+ * Same kernels (tensor cores for bf16) as moe_grouped_ffn. */
+MOE_API int moe_shared_ffn(const void* x, int T, int d, int ff, int S,
+                   const void* w1s, const void* b1s, const void* w2s, const void* b2s,
+                   void* h, void* ys, int dtype, void* stream);
+
+/* moe_combine plus the shared experts' rows:
+ *   out[t,:] = (moe_combine's value) + sum_{s<S} ys[s*T + t, :]
+ * summed in fp32, routed slots first.  ys may be NULL when S == 0. */
+MOE_API int moe_combine_shared(const void* yp, const int32_t* slot_of, const float* topk_gate,
+                       const void* ys, int S, int T, int k, int d, int dtype, void* out, void* stream);
+
 /* ---- errors, counters, timing -------------------------------------------
  * moe_get_error: synchronises `stream`, then reads and clears the current
  * device's error word.  Returns MOE_OK, MOE_ERR_BAD_ROUTING,
@@ -269,7 +369,8 @@ MOE_API uint64_t moe_launch_count(void);
 #define MOE_KERNEL_FFN2     6
 #define MOE_KERNEL_COMBINE  7
 #define MOE_KERNEL_STATS    8
-#define MOE_NUM_KERNELS     9
+#define MOE_KERNEL_REROUTE  9   /* rerouting rounds (mark + scan kernels) */
+#define MOE_NUM_KERNELS     10
 
 /* moe_timing_enable(1): from now on every kernel launch is bracketed by
  * two CUDA events on its stream (events come from a pool created here, not

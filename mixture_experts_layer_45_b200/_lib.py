@@ -27,8 +27,9 @@ MOE_F32 = 0
 MOE_BF16 = 1
 MOE_MAX_EXPERTS = 256
 MOE_MAX_TOPK = 8
+MOE_MAX_SHARED = 8
 
-KERNEL_NAMES = ["router", "count", "scan", "permute", "gather", "ffn1", "ffn2", "combine", "stats"]
+KERNEL_NAMES = ["router", "count", "scan", "permute", "gather", "ffn1", "ffn2", "combine", "stats", "reroute"]
 MOE_NUM_KERNELS = len(KERNEL_NAMES)
 
 
@@ -40,7 +41,8 @@ class MoeError(RuntimeError):
 
 class MoeStats(ctypes.Structure):
     _fields_ = [("aux_loss", ctypes.c_float), ("imbalance", ctypes.c_float), ("drop_rate", ctypes.c_float),
-                ("rows_kept", ctypes.c_int32), ("max_count", ctypes.c_int32), ("dropped", ctypes.c_int32)]
+                ("rows_kept", ctypes.c_int32), ("max_count", ctypes.c_int32), ("dropped", ctypes.c_int32),
+                ("rerouted", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -61,6 +63,15 @@ _SIGS = {
     "moe_layer_stats": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_forward": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                          ctypes.c_size_t, _P]),
+    "moe_forward_ex_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "moe_forward_ex_workspace_offset": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "moe_forward_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                            _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_dispatch_reroute_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "moe_dispatch_reroute": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P,
+                                  ctypes.c_size_t, _P]),
+    "moe_shared_ffn": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P]),
+    "moe_combine_shared": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "moe_get_error": (_I, [_P]),
     "moe_debug_gelu": (_I, [_P, _P, _I, _I, _P]),
     "moe_launch_count": (ctypes.c_uint64, []),
@@ -131,7 +142,7 @@ def moe_workspace_size(T, d, ff, E, k, dtype) -> int:
 
 
 WS_VIEWS = {"topk_idx": 0, "topk_gate": 1, "counts": 2, "offsets": 3, "perm": 4, "slot_of": 5, "row_gate": 6,
-            "xp": 7, "h": 8, "yp": 9}
+            "xp": 7, "h": 8, "yp": 9, "fallback_idx": 10, "fallback_gate": 11}
 
 
 def moe_workspace_offset(T, d, ff, E, k, dtype, which) -> int:
@@ -193,6 +204,48 @@ def moe_forward(x, w_router, logit_bias, w1, b1, w2, b2, T, d, ff, E, k, capacit
                               T, d, ff, E, k, capacity, dtype, _ptr(out), _ptr(stats), _ptr(topk_idx_out),
                               _ptr(topk_gate_out), _ptr(ws), ws_bytes, _stream(stream)),
            "moe_forward")
+
+
+def moe_forward_ex_workspace_size(T, d, ff, E, k, S, F, dtype) -> int:
+    return load().moe_forward_ex_workspace_size(T, d, ff, E, k, S, F, dtype)
+
+
+def moe_forward_ex_workspace_offset(T, d, ff, E, k, S, F, dtype, which) -> int:
+    code = WS_VIEWS[which] if isinstance(which, str) else which
+    return load().moe_forward_ex_workspace_offset(T, d, ff, E, k, S, F, dtype, code)
+
+
+def moe_forward_ex(x, w_router, logit_bias, w1, b1, w2, b2, S, w1s, b1s, w2s, b2s, reroute_rounds, T, d, ff, E, k,
+                   capacity, dtype, out, stats, topk_idx_out, topk_gate_out, ws, ws_bytes, stream=None):
+    _check(load().moe_forward_ex(_ptr(x), _ptr(w_router), _ptr(logit_bias), _ptr(w1), _ptr(b1), _ptr(w2),
+                                 _ptr(b2), S, _ptr(w1s), _ptr(b1s), _ptr(w2s), _ptr(b2s), reroute_rounds, T, d, ff,
+                                 E, k, capacity, dtype, _ptr(out), _ptr(stats), _ptr(topk_idx_out),
+                                 _ptr(topk_gate_out), _ptr(ws), ws_bytes, _stream(stream)),
+           "moe_forward_ex")
+
+
+def moe_dispatch_reroute_workspace_size(T, k, F, E) -> int:
+    return load().moe_dispatch_reroute_workspace_size(T, k, F, E)
+
+
+def moe_dispatch_reroute(ranked_idx, ranked_gate, T, k, F, E, capacity, counts, offsets, perm, slot_of, drop_mask,
+                         row_gate, x, xp, d, dtype, ws, ws_bytes, stream=None):
+    _check(load().moe_dispatch_reroute(_ptr(ranked_idx), _ptr(ranked_gate), T, k, F, E, capacity, _ptr(counts),
+                                       _ptr(offsets), _ptr(perm), _ptr(slot_of), _ptr(drop_mask), _ptr(row_gate),
+                                       _ptr(x), _ptr(xp), d, dtype, _ptr(ws), ws_bytes, _stream(stream)),
+           "moe_dispatch_reroute")
+
+
+def moe_shared_ffn(x, T, d, ff, S, w1s, b1s, w2s, b2s, h, ys, dtype, stream=None):
+    _check(load().moe_shared_ffn(_ptr(x), T, d, ff, S, _ptr(w1s), _ptr(b1s), _ptr(w2s), _ptr(b2s), _ptr(h),
+                                 _ptr(ys), dtype, _stream(stream)),
+           "moe_shared_ffn")
+
+
+def moe_combine_shared(yp, slot_of, topk_gate, ys, S, T, k, d, dtype, out, stream=None):
+    _check(load().moe_combine_shared(_ptr(yp), _ptr(slot_of), _ptr(topk_gate), _ptr(ys), S, T, k, d, dtype,
+                                     _ptr(out), _stream(stream)),
+           "moe_combine_shared")
 
 
 def moe_get_error(stream=None) -> int:

@@ -213,7 +213,7 @@ constexpr int kFwdScanThreads = 1024;
 __global__ void __launch_bounds__(kFwdScanThreads)
 forward_scan_kernel(const int32_t* __restrict__ hist, const float* __restrict__ psum_part, int nchunk, int E,
                     int T, int k, int capacity, int32_t* __restrict__ base, int32_t* __restrict__ counts,
-                    int32_t* __restrict__ offsets, moe_stats* __restrict__ st) {
+                    int32_t* __restrict__ offsets, moe_stats* __restrict__ st, int32_t* __restrict__ kept_out) {
     pdl_wait();
     pdl_release();
     __shared__ int kept[MOE_MAX_EXPERTS];
@@ -242,6 +242,7 @@ forward_scan_kernel(const int32_t* __restrict__ hist, const float* __restrict__ 
             counts[e] = carry;
             cnt[e] = carry;
             kept[e] = capacity < 0 ? carry : min(carry, capacity);
+            if (kept_out != nullptr) kept_out[e] = kept[e];
             fp[e] = (float(carry) / float(T)) * (ps / float(T));
         }
     }
@@ -296,6 +297,7 @@ forward_scan_kernel(const int32_t* __restrict__ hist, const float* __restrict__ 
                 st->rows_kept = R;
                 st->max_count = mx;
                 st->dropped = A - R;
+                st->rerouted = 0;
             }
         }
     }
@@ -303,34 +305,23 @@ forward_scan_kernel(const int32_t* __restrict__ hist, const float* __restrict__ 
 
 constexpr int kFwdThreads = 256;
 constexpr int kFwdMaxChunk = 1024;   // chunk_tokens * k
+constexpr int kFwdRankRounds = kFwdMaxChunk / kDispWarps / 32;   // 4
 
-__global__ void __launch_bounds__(kFwdThreads)
-forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, int T, int k, int E,
-                       int chunk_tokens, const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
-                       int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, float* __restrict__ row_gate,
-                       const uint8_t* __restrict__ x, int row_bytes, uint8_t* __restrict__ xp,
-                       uint8_t* __restrict__ out_zero_dropped) {
-    pdl_wait();
-    pdl_release();
-    __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
-    __shared__ int off_s[MOE_MAX_EXPERTS + 1];
-    __shared__ int slot_s[kFwdMaxChunk];
+// Stable ranks of a chunk's assignments within their expert (token order):
+// warp w ranks the contiguous assignments [w*per, (w+1)*per) with peer
+// masks, then wcnt[w][e] becomes the count of e in warps before w.  After
+// the call, assignment i = w*per + r*32 + lane (in range) has expert ex[r]
+// (-1 if outside [0,E)) and chunk rank wcnt[w][ex[r]] + rank[r].  All
+// threads of the CTA call it; it ends with __syncthreads().
+__device__ __forceinline__ int chunk_stable_ranks(const int32_t* __restrict__ idx, int a0, int na, int E,
+                                                  int (*wcnt)[MOE_MAX_EXPERTS], int* ex, int* rank) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int chunk = blockIdx.x;
-    const int A = T * k;
-    const int a0 = chunk * chunk_tokens * k;
-    const int na = min(chunk_tokens * k, A - a0);
     for (int i = tid; i < kDispWarps * MOE_MAX_EXPERTS; i += kFwdThreads) (&wcnt[0][0])[i] = 0;
-    for (int e = tid; e <= E; e += kFwdThreads) off_s[e] = offsets[e];
     __syncthreads();
-
-    // warp w ranks the contiguous assignments [w*per, (w+1)*per) of the chunk
     const int per = ((na + kDispWarps - 1) / kDispWarps + 31) & ~31;
     const uint32_t lt_mask = (1u << lane) - 1u;
-    constexpr int kMaxRounds = kFwdMaxChunk / kDispWarps / 32;   // 4
-    int ex[kMaxRounds], rank[kMaxRounds];
 #pragma unroll
-    for (int r = 0; r < kMaxRounds; ++r) {
+    for (int r = 0; r < kFwdRankRounds; ++r) {
         const int i = warp * per + r * 32 + lane;
         const bool in = (r * 32 < per) && i < na;
         int e = in ? idx[a0 + i] : -1;
@@ -354,30 +345,18 @@ forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict_
         }
     }
     __syncthreads();
-    const bool writer = blockIdx.y == 0;
-#pragma unroll
-    for (int r = 0; r < kMaxRounds; ++r) {
-        const int i = warp * per + r * 32 + lane;
-        if (!((r * 32 < per) && i < na)) continue;
-        const int a = a0 + i;
-        const int e = ex[r];
-        int slot = -1;
-        if (e >= 0) {
-            const int g = base[size_t(chunk) * E + e] + wcnt[warp][e] + rank[r];
-            if (g < off_s[e + 1] - off_s[e]) slot = off_s[e] + g;
-        }
-        slot_s[i] = slot;
-        if (writer) {
-            slot_of[a] = slot;
-            if (slot >= 0) {
-                perm[slot] = a;
-                if (row_gate != nullptr) row_gate[slot] = gate[a];
-            }
-        }
-    }
-    __syncthreads();
-    // rows of this chunk handled by this CTA: i = blockIdx.y, blockIdx.y + gridDim.y, ...,
-    // flattened into 16-byte pieces with eight independent loads in flight per thread
+    return per;
+}
+
+// Gather of a chunk's grouped rows: xp[slot] = x[token] for every kept
+// assignment (slot_s[i] >= 0), and, with out_zero_dropped, zero output rows
+// for dropped ones (k == 1 direct output).  The chunk's rows are split over
+// the gridDim.y CTAs of the chunk, flattened into 16-byte pieces with eight
+// independent loads in flight per thread.
+__device__ __forceinline__ void gather_chunk_rows(const int* slot_s, int a0, int na, int k,
+                                                  const uint8_t* __restrict__ x, int row_bytes,
+                                                  uint8_t* __restrict__ xp, uint8_t* __restrict__ out_zero_dropped) {
+    const int tid = threadIdx.x;
     const int vecs = row_bytes >> 4;
     const int Y = int(gridDim.y), y = int(blockIdx.y);
     const int my_rows = (na - y + Y - 1) / Y;
@@ -418,6 +397,340 @@ forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict_
     }
 }
 
+// drop_mask (nullable): 1 for dropped assignments, 0 for kept ones
+__global__ void __launch_bounds__(kFwdThreads)
+forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, int T, int k, int E,
+                       int chunk_tokens, const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, float* __restrict__ row_gate,
+                       const uint8_t* __restrict__ x, int row_bytes, uint8_t* __restrict__ xp,
+                       uint8_t* __restrict__ out_zero_dropped, uint8_t* __restrict__ drop_mask) {
+    pdl_wait();
+    pdl_release();
+    __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
+    __shared__ int off_s[MOE_MAX_EXPERTS + 1];
+    __shared__ int slot_s[kFwdMaxChunk];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int chunk = blockIdx.x;
+    const int A = T * k;
+    const int a0 = chunk * chunk_tokens * k;
+    const int na = min(chunk_tokens * k, A - a0);
+    for (int e = tid; e <= E; e += kFwdThreads) off_s[e] = offsets[e];
+    int ex[kFwdRankRounds], rank[kFwdRankRounds];
+    const int per = chunk_stable_ranks(idx, a0, na, E, wcnt, ex, rank);
+    const bool writer = blockIdx.y == 0;
+#pragma unroll
+    for (int r = 0; r < kFwdRankRounds; ++r) {
+        const int i = warp * per + r * 32 + lane;
+        if (!((r * 32 < per) && i < na)) continue;
+        const int a = a0 + i;
+        const int e = ex[r];
+        int slot = -1;
+        if (e >= 0) {
+            const int g = base[size_t(chunk) * E + e] + wcnt[warp][e] + rank[r];
+            if (g < off_s[e + 1] - off_s[e]) slot = off_s[e] + g;
+        }
+        slot_s[i] = slot;
+        if (writer) {
+            slot_of[a] = slot;
+            if (drop_mask != nullptr) drop_mask[a] = slot < 0 ? 1 : 0;
+            if (slot >= 0) {
+                perm[slot] = a;
+                if (row_gate != nullptr) row_gate[slot] = gate[a];
+            }
+        }
+    }
+    __syncthreads();
+    gather_chunk_rows(slot_s, a0, na, k, x, row_bytes, xp, out_zero_dropped);
+}
+
+// ---------------------------------------------------------------------------
+// Overflow rerouting (F rounds).  Round r = 1..F: every token with an
+// unserved slot offers its first unserved slot j to its r-th fallback
+// expert c = fb_idx[t, r-1]; c accepts offers in token order while it holds
+// fewer than `capacity` rows.  Expert e's rows: its own kept assignments
+// (token order), then round 1's accepted offers (token order), round 2's...
+//
+// Per-assignment state: srv[a] = 0 kept by its own expert, r >= 1 served in
+// round r, -1 not served (yet); srank[a] = its rank among the rows its
+// expert took in that round.  Per token: otok[t] = slot offered in the
+// current round (-1: none), orank[t] = the offer's rank among the chunk's
+// offers to the same expert.
+//
+//   reroute_mark_kernel(r)   grid (chunks): round 1 first ranks the chunk's
+//                            own assignments (srv / srank); round r > 1
+//                            first settles round r-1's offers; then it
+//                            makes round r's offers and their per-chunk
+//                            histogram
+//   reroute_scan_kernel(r)   one CTA: per-(chunk, expert) bases of round r's
+//                            offers, how many each expert accepts, the
+//                            experts' loads; after round F the final
+//                            offsets and statistics
+//   reroute_permute_kernel   grid (chunks, G): settles round F's offers,
+//                            writes the dispatch arrays and gathers rows
+// ---------------------------------------------------------------------------
+// Step-level input of a rerouting dispatch: splits ranked [T, k+F] (each
+// token's experts in router order) into its own choices idx/gate [T, k]
+// and fallbacks fb_idx/fb_gate [T, F], and writes each chunk's histogram of
+// the own choices.  An own choice outside [0, E) is counted nowhere (it is
+// dropped) and raises MOE_ERR_BAD_ROUTING; a fallback outside [0, E) is
+// never offered.  ranked_gate may be null (gates then read as 0).
+__global__ void __launch_bounds__(kFwdThreads)
+reroute_split_kernel(const int32_t* __restrict__ ranked_idx, const float* __restrict__ ranked_gate, int T, int k,
+                     int F, int E, int chunk_tokens, int32_t* __restrict__ idx, float* __restrict__ gate,
+                     int32_t* __restrict__ fb_idx, float* __restrict__ fb_gate, int32_t* __restrict__ hist) {
+    pdl_wait();
+    pdl_release();
+    __shared__ int h[MOE_MAX_EXPERTS];
+    for (int e = threadIdx.x; e < E; e += kFwdThreads) h[e] = 0;
+    __syncthreads();
+    const int K = k + F;
+    const int t0 = blockIdx.x * chunk_tokens;
+    const int nt = min(chunk_tokens, T - t0);
+    for (int i = threadIdx.x; i < nt * K; i += kFwdThreads) {
+        const int t = t0 + i / K;
+        const int c = i - (i / K) * K;
+        const int v = ranked_idx[size_t(t) * K + c];
+        const float g = ranked_gate != nullptr ? ranked_gate[size_t(t) * K + c] : 0.f;
+        if (c < k) {
+            idx[size_t(t) * k + c] = v;
+            gate[size_t(t) * k + c] = g;
+            if (v >= 0 && v < E)
+                atomicAdd(&h[v], 1);
+            else
+                set_error(MOE_ERR_BAD_ROUTING);
+        } else {
+            fb_idx[size_t(t) * F + (c - k)] = v;
+            fb_gate[size_t(t) * F + (c - k)] = g;
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kFwdThreads) hist[size_t(blockIdx.x) * E + e] = h[e];
+}
+
+__global__ void __launch_bounds__(kFwdThreads)
+reroute_mark_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int chunk_tokens, int capacity,
+                    const int32_t* __restrict__ base, const int32_t* __restrict__ fb_idx, int F, int r,
+                    const int32_t* __restrict__ prev_rbase, const int32_t* __restrict__ prev_acc,
+                    int32_t* __restrict__ srv, int32_t* __restrict__ srank, int32_t* __restrict__ otok,
+                    int32_t* __restrict__ orank, int32_t* __restrict__ rhist) {
+    pdl_wait();
+    pdl_release();
+    __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
+    __shared__ int srv_s[kFwdMaxChunk];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int chunk = blockIdx.x;
+    const int t0 = chunk * chunk_tokens;
+    const int nt = min(chunk_tokens, T - t0);
+    const int a0 = t0 * k;
+    const int na = nt * k;
+    if (r == 1) {
+        int ex[kFwdRankRounds], rank[kFwdRankRounds];
+        const int per = chunk_stable_ranks(idx, a0, na, E, wcnt, ex, rank);
+#pragma unroll
+        for (int q = 0; q < kFwdRankRounds; ++q) {
+            const int i = warp * per + q * 32 + lane;
+            if (!((q * 32 < per) && i < na)) continue;
+            const int e = ex[q];
+            int sv = -1, g = 0;
+            if (e >= 0) {
+                g = base[size_t(chunk) * E + e] + wcnt[warp][e] + rank[q];
+                if (g < capacity) sv = 0;
+            }
+            srv_s[i] = sv;
+            srv[a0 + i] = sv;
+            srank[a0 + i] = g;
+        }
+    } else {
+        for (int i = tid; i < na; i += kFwdThreads) srv_s[i] = srv[a0 + i];
+        __syncthreads();
+        // settle round r-1: an offer is accepted when its rank among all
+        // offers to its expert is below what that expert accepted
+        for (int i = tid; i < nt; i += kFwdThreads) {
+            const int t = t0 + i;
+            const int j = otok[t];
+            if (j < 0) continue;
+            const int c = fb_idx[size_t(t) * F + (r - 2)];
+            const int g = prev_rbase[size_t(chunk) * E + c] + orank[t];
+            if (g < prev_acc[c]) {
+                srv_s[i * k + j] = r - 1;
+                srv[a0 + i * k + j] = r - 1;
+                srank[a0 + i * k + j] = g;
+            }
+        }
+    }
+    __syncthreads();   // every read of wcnt above is done; srv_s is complete
+    for (int i = tid; i < kDispWarps * MOE_MAX_EXPERTS; i += kFwdThreads) (&wcnt[0][0])[i] = 0;
+    __syncthreads();
+    // round r's offers: token i of the chunk is thread i (chunk_tokens <= 128)
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int c = -1, j = -1, local = 0;
+    if (tid < nt) {
+        for (int jj = 0; jj < k; ++jj)
+            if (srv_s[tid * k + jj] < 0) {
+                j = jj;
+                break;
+            }
+        if (j >= 0) c = fb_idx[size_t(t0 + tid) * F + (r - 1)];
+        if (c >= E || c < 0) {   // a fallback outside [0, E) cannot be served
+            c = -1;
+            j = -1;
+        }
+    }
+    if (tid < 128) {
+        const uint32_t peers = __match_any_sync(0xffffffffu, c);
+        local = __popc(peers & lt_mask);
+        if (c >= 0 && (peers & lt_mask) == 0) wcnt[warp][c] = __popc(peers);
+    }
+    __syncthreads();
+    if (tid < nt) {
+        int before = 0;
+        if (c >= 0)
+            for (int w = 0; w < warp; ++w) before += wcnt[w][c];
+        otok[t0 + tid] = j;
+        orank[t0 + tid] = before + local;
+    }
+    for (int e = tid; e < E; e += kFwdThreads) {
+        int tot = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) tot += wcnt[w][e];
+        rhist[size_t(chunk) * E + e] = tot;
+    }
+}
+
+// One CTA; warp w scans experts w, w+32, ... over the chunks (fixed order).
+// load [E]: rows each expert holds (in: before round r, out: after).
+__global__ void __launch_bounds__(kFwdScanThreads)
+reroute_scan_kernel(const int32_t* __restrict__ rhist, int nchunk, int E, int capacity, int r, int F, int T, int k,
+                    int32_t* __restrict__ rbase, int32_t* __restrict__ load, int32_t* __restrict__ acc,
+                    int32_t* __restrict__ start, int32_t* __restrict__ offsets, moe_stats* __restrict__ st) {
+    pdl_wait();
+    pdl_release();
+    __shared__ int load_s[MOE_MAX_EXPERTS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = warp; e < E; e += kFwdScanThreads / 32) {
+        int carry = 0;
+        for (int b0 = 0; b0 < nchunk; b0 += 32) {
+            const int b = b0 + lane;
+            const int h = b < nchunk ? rhist[size_t(b) * E + e] : 0;
+            int incl = h;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (b < nchunk) rbase[size_t(b) * E + e] = carry + incl - h;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            const int l = load[e];
+            const int a = min(carry, max(capacity - l, 0));
+            acc[e] = a;
+            start[e] = l;
+            load[e] = l + a;
+            load_s[e] = l + a;
+        }
+    }
+    if (r != F) return;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        constexpr int PER = MOE_MAX_EXPERTS / 32;
+        int local[PER];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            local[i] = e < E ? load_s[e] : 0;
+            sum += local[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            if (e < E) offsets[e] = run;
+            run += local[i];
+        }
+        if (lane == 31) {
+            offsets[E] = incl;
+            if (st != nullptr) {
+                // the primary dispatch's statistics are already in st
+                const int A = T * k;
+                const int R = incl;
+                st->rerouted = R - st->rows_kept;
+                st->rows_kept = R;
+                st->dropped = A - R;
+                st->drop_rate = float(A - R) / float(A);
+            }
+        }
+    }
+}
+
+// start: [F][E] row start of each round's accepted offers within an expert
+__global__ void __launch_bounds__(kFwdThreads)
+reroute_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate,
+                       const int32_t* __restrict__ fb_idx, const float* __restrict__ fb_gate, int T, int k, int E,
+                       int F, int chunk_tokens, const int32_t* __restrict__ srv, const int32_t* __restrict__ srank,
+                       const int32_t* __restrict__ otok, const int32_t* __restrict__ orank,
+                       const int32_t* __restrict__ last_rbase, const int32_t* __restrict__ last_acc,
+                       const int32_t* __restrict__ start, const int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, float* __restrict__ row_gate,
+                       const uint8_t* __restrict__ x, int row_bytes, uint8_t* __restrict__ xp,
+                       uint8_t* __restrict__ out_zero_dropped, uint8_t* __restrict__ drop_mask) {
+    pdl_wait();
+    pdl_release();
+    __shared__ int off_s[MOE_MAX_EXPERTS + 1];
+    __shared__ int slot_s[kFwdMaxChunk];
+    const int tid = threadIdx.x;
+    const int chunk = blockIdx.x;
+    const int t0 = chunk * chunk_tokens;
+    const int nt = min(chunk_tokens, T - t0);
+    const int a0 = t0 * k;
+    const int na = nt * k;
+    for (int e = tid; e <= E; e += kFwdThreads) off_s[e] = offsets[e];
+    __syncthreads();
+    const bool writer = blockIdx.y == 0;
+    for (int i = tid; i < na; i += kFwdThreads) {
+        const int a = a0 + i;
+        const int t = a / k;
+        const int j = a - t * k;
+        const int sv = srv[a];
+        int slot = -1;
+        float g = 0.f;
+        if (sv == 0) {
+            const int e = idx[a];
+            slot = off_s[e] + srank[a];
+            g = gate[a];
+        } else if (sv > 0) {
+            const int c = fb_idx[size_t(t) * F + (sv - 1)];
+            slot = off_s[c] + start[size_t(sv - 1) * E + c] + srank[a];
+            g = fb_gate[size_t(t) * F + (sv - 1)];
+        } else if (otok[t] == j) {
+            const int c = fb_idx[size_t(t) * F + (F - 1)];
+            const int gg = last_rbase[size_t(chunk) * E + c] + orank[t];
+            if (gg < last_acc[c]) {
+                slot = off_s[c] + start[size_t(F - 1) * E + c] + gg;
+                g = fb_gate[size_t(t) * F + (F - 1)];
+            }
+        }
+        slot_s[i] = slot;
+        if (writer) {
+            slot_of[a] = slot;
+            if (drop_mask != nullptr) drop_mask[a] = slot < 0 ? 1 : 0;
+            if (slot >= 0) {
+                perm[slot] = a;
+                if (row_gate != nullptr) row_gate[slot] = g;
+            }
+        }
+    }
+    __syncthreads();
+    gather_chunk_rows(slot_s, a0, na, k, x, row_bytes, xp, out_zero_dropped);
+}
+
 // ---------------------------------------------------------------------------
 // Step 4: combine.  out[t] = sum over kept slots j (in slot order) of
 // w_tj * yp[slot_of[t*k+j]]; w_tj = gate or 1.  fp32 accumulation.
@@ -444,11 +757,13 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
 }
 
 // One warp per token; each lane handles 16-byte pieces of the row, four at a
-// time, so 4 * k independent loads are in flight before the adds.
+// time, so 4 * k independent loads are in flight before the adds.  With
+// S > 0 shared experts, ys [S, Tn, d] holds their outputs and each adds its
+// row of token t with weight 1 after the routed slots.
 template <typename T>
 __global__ void __launch_bounds__(256)
 combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
-               int Tn, int k, int d, T* __restrict__ out) {
+               int Tn, int k, int d, T* __restrict__ out, const T* __restrict__ ys, int S) {
     pdl_wait();
     pdl_release();
     constexpr int EPV = 16 / sizeof(T);   // elements per 16-byte piece
@@ -470,14 +785,14 @@ combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, co
             for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int i = 0; i < EPV; ++i) acc[u][i] = 0.f;
-#pragma unroll
-            for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-                if (slot[j] < 0) continue;
+            // routed slots (the unrolled loop lets all k rows' loads be in
+            // flight together), then the shared experts' rows one at a time
+            auto add_row = [&](const T* src, float wj) {
                 uint4 raw[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int c = c0 + u * 32;
-                    raw[u] = (c < pieces) ? __ldg(reinterpret_cast<const uint4*>(yp + size_t(slot[j]) * d) + c)
+                    raw[u] = (c < pieces) ? __ldg(reinterpret_cast<const uint4*>(src) + c)
                                           : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
@@ -492,9 +807,14 @@ combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, co
                         v[2] = __uint_as_float(raw[u].z); v[3] = __uint_as_float(raw[u].w);
                     }
 #pragma unroll
-                    for (int i = 0; i < EPV; ++i) acc[u][i] = fmaf(w[j], v[i], acc[u][i]);
+                    for (int i = 0; i < EPV; ++i) acc[u][i] = fmaf(wj, v[i], acc[u][i]);
                 }
-            }
+            };
+#pragma unroll
+            for (int j = 0; j < MOE_MAX_TOPK; ++j)
+                if (slot[j] >= 0) add_row(yp + size_t(slot[j]) * d, w[j]);
+#pragma unroll 1
+            for (int sx = 0; sx < S; ++sx) add_row(ys + (size_t(sx) * Tn + t) * d, 1.f);
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int c = c0 + u * 32;
@@ -558,6 +878,7 @@ stats_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ off
         st->rows_kept = R;
         st->max_count = s_max[0];
         st->dropped = A - R;
+        st->rerouted = 0;
     }
 }
 

@@ -20,31 +20,62 @@ namespace moe {
 
 enum FfnMode { kFc1Gelu = 0, kFc2Gate = 1 };
 
+// Shared always-on experts (notebook section "Exercises", item 3: every
+// token also passes through a few experts outside the router) run as S
+// extra row groups after the E routed ones, in the same launch: group E + s
+// has `rows` rows (all tokens), reads A rows arow0 + s * astride ..., weight
+// panel s of the shared weight tensor, and writes C rows crow0 + s * rows ...
+// with gate 1.  S = 0 leaves only the routed groups.
+struct SharedGroups {
+    int S;
+    int rows;
+    int arow0, astride;
+    int crow0;
+};
+
+constexpr int kMaxGroups = MOE_MAX_EXPERTS + MOE_MAX_SHARED;
+
 struct TileTable {
-    int start[MOE_MAX_EXPERTS + 1];   // first tile of each expert; start[E] = total
-    int mtiles[MOE_MAX_EXPERTS];      // M tiles of each expert
-    int off[MOE_MAX_EXPERTS + 1];     // row offsets (copy of `offsets`)
+    int start[kMaxGroups + 1];   // first tile of each group; start[G] = total
+    int mtiles[kMaxGroups];      // M tiles of each group
+    int arow[kMaxGroups];        // first A row of each group
+    int crow[kMaxGroups];        // first C row (and row_gate / out_rows index)
+    int rows[kMaxGroups];        // rows of each group
 };
 
 // Must be called by all threads of the CTA; ends with __syncthreads().
-__device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ offsets, int E, int BM, int ntiles_n,
-                                                 TileTable& tt) {
+// Routed group e < E covers rows offsets[e] .. offsets[e+1]-1 of A and C.
+__device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ offsets, int E, const SharedGroups& sh,
+                                                 int BM, int ntiles_n, TileTable& tt) {
     pdl_wait();
     pdl_release();
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) tt.off[e] = offsets[e];
+    const int G = E + sh.S;
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+        if (g < E) {
+            const int lo = offsets[g];
+            tt.arow[g] = lo;
+            tt.crow[g] = lo;
+            tt.rows[g] = offsets[g + 1] - lo;
+        } else {
+            const int s = g - E;
+            tt.arow[g] = sh.arow0 + s * sh.astride;
+            tt.crow[g] = sh.crow0 + s * sh.rows;
+            tt.rows[g] = sh.rows;
+        }
+    }
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
-        constexpr int PER = MOE_MAX_EXPERTS / 32;
+        constexpr int PER = (kMaxGroups + 31) / 32;
         int tl[PER];
         int sum = 0;
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-            const int e = lane * PER + i;
+            const int g = lane * PER + i;
             int mt = 0;
-            if (e < E) {
-                mt = (tt.off[e + 1] - tt.off[e] + BM - 1) / BM;
-                tt.mtiles[e] = mt;
+            if (g < G) {
+                mt = (tt.rows[g] + BM - 1) / BM;
+                tt.mtiles[g] = mt;
             }
             tl[i] = mt * ntiles_n;
             sum += tl[i];
@@ -58,27 +89,27 @@ __device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ off
         int run = incl - sum;
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-            const int e = lane * PER + i;
-            if (e < E) tt.start[e] = run;
+            const int g = lane * PER + i;
+            if (g < G) tt.start[g] = run;
             run += tl[i];
         }
-        if (lane == 31) tt.start[E] = incl;
+        if (lane == 31) tt.start[G] = incl;
     }
     __syncthreads();
 }
 
 struct TileCoord {
-    int e, mt, nt;
+    int e, mt, nt;   // e: group (routed expert, or E + shared expert)
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const TileTable& tt, int E, int t) {
-    int lo = 0, hi = E - 1;   // last e with start[e] <= t (experts with no tiles are skipped)
+__device__ __forceinline__ TileCoord decode_tile(const TileTable& tt, int G, int t) {
+    int lo = 0, hi = G - 1;   // last g with start[g] <= t (groups with no tiles are skipped)
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (tt.start[mid] <= t) lo = mid; else hi = mid - 1;
     }
-    // experts without tiles have start[e] == start[e+1], so the last e with
-    // start[e] <= t is the one whose range [start[e], start[e+1]) holds t
+    // groups without tiles have start[g] == start[g+1], so the last g with
+    // start[g] <= t is the one whose range [start[g], start[g+1]) holds t
     TileCoord c;
     c.e = lo;
     const int local = t - tt.start[lo];
@@ -94,26 +125,31 @@ __device__ __forceinline__ TileCoord decode_tile(const TileTable& tt, int E, int
 constexpr int kSgBM = 128, kSgBN = 128, kSgBK = 8, kSgThreads = 256;
 constexpr int kSgLd = kSgBM + 4;
 
+// A2 / W2 / bias2: the shared experts' A rows and parameters (used when sh.S > 0)
 template <int MODE>
 __global__ void __launch_bounds__(kSgThreads)
 ffn_simt_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ offsets, int E, int N, int K,
                     const float* __restrict__ W, const float* __restrict__ bias, const float* __restrict__ row_gate,
-                    const int32_t* __restrict__ out_rows, float* __restrict__ C) {
+                    const int32_t* __restrict__ out_rows, float* __restrict__ C, SharedGroups sh,
+                    const float* __restrict__ A2, const float* __restrict__ W2, const float* __restrict__ bias2) {
     __shared__ TileTable tt;
     __shared__ __align__(16) float As[2][kSgBK][kSgLd];
     __shared__ __align__(16) float Bs[2][kSgBK][kSgLd];
     const int ntn = (N + kSgBN - 1) / kSgBN;
-    build_tile_table(offsets, E, kSgBM, ntn, tt);
-    const int total = tt.start[E];
+    build_tile_table(offsets, E, sh, kSgBM, ntn, tt);
+    const int G = E + sh.S;
+    const int total = tt.start[G];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int lrow = tid >> 1, lk = (tid & 1) * 4;   // loader: one float4 of A and of W per thread
 
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-        const TileCoord tc = decode_tile(tt, E, t);
-        const int rows = tt.off[tc.e + 1] - tt.off[tc.e];
+        const TileCoord tc = decode_tile(tt, G, t);
+        const bool shared_g = tc.e >= E;
+        const int rows = tt.rows[tc.e];
         const int m0 = tc.mt * kSgBM, n0 = tc.nt * kSgBN;
-        const float* Ab = A + size_t(tt.off[tc.e]) * K;
-        const float* Wb = W + size_t(tc.e) * N * K;
+        const float* Ab = (shared_g ? A2 : A) + size_t(tt.arow[tc.e]) * K;
+        const float* Wb = shared_g ? W2 + size_t(tc.e - E) * N * K : W + size_t(tc.e) * N * K;
+        const float* bb = shared_g ? bias2 + size_t(tc.e - E) * N : bias + size_t(tc.e) * N;
 
         float acc[8][8];
 #pragma unroll
@@ -169,9 +205,9 @@ ffn_simt_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ off
         for (int i = 0; i < 8; ++i) {
             const int r = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
             if (r >= rows) continue;
-            const size_t grow = size_t(tt.off[tc.e]) + r;
-            const size_t crow = (out_rows != nullptr) ? size_t(out_rows[grow]) : grow;
-            const float g = (MODE == kFc2Gate && row_gate != nullptr) ? row_gate[grow] : 1.f;
+            const size_t grow = size_t(tt.crow[tc.e]) + r;
+            const size_t crow = (out_rows != nullptr && !shared_g) ? size_t(out_rows[grow]) : grow;
+            const float g = (MODE == kFc2Gate && row_gate != nullptr && !shared_g) ? row_gate[grow] : 1.f;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int n = n0 + h * 64 + tx * 4;
@@ -179,7 +215,7 @@ ffn_simt_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ off
                 float v[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const float c = acc[i][h * 4 + j] + bias[size_t(tc.e) * N + n + j];
+                    const float c = acc[i][h * 4 + j] + bb[n + j];
                     v[j] = (MODE == kFc1Gelu) ? gelu_erf(c) : g * c;
                 }
                 *reinterpret_cast<float4*>(C + crow * N + n) = make_float4(v[0], v[1], v[2], v[3]);
@@ -219,12 +255,15 @@ struct TcCfg {
     static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;   // + alignment slack
 };
 
+// tmA2 / tmB2 / bias2: the shared experts' A rows and parameters (used when sh.S > 0)
 template <int BN, int STAGES, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
 ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const int32_t* __restrict__ offsets, int E, int N, int K,
                    const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
-                   const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C) {
+                   const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C, SharedGroups sh,
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                   const __nv_bfloat16* __restrict__ bias2) {
     using Cfg = TcCfg<BN, STAGES>;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN: whole 32-column epilogue chunks, MMA N <= 256");
     __shared__ TileTable tt;
@@ -251,6 +290,10 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (sh.S > 0) {
+            tma_prefetch_desc(&tmA2);
+            tma_prefetch_desc(&tmB2);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&tmem_slot, Cfg::kTmemCols);
@@ -258,10 +301,11 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         tc_fence_before();
     }
     const int ntn = (N + BN - 1) / BN;
-    build_tile_table(offsets, E, kTcBM, ntn, tt);   // contains __syncthreads()
+    build_tile_table(offsets, E, sh, kTcBM, ntn, tt);   // contains __syncthreads()
     tc_fence_after();
     const uint32_t tmem_base = tmem_slot;
-    const int total = tt.start[E];
+    const int G = E + sh.S;
+    const int total = tt.start[G];
     const int KB = (K + kTcBK - 1) / kTcBK;
     volatile int* abort_p = &abort_flag;
 
@@ -274,16 +318,20 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const TileCoord tc = decode_tile(tt, E, t);
-                const int row0 = tt.off[tc.e] + tc.mt * kTcBM;
+                const TileCoord tc = decode_tile(tt, G, t);
+                const bool shared_g = tc.e >= E;
+                const CUtensorMap* ma = shared_g ? &tmA2 : &tmA;
+                const CUtensorMap* mb = shared_g ? &tmB2 : &tmB;
+                const int widx = shared_g ? tc.e - E : tc.e;
+                const int row0 = tt.arow[tc.e] + tc.mt * kTcBM;
                 const int n0 = tc.nt * BN;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) { ok = false; break; }
                     uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
                     uint8_t* sb = sa + Cfg::kABytes;
                     mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
-                    tma_load_2d(sa, &tmA, &full_bar[stage], kb * kTcBK, row0);
-                    tma_load_3d(sb, &tmB, &full_bar[stage], kb * kTcBK, n0, tc.e);
+                    tma_load_2d(sa, ma, &full_bar[stage], kb * kTcBK, row0);
+                    tma_load_3d(sb, mb, &full_bar[stage], kb * kTcBK, n0, widx);
                     last_parity[stage] = int(phase);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -347,19 +395,22 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             // all epilogue warps stop together once any wait has given up, so
             // none is left behind at a named barrier
             if (named_bar_red_or(1, 32 * kTcEpiWarps, failed || *abort_p)) break;
-            const TileCoord tc = decode_tile(tt, E, t);
-            const int rows = tt.off[tc.e + 1] - tt.off[tc.e];
+            const TileCoord tc = decode_tile(tt, G, t);
+            const bool shared_g = tc.e >= E;
+            const int rows = tt.rows[tc.e];
             const int r_in = tc.mt * kTcBM + q * 32 + lane;
             const bool valid = r_in < rows;
-            const size_t grow = size_t(tt.off[tc.e]) + r_in;
-            // destination row: the grouped row, or (direct output) the row out_rows names
-            const size_t crow = (out_rows != nullptr && valid) ? size_t(out_rows[grow]) : grow;
+            const size_t grow = size_t(tt.crow[tc.e]) + r_in;
+            // destination row: the grouped row, or (direct output of a routed
+            // group) the row out_rows names
+            const size_t crow = (out_rows != nullptr && valid && !shared_g) ? size_t(out_rows[grow]) : grow;
             const int n0 = tc.nt * BN;
-            float g = 1.f;
-            if (MODE == kFc2Gate && row_gate != nullptr && valid) g = row_gate[grow];
+            float g = 1.f;   // shared experts are ungated
+            if (MODE == kFc2Gate && row_gate != nullptr && valid && !shared_g) g = row_gate[grow];
+            const __nv_bfloat16* bb = shared_g ? bias2 + size_t(tc.e - E) * N : bias + size_t(tc.e) * N;
             // (the barrier above also ends every read of the previous tile's bias)
             for (int i = etid; i < BN; i += 32 * kTcEpiWarps)
-                sbias[i] = (n0 + i < N) ? __bfloat162float(bias[size_t(tc.e) * N + n0 + i]) : 0.f;
+                sbias[i] = (n0 + i < N) ? __bfloat162float(bb[n0 + i]) : 0.f;
             named_bar_sync(1, 32 * kTcEpiWarps);   // this tile's bias is visible
             if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_p)) {
                 failed = true;

@@ -148,9 +148,66 @@ int check_sizes(int T, int d, int ff, int E, int k, int dtype, bool need_ff) {
     return MOE_OK;
 }
 
+int check_shared(int T, int k, int S) {
+    if (S < 0) return MOE_ERR_INVALID_ARG;
+    if (S > MOE_MAX_SHARED) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(T) * (k + S) >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+// F rerouting rounds need k + F distinct experts per token
+int check_reroute(int k, int E, int F) {
+    if (F < 0) return MOE_ERR_INVALID_ARG;
+    if (k + F > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (k + F > E) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Scratch of a rerouting dispatch (F rounds, nchunk chunks).
+struct RerouteWs {
+    int32_t* srv;     // [T*k]
+    int32_t* srank;   // [T*k]
+    int32_t* otok;    // [T]
+    int32_t* orank;   // [T]
+    int32_t* rhist;   // [nchunk][E]
+    int32_t* rbase;   // [F][nchunk][E]
+    int32_t* load;    // [E]
+    int32_t* acc;     // [F][E]
+    int32_t* start;   // [F][E]
+};
+
+size_t reroute_ws_bytes(int T, int k, int E, int F, int nchunk) {
+    const size_t A = size_t(T) * k;
+    return align256(A * 4) * 2 + align256(size_t(T) * 4) * 2 + align256(size_t(nchunk) * E * 4) +
+           align256(size_t(F) * nchunk * E * 4) + align256(size_t(E) * 4) + align256(size_t(F) * E * 4) * 2;
+}
+
+RerouteWs carve_reroute_ws(void* base, int T, int k, int E, int F, int nchunk) {
+    uint8_t* p = static_cast<uint8_t*>(base);
+    auto take = [&](size_t bytes) {
+        int32_t* r = reinterpret_cast<int32_t*>(p);
+        p += align256(bytes);
+        return r;
+    };
+    const size_t A = size_t(T) * k;
+    RerouteWs w;
+    w.srv = take(A * 4);
+    w.srank = take(A * 4);
+    w.otok = take(size_t(T) * 4);
+    w.orank = take(size_t(T) * 4);
+    w.rhist = take(size_t(nchunk) * E * 4);
+    w.rbase = take(size_t(F) * nchunk * E * 4);
+    w.load = take(size_t(E) * 4);
+    w.acc = take(size_t(F) * E * 4);
+    w.start = take(size_t(F) * E * 4);
+    return w;
+}
+
 struct WsLayout {
     size_t idx, gate, counts, offsets, perm, slot_of, row_gate, xp, h, yp;
-    size_t fhist, fbase, fpsum, total;   // per-router-chunk arrays of the forward path
+    size_t fhist, fbase, fpsum;   // per-router-chunk arrays of the forward path
+    size_t fb_idx, fb_gate, reroute;   // overflow rerouting (F > 0)
+    size_t total;
 };
 
 // tokens per router CTA (= one dispatch chunk of the forward path)
@@ -161,9 +218,12 @@ size_t dispatch_ws_bytes(int A, int E) {
     return 2 * align256(size_t(nblk) * E * sizeof(int32_t));
 }
 
-WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype) {
+// S shared experts add S * T rows to h and yp, after the T * k routed rows;
+// F rerouting rounds add the fallback lists and the rerouting scratch
+WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype, int S = 0, int F = 0) {
     WsLayout L{};
     const size_t A = size_t(T) * k, es = elem_bytes(dtype);
+    const size_t HR = A + size_t(S) * T;   // rows of h and yp
     size_t o = 0;
     auto take = [&](size_t bytes) {
         const size_t r = o;
@@ -178,12 +238,15 @@ WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype) {
     L.slot_of = take(A * 4);
     L.row_gate = take(A * 4);
     L.xp = take(A * d * es);
-    L.h = take(A * ff * es);
-    L.yp = take(A * d * es);
+    L.h = take(HR * ff * es);
+    L.yp = take(HR * d * es);
     const size_t nchunk = size_t(std::max(1, ceil_div(T, router_chunk_tokens(dtype))));
     L.fhist = take(nchunk * E * 4);
     L.fbase = take(nchunk * E * 4);
     L.fpsum = take(nchunk * E * 4);
+    L.fb_idx = take(size_t(T) * F * 4);
+    L.fb_gate = take(size_t(T) * F * 4);
+    L.reroute = take(F > 0 ? reroute_ws_bytes(T, k, E, F, int(nchunk)) : 0);
     L.total = o;
     return L;
 }
@@ -243,22 +306,36 @@ bool set_smem_attr(K kernel, size_t bytes) {
 // ---------------------------------------------------------------------------
 // step launchers (arguments already validated)
 // ---------------------------------------------------------------------------
+// F > 0: also the next F experts of each token (fallbacks for overflow
+// rerouting) into fb_idx / fb_gate [T, F]
+struct RouterOut {
+    int32_t* idx;
+    float* gate;
+    float* psum;        // [E] atomic sums (zeroed here), or null
+    float* psum_part;   // [tiles][E] per-tile sums, or null
+    int32_t* hist;      // [tiles][E] per-tile histograms, or null
+    int F;
+    int32_t* fb_idx;
+    float* fb_gate;
+};
+
 template <typename Tin, int EP>
-int launch_router_ep(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                     float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+int launch_router_ep(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
+                     const RouterOut& o, cudaStream_t s) {
     auto kern = router_topk_kernel<Tin, EP>;
     const size_t smem = router_smem_bytes<EP>();
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     Launch L(MOE_KERNEL_ROUTER, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(kern, dim3(ceil_div(T, kRouterTM)), dim3(kRouterThreads), smem, s, static_cast<const Tin*>(x), static_cast<const Tin*>(wr),
-                                                              bias, T, d, E, k, idx, gate, psum, psum_part, hist);
+    launch_err = launch_pdl(kern, dim3(ceil_div(T, kRouterTM)), dim3(kRouterThreads), smem, s,
+                            static_cast<const Tin*>(x), static_cast<const Tin*>(wr), bias, T, d, E, k, o.idx, o.gate,
+                            o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate);
     return L.finish(launch_err);
 }
 
 template <int EP, int KMAX>
-int launch_router_tc(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                     float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
+int launch_router_tc(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
+                     const RouterOut& o, cudaStream_t s) {
     CUtensorMap tmX, tmW;
     if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), kRtBM)) return MOE_ERR_UNSUPPORTED;
     if (!make_map_2d(&tmW, wr, uint64_t(d), uint64_t(E), EP)) return MOE_ERR_UNSUPPORTED;
@@ -268,44 +345,45 @@ int launch_router_tc(const void* x, const void* wr, const float* bias, int T, in
     Launch L(MOE_KERNEL_ROUTER, s);
     cudaError_t launch_err;
     launch_err = launch_pdl(kern, dim3(ceil_div(T, kRtBM)), dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k,
-                            idx, gate, psum, psum_part, hist);
+                            o.idx, o.gate, o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate);
     return L.finish(launch_err);
 }
 
 template <int KMAX>
-int launch_router_tc_k(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                       float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
-    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 128)
-        return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+int launch_router_tc_k(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
+                       const RouterOut& o, cudaStream_t s) {
+    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 128) return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, o, s);
 }
 
 template <typename Tin>
-int launch_router_t(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int32_t* idx,
-                    float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
-    if (E <= 16) return launch_router_ep<Tin, 16>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 32) return launch_router_ep<Tin, 32>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 64) return launch_router_ep<Tin, 64>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    if (E <= 128) return launch_router_ep<Tin, 128>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-    return launch_router_ep<Tin, 256>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+int launch_router_t(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
+                    const RouterOut& o, cudaStream_t s) {
+    if (E <= 16) return launch_router_ep<Tin, 16>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 32) return launch_router_ep<Tin, 32>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 64) return launch_router_ep<Tin, 64>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 128) return launch_router_ep<Tin, 128>(x, wr, bias, T, d, E, k, o, s);
+    return launch_router_ep<Tin, 256>(x, wr, bias, T, d, E, k, o, s);
 }
 
-// bf16: tcgen05 router (128-token tiles); f32: SIMT fp32 router (32-token tiles).  prob_sum (atomic, zeroed here) or psum_part/hist (per
-// tile) as requested.
+// bf16: tcgen05 router (128-token tiles); f32: SIMT fp32 router (32-token
+// tiles).  prob_sum (atomic, zeroed here) or psum_part/hist (per tile) as
+// requested in `o`.
 int run_router(const void* x, const void* wr, const float* bias, int T, int d, int E, int k, int dtype,
-               int32_t* idx, float* gate, float* psum, float* psum_part, int32_t* hist, cudaStream_t s) {
-    if (psum != nullptr && psum_part == nullptr &&
-        cudaMemsetAsync(psum, 0, size_t(E) * sizeof(float), s) != cudaSuccess)
+               const RouterOut& o, cudaStream_t s) {
+    if (o.psum != nullptr && o.psum_part == nullptr &&
+        cudaMemsetAsync(o.psum, 0, size_t(E) * sizeof(float), s) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (dtype == MOE_BF16) {
-        if (k == 1) return launch_router_tc_k<1>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-        if (k == 2) return launch_router_tc_k<2>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
-        return launch_router_tc_k<MOE_MAX_TOPK>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+        const int ksel = k + o.F;
+        if (ksel == 1) return launch_router_tc_k<1>(x, wr, bias, T, d, E, k, o, s);
+        if (ksel == 2) return launch_router_tc_k<2>(x, wr, bias, T, d, E, k, o, s);
+        return launch_router_tc_k<MOE_MAX_TOPK>(x, wr, bias, T, d, E, k, o, s);
     }
-    return launch_router_t<float>(x, wr, bias, T, d, E, k, idx, gate, psum, psum_part, hist, s);
+    return launch_router_t<float>(x, wr, bias, T, d, E, k, o, s);
 }
 
 int run_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int capacity, int32_t* counts,
@@ -351,96 +429,216 @@ int run_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int
 // tiles measured slower on every workload: more A re-reads per FLOP)
 constexpr int kTcBN = 256, kTcStages = 4;
 
+// The shared always-on experts of one FFN GEMM (host side): S groups of
+// `g.rows` rows each, A rows from `a` (a_rows rows in all), weights [S, N, K]
+// and biases [S, N].  S = 0: none.
+struct SharedArgs {
+    const void* a = nullptr;
+    int a_rows = 0;
+    const void* w = nullptr;
+    const void* bias = nullptr;
+    SharedGroups g{};
+};
+
+// Routed groups: E experts over rows offsets[0..E] of `a` (a_rows rows;
+// routed_rows_ub bounds offsets[E]).  E may be 0 when only shared groups run.
 template <int BN, int STAGES, int MODE>
-int launch_tc(const void* a, int a_cols, int max_rows, const void* w, int N, int E, const int32_t* offsets,
-              const void* bias, const float* row_gate, const int32_t* out_rows, void* c, int kernel_id,
-              cudaStream_t s) {
-    CUtensorMap tmA, tmB;
-    if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(max_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
-    if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), BN)) return MOE_ERR_UNSUPPORTED;
+int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
+              const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
+              const SharedArgs& sa, int kernel_id, cudaStream_t s) {
+    CUtensorMap tmA, tmB, tmA2, tmB2;
+    if (sa.g.S > 0) {
+        if (!make_map_2d(&tmA2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
+        if (!make_map_3d(&tmB2, sa.w, uint64_t(a_cols), uint64_t(N), uint64_t(sa.g.S), BN))
+            return MOE_ERR_UNSUPPORTED;
+    }
+    if (E > 0) {
+        if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(a_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
+        if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), BN)) return MOE_ERR_UNSUPPORTED;
+    } else {
+        tmA = tmA2;
+        tmB = tmB2;
+    }
+    if (sa.g.S == 0) {
+        tmA2 = tmA;
+        tmB2 = tmB;
+    }
     auto kern = ffn_tc_bf16_kernel<BN, STAGES, MODE>;
     const size_t smem = TcCfg<BN, STAGES>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
-    const long long tiles_ub = (static_cast<long long>(ceil_div(max_rows, kTcBM)) + E) * ceil_div(N, BN);
+    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kTcBM)) + E +
+                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kTcBM);
+    const long long tiles_ub = mt_ub * ceil_div(N, BN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, s, tmA, tmB, offsets, E, N, a_cols, static_cast<const __nv_bfloat16*>(bias),
-                                        row_gate, out_rows, static_cast<__nv_bfloat16*>(c));
+    launch_err = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, s, tmA, tmB, offsets, E, N, a_cols,
+                            static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
+                            static_cast<__nv_bfloat16*>(c), sa.g, tmA2, tmB2,
+                            static_cast<const __nv_bfloat16*>(sa.bias));
     return L.finish(launch_err);
 }
 
 template <int MODE>
-int launch_simt(const void* a, int K, int max_rows, const void* w, int N, int E, const int32_t* offsets,
-                const void* bias, const float* row_gate, const int32_t* out_rows, void* c, int kernel_id,
-                cudaStream_t s) {
-    const long long tiles_ub = (static_cast<long long>(ceil_div(max_rows, kSgBM)) + E) * ceil_div(N, kSgBN);
+int launch_simt(const void* a, int K, int routed_rows_ub, const void* w, int N, int E, const int32_t* offsets,
+                const void* bias, const float* row_gate, const int32_t* out_rows, void* c, const SharedArgs& sa,
+                int kernel_id, cudaStream_t s) {
+    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kSgBM)) + E +
+                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kSgBM);
+    const long long tiles_ub = mt_ub * ceil_div(N, kSgBN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, 2ll * num_sms())));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(ffn_simt_f32_kernel<MODE>, dim3(grid), dim3(kSgThreads), 0, s, static_cast<const float*>(a), offsets, E, N, K,
-                                                          static_cast<const float*>(w),
-                                                          static_cast<const float*>(bias), row_gate, out_rows,
-                                                          static_cast<float*>(c));
+    launch_err = launch_pdl(ffn_simt_f32_kernel<MODE>, dim3(grid), dim3(kSgThreads), 0, s,
+                            static_cast<const float*>(a), offsets, E, N, K, static_cast<const float*>(w),
+                            static_cast<const float*>(bias), row_gate, out_rows, static_cast<float*>(c), sa.g,
+                            static_cast<const float*>(sa.a), static_cast<const float*>(sa.w),
+                            static_cast<const float*>(sa.bias));
     return L.finish(launch_err);
 }
 
-// out_rows (nullable): fc2 writes grouped row r to row out_rows[r] of yp
-// (the direct output of a k == 1 layer, out_rows = perm)
+// The shared experts of a layer (S = 0: none): parameters [S, ...] and the
+// tokens x [T, d] they read.
+struct SharedExperts {
+    int S = 0;
+    int T = 0;
+    const void* x = nullptr;
+    const void *w1 = nullptr, *b1 = nullptr, *w2 = nullptr, *b2 = nullptr;
+};
+
+// Grouped FFN over the E routed groups (rows offsets[e] .. offsets[e+1]-1 of
+// xp, routed rows < max_rows) and the shared experts.  h and yp hold
+// max_rows routed rows followed by S * T shared rows (shared expert s, token
+// t at row max_rows + s * T + t).  out_rows (nullable): fc2 writes routed
+// row r to row out_rows[r] of yp (the direct output of a k == 1 layer).
 int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
             const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp, int dtype,
-            const int32_t* out_rows, cudaStream_t s) {
+            const int32_t* out_rows, const SharedExperts& se, cudaStream_t s) {
+    const int h_rows = max_rows + se.S * se.T;
+    SharedArgs s1, s2;
+    if (se.S > 0) {
+        // fc1 of shared expert s: A = x (every shared expert reads the same rows)
+        s1.a = se.x;
+        s1.a_rows = se.T;
+        s1.w = se.w1;
+        s1.bias = se.b1;
+        s1.g = SharedGroups{se.S, se.T, 0, 0, max_rows};
+        // fc2 of shared expert s: A = its rows of h
+        s2.a = h;
+        s2.a_rows = h_rows;
+        s2.w = se.w2;
+        s2.bias = se.b2;
+        s2.g = SharedGroups{se.S, se.T, max_rows, se.T, max_rows};
+    }
     int rc;
     if (dtype == MOE_BF16) {
-        rc = launch_tc<kTcBN, kTcStages, kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h,
-                                                   MOE_KERNEL_FFN1, s);
+        rc = launch_tc<kTcBN, kTcStages, kFc1Gelu>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr,
+                                                   nullptr, h, s1, MOE_KERNEL_FFN1, s);
         if (rc != MOE_OK) return rc;
-        return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp,
-                                                     MOE_KERNEL_FFN2, s);
+        return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate,
+                                                     out_rows, yp, s2, MOE_KERNEL_FFN2, s);
     }
-    rc = launch_simt<kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, MOE_KERNEL_FFN1, s);
+    rc = launch_simt<kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, s1, MOE_KERNEL_FFN1,
+                               s);
     if (rc != MOE_OK) return rc;
-    return launch_simt<kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, MOE_KERNEL_FFN2,
-                                 s);
+    return launch_simt<kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, s2,
+                                 MOE_KERNEL_FFN2, s);
 }
 
 // Dispatch of the fused forward path from the router's per-chunk histograms
 // and probability sums: one scan CTA (+ statistics), then the permute /
 // gather kernel over (chunk, G) CTAs.
+int permute_split(int nchunk) { return std::max(1, std::min(8, ceil_div(2 * num_sms(), nchunk))); }
+
 int run_forward_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int capacity, int chunk_tokens,
                          const int32_t* fhist, const float* fpsum, int32_t* fbase, int32_t* counts, int32_t* offsets,
-                         int32_t* perm, int32_t* slot_of, float* row_gate, moe_stats* st, const void* x, void* xp,
-                         int d, int dtype, void* out_zero_dropped, cudaStream_t s) {
+                         int32_t* perm, int32_t* slot_of, uint8_t* drop_mask, float* row_gate, moe_stats* st,
+                         const void* x, void* xp, int d, int dtype, void* out_zero_dropped, cudaStream_t s) {
     const int nchunk = ceil_div(T, chunk_tokens);
     int rc;
     {
         Launch L(MOE_KERNEL_SCAN, s);
         cudaError_t launch_err;
-        launch_err = launch_pdl(forward_scan_kernel, dim3(1), dim3(kFwdScanThreads), 0, s, fhist, fpsum, nchunk, E, T, k, capacity, fbase, counts,
-                                                       offsets, st);
+        launch_err = launch_pdl(forward_scan_kernel, dim3(1), dim3(kFwdScanThreads), 0, s, fhist, fpsum, nchunk, E,
+                                T, k, capacity, fbase, counts, offsets, st, static_cast<int32_t*>(nullptr));
         if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
     }
-    const int G = std::max(1, std::min(8, ceil_div(2 * num_sms(), nchunk)));
     const int row_bytes = int(size_t(d) * elem_bytes(dtype));
     Launch L(MOE_KERNEL_PERMUTE, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(forward_permute_kernel, dim3(dim3(nchunk, G)), dim3(kFwdThreads), 0, s, 
-        idx, gate, T, k, E, chunk_tokens, fbase, offsets, perm, slot_of, row_gate, static_cast<const uint8_t*>(x),
-        row_bytes, static_cast<uint8_t*>(xp), static_cast<uint8_t*>(out_zero_dropped));
+    launch_err = launch_pdl(forward_permute_kernel, dim3(nchunk, permute_split(nchunk)), dim3(kFwdThreads), 0, s,
+                            idx, gate, T, k, E, chunk_tokens, fbase, offsets, perm, slot_of, row_gate,
+                            static_cast<const uint8_t*>(x), row_bytes, static_cast<uint8_t*>(xp),
+                            static_cast<uint8_t*>(out_zero_dropped), drop_mask);
     return L.finish(launch_err);
 }
 
+// Dispatch with F >= 1 rerouting rounds (capacity >= 0), from per-chunk
+// histograms of the own choices: scan, F x (mark, scan), permute / gather.
+int run_reroute_dispatch(const int32_t* idx, const float* gate, const int32_t* fb_idx, const float* fb_gate, int T,
+                         int k, int E, int capacity, int F, int chunk_tokens, const int32_t* fhist,
+                         const float* fpsum, int32_t* fbase, int32_t* counts, int32_t* offsets, int32_t* perm,
+                         int32_t* slot_of, uint8_t* drop_mask, float* row_gate, moe_stats* st, const void* x,
+                         void* xp, int d, int dtype, void* out_zero_dropped, const RerouteWs& rw, cudaStream_t s) {
+    const int nchunk = ceil_div(T, chunk_tokens);
+    const size_t ce = size_t(nchunk) * E;
+    int rc;
+    {
+        Launch L(MOE_KERNEL_SCAN, s);
+        cudaError_t launch_err;
+        launch_err = launch_pdl(forward_scan_kernel, dim3(1), dim3(kFwdScanThreads), 0, s, fhist, fpsum, nchunk, E,
+                                T, k, capacity, fbase, counts, offsets, st, rw.load);
+        if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
+    }
+    for (int r = 1; r <= F; ++r) {
+        {
+            Launch L(MOE_KERNEL_REROUTE, s);
+            cudaError_t launch_err;
+            const int32_t* prev_rbase = r > 1 ? rw.rbase + size_t(r - 2) * ce : nullptr;
+            const int32_t* prev_acc = r > 1 ? rw.acc + size_t(r - 2) * E : nullptr;
+            launch_err = launch_pdl(reroute_mark_kernel, dim3(nchunk), dim3(kFwdThreads), 0, s, idx, T, k, E,
+                                    chunk_tokens, capacity, static_cast<const int32_t*>(fbase), fb_idx, F, r,
+                                    prev_rbase, prev_acc, rw.srv, rw.srank, rw.otok, rw.orank, rw.rhist);
+            if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
+        }
+        {
+            Launch L(MOE_KERNEL_REROUTE, s);
+            cudaError_t launch_err;
+            launch_err = launch_pdl(reroute_scan_kernel, dim3(1), dim3(kFwdScanThreads), 0, s,
+                                    static_cast<const int32_t*>(rw.rhist), nchunk, E, capacity, r, F, T, k,
+                                    rw.rbase + size_t(r - 1) * ce, rw.load, rw.acc + size_t(r - 1) * E,
+                                    rw.start + size_t(r - 1) * E, offsets, st);
+            if ((rc = L.finish(launch_err)) != MOE_OK) return rc;
+        }
+    }
+    const int row_bytes = int(size_t(d) * elem_bytes(dtype));
+    Launch L(MOE_KERNEL_PERMUTE, s);
+    cudaError_t launch_err;
+    launch_err = launch_pdl(reroute_permute_kernel, dim3(nchunk, permute_split(nchunk)), dim3(kFwdThreads), 0, s,
+                            idx, gate, fb_idx, fb_gate, T, k, E, F, chunk_tokens,
+                            static_cast<const int32_t*>(rw.srv), static_cast<const int32_t*>(rw.srank),
+                            static_cast<const int32_t*>(rw.otok), static_cast<const int32_t*>(rw.orank),
+                            static_cast<const int32_t*>(rw.rbase + size_t(F - 1) * ce),
+                            static_cast<const int32_t*>(rw.acc + size_t(F - 1) * E),
+                            static_cast<const int32_t*>(rw.start), static_cast<const int32_t*>(offsets), perm,
+                            slot_of, row_gate, static_cast<const uint8_t*>(x), row_bytes, static_cast<uint8_t*>(xp),
+                            static_cast<uint8_t*>(out_zero_dropped), drop_mask);
+    return L.finish(launch_err);
+}
+
+// ys (nullable when S == 0): [S, T, d] shared-expert outputs added with weight 1
 int run_combine(const void* yp, const int32_t* slot_of, const float* gate, int T, int k, int d, int dtype, void* out,
-                cudaStream_t s) {
+                const void* ys, int S, cudaStream_t s) {
     const int grid = std::max(1, std::min(ceil_div(T, 8), num_sms() * 16));
     Launch L(MOE_KERNEL_COMBINE, s);
     cudaError_t launch_err;
     if (dtype == MOE_BF16)
-        launch_err = launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(yp), slot_of, gate, T,
-                                                            k, d, static_cast<__nv_bfloat16*>(out));
+        launch_err = launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
+                                static_cast<const __nv_bfloat16*>(yp), slot_of, gate, T, k, d,
+                                static_cast<__nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(ys), S);
     else
-        launch_err = launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, static_cast<const float*>(yp), slot_of, gate, T, k, d,
-                                                   static_cast<float*>(out));
+        launch_err = launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, static_cast<const float*>(yp),
+                                slot_of, gate, T, k, d, static_cast<float*>(out), static_cast<const float*>(ys), S);
     return L.finish(launch_err);
 }
 
@@ -515,13 +713,25 @@ int moe_capacity(int T, int k, int E, double cf) {
 }
 
 size_t moe_workspace_size(int T, int d, int ff, int E, int k, int dtype) {
-    if (check_sizes(T, d, ff, E, k, dtype, true) != MOE_OK) return 0;
-    return ws_layout(T, d, ff, E, k, dtype).total;
+    return moe_forward_ex_workspace_size(T, d, ff, E, k, 0, 0, dtype);
+}
+
+size_t moe_forward_ex_workspace_size(int T, int d, int ff, int E, int k, int S, int F, int dtype) {
+    if (check_sizes(T, d, ff, E, k, dtype, true) != MOE_OK || check_shared(T, k, S) != MOE_OK ||
+        check_reroute(k, E, F) != MOE_OK)
+        return 0;
+    return ws_layout(T, d, ff, E, k, dtype, S, F).total;
 }
 
 size_t moe_workspace_offset(int T, int d, int ff, int E, int k, int dtype, int which) {
-    if (check_sizes(T, d, ff, E, k, dtype, true) != MOE_OK) return size_t(-1);
-    const WsLayout L = ws_layout(T, d, ff, E, k, dtype);
+    return moe_forward_ex_workspace_offset(T, d, ff, E, k, 0, 0, dtype, which);
+}
+
+size_t moe_forward_ex_workspace_offset(int T, int d, int ff, int E, int k, int S, int F, int dtype, int which) {
+    if (check_sizes(T, d, ff, E, k, dtype, true) != MOE_OK || check_shared(T, k, S) != MOE_OK ||
+        check_reroute(k, E, F) != MOE_OK)
+        return size_t(-1);
+    const WsLayout L = ws_layout(T, d, ff, E, k, dtype, S, F);
     switch (which) {
         case MOE_WS_TOPK_IDX: return L.idx;
         case MOE_WS_TOPK_GATE: return L.gate;
@@ -533,6 +743,8 @@ size_t moe_workspace_offset(int T, int d, int ff, int E, int k, int dtype, int w
         case MOE_WS_XP: return L.xp;
         case MOE_WS_H: return L.h;
         case MOE_WS_YP: return L.yp;
+        case MOE_WS_FALLBACK_IDX: return L.fb_idx;
+        case MOE_WS_FALLBACK_GATE: return L.fb_gate;
         default: return size_t(-1);
     }
 }
@@ -554,8 +766,8 @@ int moe_router_topk(const void* x, const void* w_router, const float* logit_bias
     }
     if (!x || !w_router || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
-    return run_router(x, w_router, logit_bias, T, d, E, k, dtype, topk_idx, topk_gate, prob_sum, nullptr, nullptr,
-                      static_cast<cudaStream_t>(stream));
+    RouterOut o{topk_idx, topk_gate, prob_sum, nullptr, nullptr, 0, nullptr, nullptr};
+    return run_router(x, w_router, logit_bias, T, d, E, k, dtype, o, static_cast<cudaStream_t>(stream));
 }
 
 int moe_dispatch(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E, int capacity,
@@ -612,6 +824,87 @@ int moe_dispatch_noalloc(const int32_t* topk_idx, const float* topk_gate, int T,
                         x, xp, d, dtype, scratch, s);
 }
 
+// step-level rerouting dispatch: chunks of kRerouteChunk tokens
+constexpr int kRerouteChunk = 128;
+
+struct RerouteStepWs {
+    size_t idx, gate, fb_idx, fb_gate, hist, base, reroute, total;
+};
+
+RerouteStepWs reroute_step_layout(int T, int k, int F, int E) {
+    RerouteStepWs L{};
+    const int nchunk = std::max(1, ceil_div(T, kRerouteChunk));
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t r = o;
+        o += align256(std::max<size_t>(bytes, 1));
+        return r;
+    };
+    L.idx = take(size_t(T) * k * 4);
+    L.gate = take(size_t(T) * k * 4);
+    L.fb_idx = take(size_t(T) * F * 4);
+    L.fb_gate = take(size_t(T) * F * 4);
+    L.hist = take(size_t(nchunk) * E * 4);
+    L.base = take(size_t(nchunk) * E * 4);
+    L.reroute = take(F > 0 ? reroute_ws_bytes(T, k, E, F, nchunk) : 0);
+    L.total = o;
+    return L;
+}
+
+size_t moe_dispatch_reroute_workspace_size(int T, int k, int F, int E) {
+    if (T < 0 || k < 1 || E < 1 || E > MOE_MAX_EXPERTS || check_reroute(k, E, F) != MOE_OK ||
+        static_cast<long long>(T) * (k + F) >= (1ll << 31))
+        return 0;
+    return reroute_step_layout(T, k, F, E).total;
+}
+
+int moe_dispatch_reroute(const int32_t* ranked_idx, const float* ranked_gate, int T, int k, int F, int E,
+                         int capacity, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                         uint8_t* drop_mask, float* row_gate, const void* x, void* xp, int d, int dtype, void* ws,
+                         size_t ws_bytes, void* stream) {
+    const bool want_rows = (x != nullptr || xp != nullptr);
+    int rc = want_rows ? check_sizes(T, d, 8, E, k, dtype, false) : check_sizes(T, 8, 8, E, k, MOE_F32, false);
+    if (rc != MOE_OK) return rc;
+    if ((rc = check_reroute(k, E, F)) != MOE_OK) return rc;
+    if (static_cast<long long>(T) * (k + F) >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (cudaMemsetAsync(counts, 0, size_t(E) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(offsets, 0, size_t(E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (want_rows && (!x || !xp || !aligned16(x) || !aligned16(xp))) return MOE_ERR_INVALID_ARG;
+    if (row_gate != nullptr && ranked_gate == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!ranked_idx || !perm || !slot_of) return MOE_ERR_INVALID_ARG;
+    const RerouteStepWs L = reroute_step_layout(T, k, F, E);
+    if (ws == nullptr || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return MOE_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
+    float* gate = reinterpret_cast<float*>(w + L.gate);
+    int32_t* fb_idx = reinterpret_cast<int32_t*>(w + L.fb_idx);
+    float* fb_gate = reinterpret_cast<float*>(w + L.fb_gate);
+    int32_t* hist = reinterpret_cast<int32_t*>(w + L.hist);
+    int32_t* base = reinterpret_cast<int32_t*>(w + L.base);
+    const int nchunk = ceil_div(T, kRerouteChunk);
+    {
+        Launch Lk(MOE_KERNEL_COUNT, s);
+        cudaError_t launch_err;
+        launch_err = launch_pdl(reroute_split_kernel, dim3(nchunk), dim3(kFwdThreads), 0, s, ranked_idx, ranked_gate,
+                                T, k, F, E, kRerouteChunk, idx, gate, fb_idx, fb_gate, hist);
+        if ((rc = Lk.finish(launch_err)) != MOE_OK) return rc;
+    }
+    // without x the permute kernels gather nothing (zero row bytes)
+    const int dd = want_rows ? d : 0;
+    if (F > 0 && capacity >= 0)
+        return run_reroute_dispatch(idx, gate, fb_idx, fb_gate, T, k, E, capacity, F, kRerouteChunk, hist, nullptr,
+                                    base, counts, offsets, perm, slot_of, drop_mask, row_gate, nullptr, x, xp, dd,
+                                    dtype, nullptr, carve_reroute_ws(w + L.reroute, T, k, E, F, nchunk), s);
+    return run_forward_dispatch(idx, gate, T, k, E, capacity, kRerouteChunk, hist, nullptr, base, counts, offsets,
+                                perm, slot_of, drop_mask, row_gate, nullptr, x, xp, dd, dtype, nullptr, s);
+}
+
 int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
                     const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp,
                     int dtype, void* stream) {
@@ -623,7 +916,29 @@ int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E,
         !aligned16(yp))
         return MOE_ERR_INVALID_ARG;
     return run_ffn(xp, offsets, max_rows, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype, nullptr,
-                   static_cast<cudaStream_t>(stream));
+                   SharedExperts{}, static_cast<cudaStream_t>(stream));
+}
+
+int moe_shared_ffn(const void* x, int T, int d, int ff, int S, const void* w1s, const void* b1s, const void* w2s,
+                   const void* b2s, void* h, void* ys, int dtype, void* stream) {
+    int rc = check_sizes(T, d, ff, 1, 1, dtype, true);
+    if (rc != MOE_OK) return rc;
+    if ((rc = check_shared(T, 0, S)) != MOE_OK) return rc;
+    if (T == 0 || S == 0) return MOE_OK;
+    if (!x || !w1s || !b1s || !w2s || !b2s || !h || !ys) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w1s) || !aligned16(b1s) || !aligned16(w2s) || !aligned16(b2s) ||
+        !aligned16(h) || !aligned16(ys))
+        return MOE_ERR_INVALID_ARG;
+    SharedExperts se;
+    se.S = S;
+    se.T = T;
+    se.x = x;
+    se.w1 = w1s;
+    se.b1 = b1s;
+    se.w2 = w2s;
+    se.b2 = b2s;
+    return run_ffn(nullptr, nullptr, 0, 0, d, ff, nullptr, nullptr, nullptr, nullptr, nullptr, h, ys, dtype,
+                   nullptr, se, static_cast<cudaStream_t>(stream));
 }
 
 int moe_combine(const void* yp, const int32_t* slot_of, const float* topk_gate, int T, int k, int d, int dtype,
@@ -633,7 +948,18 @@ int moe_combine(const void* yp, const int32_t* slot_of, const float* topk_gate, 
     if (T == 0) return MOE_OK;
     if (!yp || !slot_of || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    return run_combine(yp, slot_of, topk_gate, T, k, d, dtype, out, static_cast<cudaStream_t>(stream));
+    return run_combine(yp, slot_of, topk_gate, T, k, d, dtype, out, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+int moe_combine_shared(const void* yp, const int32_t* slot_of, const float* topk_gate, const void* ys, int S, int T,
+                       int k, int d, int dtype, void* out, void* stream) {
+    int rc = check_sizes(T, d, 8, k, k, dtype, false);
+    if (rc != MOE_OK) return rc;
+    if ((rc = check_shared(T, k, S)) != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!yp || !slot_of || !out || (S > 0 && !ys)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(yp) || !aligned16(out) || (S > 0 && !aligned16(ys))) return MOE_ERR_INVALID_ARG;
+    return run_combine(yp, slot_of, topk_gate, T, k, d, dtype, out, ys, S, static_cast<cudaStream_t>(stream));
 }
 
 int moe_layer_stats(const int32_t* counts, const int32_t* offsets, const float* prob_sum, int T, int k, int E,
@@ -649,14 +975,28 @@ int moe_forward(const void* x, const void* w_router, const float* logit_bias, co
                 const void* w2, const void* b2, int T, int d, int ff, int E, int k, int capacity, int dtype,
                 void* out, moe_stats* stats, int32_t* topk_idx_out, float* topk_gate_out, void* ws,
                 size_t ws_bytes, void* stream) {
+    return moe_forward_ex(x, w_router, logit_bias, w1, b1, w2, b2, 0, nullptr, nullptr, nullptr, nullptr, 0, T, d,
+                          ff, E, k, capacity, dtype, out, stats, topk_idx_out, topk_gate_out, ws, ws_bytes, stream);
+}
+
+int moe_forward_ex(const void* x, const void* w_router, const float* logit_bias, const void* w1, const void* b1,
+                   const void* w2, const void* b2, int S, const void* w1s, const void* b1s, const void* w2s,
+                   const void* b2s, int reroute_rounds, int T, int d, int ff, int E, int k, int capacity, int dtype,
+                   void* out, moe_stats* stats, int32_t* topk_idx_out, float* topk_gate_out, void* ws,
+                   size_t ws_bytes, void* stream) {
     int rc = check_sizes(T, d, ff, E, k, dtype, true);
     if (rc != MOE_OK) return rc;
+    if ((rc = check_shared(T, k, S)) != MOE_OK) return rc;
+    if ((rc = check_reroute(k, E, reroute_rounds)) != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
     if (!x || !w_router || !w1 || !b1 || !w2 || !b2 || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router) || !aligned16(w1) || !aligned16(b1) || !aligned16(w2) ||
         !aligned16(b2) || !aligned16(out))
         return MOE_ERR_INVALID_ARG;
-    const WsLayout L = ws_layout(T, d, ff, E, k, dtype);
+    if (S > 0 && (!w1s || !b1s || !w2s || !b2s || !aligned16(w1s) || !aligned16(b1s) || !aligned16(w2s) ||
+                  !aligned16(b2s)))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, ff, E, k, dtype, S, reroute_rounds);
     if (ws == nullptr || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
         return MOE_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -671,24 +1011,47 @@ int moe_forward(const void* x, const void* w_router, const float* logit_bias, co
     int32_t* fhist = reinterpret_cast<int32_t*>(w + L.fhist);
     int32_t* fbase = reinterpret_cast<int32_t*>(w + L.fbase);
     float* fpsum = stats ? reinterpret_cast<float*>(w + L.fpsum) : nullptr;   // only the statistics need it
+    int32_t* fb_idx = reinterpret_cast<int32_t*>(w + L.fb_idx);
+    float* fb_gate = reinterpret_cast<float*>(w + L.fb_gate);
     void* xp = w + L.xp;
     void* h = w + L.h;
     void* yp = w + L.yp;
     const int A = T * k;
-    // top-1: every token has one assignment, so fc2 writes the output row of
-    // its token directly (rows of dropped tokens are zeroed by the dispatch)
-    const bool direct = (k == 1);
+    const int chunk_tokens = router_chunk_tokens(dtype);
+    // rerouting only matters when a capacity can drop assignments
+    const int F = capacity >= 0 ? reroute_rounds : 0;
+    // top-1 without shared experts: every token has one contribution, so fc2
+    // writes the output row of its token directly (rows of dropped tokens
+    // are zeroed by the dispatch) and no combine runs
+    const bool direct = (k == 1 && S == 0);
+    SharedExperts se;
+    se.S = S;
+    se.T = T;
+    se.x = x;
+    se.w1 = w1s;
+    se.b1 = b1s;
+    se.w2 = w2s;
+    se.b2 = b2s;
 
-    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, idx, gate, nullptr, fpsum, fhist, s)) != MOE_OK)
-        return rc;
-    if ((rc = run_forward_dispatch(idx, gate, T, k, E, capacity, router_chunk_tokens(dtype), fhist, fpsum, fbase,
-                                   counts, offsets, perm, slot_of, row_gate, stats, x, xp, d, dtype,
-                                   direct ? out : nullptr, s)) != MOE_OK)
-        return rc;
+    RouterOut ro{idx, gate, nullptr, fpsum, fhist, F, fb_idx, fb_gate};
+    if ((rc = run_router(x, w_router, logit_bias, T, d, E, k, dtype, ro, s)) != MOE_OK) return rc;
+    if (F > 0)
+        rc = run_reroute_dispatch(idx, gate, fb_idx, fb_gate, T, k, E, capacity, F, chunk_tokens, fhist, fpsum,
+                                  fbase, counts, offsets, perm, slot_of, nullptr, row_gate, stats, x, xp, d, dtype,
+                                  direct ? out : nullptr,
+                                  carve_reroute_ws(w + L.reroute, T, k, E, F, ceil_div(T, chunk_tokens)), s);
+    else
+        rc = run_forward_dispatch(idx, gate, T, k, E, capacity, chunk_tokens, fhist, fpsum, fbase, counts, offsets,
+                                  perm, slot_of, nullptr, row_gate, stats, x, xp, d, dtype, direct ? out : nullptr,
+                                  s);
+    if (rc != MOE_OK) return rc;
     if ((rc = run_ffn(xp, offsets, A, E, d, ff, w1, b1, w2, b2, row_gate, h, direct ? out : yp, dtype,
-                      direct ? perm : nullptr, s)) != MOE_OK)
+                      direct ? perm : nullptr, se, s)) != MOE_OK)
         return rc;
-    if (!direct && (rc = run_combine(yp, slot_of, nullptr, T, k, d, dtype, out, s)) != MOE_OK) return rc;
+    if (!direct) {
+        const void* ys = static_cast<const uint8_t*>(yp) + size_t(A) * d * elem_bytes(dtype);
+        if ((rc = run_combine(yp, slot_of, nullptr, T, k, d, dtype, out, ys, S, s)) != MOE_OK) return rc;
+    }
     return MOE_OK;
 }
 

@@ -40,11 +40,15 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
 // prob_sum:  [E], accumulated with one atomicAdd per CTA and expert (caller zeroes it), or
 // psum_part: [gridDim.x][E] per-CTA sums (deterministic), and
 // hist:      [gridDim.x][E] per-CTA counts of the chosen experts; each may be null.
+// F > 0: the token's next F experts in the same order (its fallback experts
+// for overflow rerouting) go to fb_idx / fb_gate [T, F]; hist counts only
+// the first k.
 template <typename Tin, int EP>
 __global__ void __launch_bounds__(kRouterThreads)
 router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const float* __restrict__ bias,
                    int T, int d, int E, int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
-                   float* __restrict__ prob_sum, float* __restrict__ psum_part, int32_t* __restrict__ hist) {
+                   float* __restrict__ prob_sum, float* __restrict__ psum_part, int32_t* __restrict__ hist,
+                   int F, int32_t* __restrict__ fb_idx, float* __restrict__ fb_gate) {
     constexpr int EPT = EP / 16;          // experts per thread
     constexpr int NV = (EP + 31) / 32;    // expert values per lane in the softmax
     extern __shared__ __align__(16) float smem[];
@@ -147,7 +151,7 @@ router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const 
         for (int c = 0; c < NV; ++c) psum[c] += p[c] * inv;
 
         uint32_t taken = 0;
-        for (int j = 0; j < k; ++j) {
+        for (int j = 0; j < k + F; ++j) {
             float bv = -INFINITY;
             int be = 0x7fffffff;
 #pragma unroll
@@ -169,9 +173,14 @@ router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const 
             }
             if ((be & 31) == lane) taken |= 1u << (be >> 5);
             if (lane == 0) {
-                topk_idx[size_t(t) * k + j] = be;
-                topk_gate[size_t(t) * k + j] = expf(bv - m) * inv;
-                atomicAdd(&s_hist[be], 1);
+                if (j < k) {
+                    topk_idx[size_t(t) * k + j] = be;
+                    topk_gate[size_t(t) * k + j] = expf(bv - m) * inv;
+                    atomicAdd(&s_hist[be], 1);
+                } else {
+                    fb_idx[size_t(t) * F + (j - k)] = be;
+                    fb_gate[size_t(t) * F + (j - k)] = expf(bv - m) * inv;
+                }
             }
         }
     }
@@ -216,12 +225,14 @@ struct RtCfg {
     static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024;
 };
 
+// KMAX >= k + F: the selection also yields the F fallback experts (fb_idx /
+// fb_gate [T, F]), as in router_topk_kernel.
 template <int EP, int KMAX>
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ bias, int T, int d, int E, int k, int32_t* __restrict__ topk_idx,
                  float* __restrict__ topk_gate, float* __restrict__ prob_sum, float* __restrict__ psum_part,
-                 int32_t* __restrict__ hist) {
+                 int32_t* __restrict__ hist, int F, int32_t* __restrict__ fb_idx, float* __restrict__ fb_gate) {
     using Cfg = RtCfg<EP>;
     constexpr int S = Cfg::kStages;
     constexpr int NCH = (EP + 31) / 32;   // 32-column TMEM chunks
@@ -371,14 +382,20 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         if (valid && ok) {
 #pragma unroll
             for (int j = 0; j < KMAX; ++j) {
-                if (j < k) {
-                    // fewer than k finite logits cannot happen for k <= E with finite inputs;
+                if (j < k + F) {
+                    // fewer than k + F finite logits cannot happen for k + F <= E with finite inputs;
                     // guard so an all-NaN row still yields valid, distinct indices
                     int e = ti[j];
                     if (e >= E) e = j;
-                    topk_idx[size_t(t) * k + j] = e;
-                    topk_gate[size_t(t) * k + j] = (tv[j] == -INFINITY) ? 0.f : expf(tv[j] - m) * inv;
-                    atomicAdd(&s_hist[e], 1);
+                    const float g = (tv[j] == -INFINITY) ? 0.f : expf(tv[j] - m) * inv;
+                    if (j < k) {
+                        topk_idx[size_t(t) * k + j] = e;
+                        topk_gate[size_t(t) * k + j] = g;
+                        atomicAdd(&s_hist[e], 1);
+                    } else {
+                        fb_idx[size_t(t) * F + (j - k)] = e;
+                        fb_gate[size_t(t) * F + (j - k)] = g;
+                    }
                 }
             }
         }

@@ -41,6 +41,15 @@ class MoEParams:
     w2: torch.Tensor
     b2: torch.Tensor
     dtype: int
+    # shared always-on experts [S, ...] (None: no shared experts)
+    shared_w1: Optional[torch.Tensor] = None
+    shared_b1: Optional[torch.Tensor] = None
+    shared_w2: Optional[torch.Tensor] = None
+    shared_b2: Optional[torch.Tensor] = None
+
+    @property
+    def S(self):
+        return 0 if self.shared_w1 is None else self.shared_w1.shape[0]
 
     @property
     def E(self):
@@ -57,12 +66,16 @@ class MoEParams:
     @classmethod
     def from_arrays(cls, inputs: Dict[str, np.ndarray], dtype: int, device="cuda") -> "MoEParams":
         bias = inputs.get("logit_bias")
+        shared = {}
+        if inputs.get("shared_w1") is not None:
+            shared = {key: to_device(inputs[key], dtype, device)
+                      for key in ("shared_w1", "shared_b1", "shared_w2", "shared_b2")}
         return cls(
             w_router=to_device(inputs["w_router"], dtype, device),
             logit_bias=None if bias is None else torch.from_numpy(np.asarray(bias, np.float32)).to(device),
             w1=to_device(inputs["w1"], dtype, device), b1=to_device(inputs["b1"], dtype, device),
             w2=to_device(inputs["w2"], dtype, device), b2=to_device(inputs["b2"], dtype, device),
-            dtype=dtype)
+            dtype=dtype, **shared)
 
 
 def read_stats(stats_buf: torch.Tensor) -> Dict[str, float]:
@@ -72,12 +85,16 @@ def read_stats(stats_buf: torch.Tensor) -> Dict[str, float]:
 
 
 class MoELayer:
-    """One MoE layer bound to device parameters; reuses its workspace."""
+    """One MoE layer bound to device parameters (routed experts and, if the
+    parameters have them, shared always-on experts); reuses its workspace.
+    ``reroute`` > 0 gives assignments dropped at capacity that many rounds
+    of fallback experts (moe_forward_ex)."""
 
-    def __init__(self, params: MoEParams, k: int, capacity: int = -1):
+    def __init__(self, params: MoEParams, k: int, capacity: int = -1, reroute: int = 0):
         self.p = params
         self.k = k
         self.capacity = capacity
+        self.reroute = reroute
         self._ws = None
         self._ws_T = -1
         self.stats_buf = torch.zeros(ctypes.sizeof(_lib.MoeStats), dtype=torch.uint8,
@@ -85,7 +102,8 @@ class MoELayer:
 
     def workspace(self, T: int) -> torch.Tensor:
         if self._ws is None or self._ws_T < T:
-            n = _lib.moe_workspace_size(T, self.p.d, self.p.ff, self.p.E, self.k, self.p.dtype)
+            n = _lib.moe_forward_ex_workspace_size(T, self.p.d, self.p.ff, self.p.E, self.k, self.p.S,
+                                                   self.reroute, self.p.dtype)
             if n == 0:
                 raise ValueError("invalid layer sizes")
             self._ws = torch.empty(n, dtype=torch.uint8, device=self.p.w1.device)
@@ -102,9 +120,15 @@ class MoELayer:
             out = torch.empty_like(x)
         ws = self.workspace(T)
         p = self.p
-        _lib.moe_forward(x, p.w_router, p.logit_bias, p.w1, p.b1, p.w2, p.b2, T, p.d, p.ff, p.E, self.k,
-                         self.capacity, p.dtype, out, self.stats_buf if stats else None, topk_idx, topk_gate,
-                         ws, ws.numel(), stream)
+        if p.S == 0 and self.reroute == 0:
+            _lib.moe_forward(x, p.w_router, p.logit_bias, p.w1, p.b1, p.w2, p.b2, T, p.d, p.ff, p.E, self.k,
+                             self.capacity, p.dtype, out, self.stats_buf if stats else None, topk_idx, topk_gate,
+                             ws, ws.numel(), stream)
+        else:
+            _lib.moe_forward_ex(x, p.w_router, p.logit_bias, p.w1, p.b1, p.w2, p.b2, p.S, p.shared_w1,
+                                p.shared_b1, p.shared_w2, p.shared_b2, self.reroute, T, p.d, p.ff, p.E, self.k,
+                                self.capacity, p.dtype, out, self.stats_buf if stats else None, topk_idx,
+                                topk_gate, ws, ws.numel(), stream)
         return out
 
     __call__ = forward
@@ -112,7 +136,8 @@ class MoELayer:
     def workspace_view(self, T: int, which: str, dtype, count: int) -> torch.Tensor:
         """A view of one of moe_forward's intermediate arrays in the workspace
         (valid after a forward call on T tokens; for inspection and tests)."""
-        off = _lib.moe_workspace_offset(T, self.p.d, self.p.ff, self.p.E, self.k, self.p.dtype, which)
+        off = _lib.moe_forward_ex_workspace_offset(T, self.p.d, self.p.ff, self.p.E, self.k, self.p.S,
+                                                   self.reroute, self.p.dtype, which)
         ws = self.workspace(T)
         nbytes = count * torch.tensor([], dtype=dtype).element_size()
         return ws[off:off + nbytes].view(dtype)

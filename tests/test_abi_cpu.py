@@ -128,3 +128,89 @@ def test_no_launch_and_timing_read_without_gpu(lib):
     assert lib.moe_timing_enable(0) == _lib.MOE_OK
     t = _lib.moe_timing_read()
     assert set(t) == set(_lib.KERNEL_NAMES) and all(v == (0.0, 0) for v in t.values())
+
+
+def test_shared_workspace_size_and_offsets(lib):
+    T, d, ff, E, k = 4096, 768, 3072, 32, 1
+    base = _lib.moe_workspace_size(T, d, ff, E, k, _lib.MOE_BF16)
+    assert _lib.moe_forward_ex_workspace_size(T, d, ff, E, k, 0, 0, _lib.MOE_BF16) == base
+    two = _lib.moe_forward_ex_workspace_size(T, d, ff, E, k, 2, 0, _lib.MOE_BF16)
+    assert two >= base + 2 * T * (ff + d) * 2          # S*T more rows of h and yp
+    # routed rows first, then the shared rows: yp holds (T*k + S*T) rows
+    yp = _lib.moe_forward_ex_workspace_offset(T, d, ff, E, k, 2, 0, _lib.MOE_BF16, "yp")
+    h = _lib.moe_forward_ex_workspace_offset(T, d, ff, E, k, 2, 0, _lib.MOE_BF16, "h")
+    assert yp - h >= (T * k + 2 * T) * ff * 2
+    assert _lib.moe_forward_ex_workspace_size(T, d, ff, E, k, _lib.MOE_MAX_SHARED + 1, 0, _lib.MOE_BF16) == 0
+    assert _lib.moe_forward_ex_workspace_size(T, d, ff, E, k, -1, 0, _lib.MOE_BF16) == 0
+    assert _lib.moe_forward_ex_workspace_size(1 << 28, d, ff, E, k, 7, 0, _lib.MOE_BF16) == 0   # T*(k+S) overflows
+
+
+def forward_shared(lib, ws_bytes, ws=FAKE, S=2, shared=FAKE, F=0, **kw):
+    a = dict(T=256, d=64, ff=128, E=8, k=2, cap=-1, dtype=_lib.MOE_BF16, out=FAKE)
+    a.update(kw)
+    return lib.moe_forward_ex(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, S, shared, FAKE, FAKE, FAKE, F,
+                              a["T"], a["d"], a["ff"], a["E"], a["k"], a["cap"], a["dtype"], a["out"], None,
+                              None, None, ws, ws_bytes, None)
+
+
+def test_forward_shared_checks(lib):
+    need = _lib.moe_forward_ex_workspace_size(256, 64, 128, 8, 2, 2, 0, _lib.MOE_BF16)
+    assert need > _lib.moe_workspace_size(256, 64, 128, 8, 2, _lib.MOE_BF16)
+    assert forward_shared(lib, need - 1) == _lib.MOE_ERR_WORKSPACE
+    assert forward_shared(lib, need, shared=None) == _lib.MOE_ERR_INVALID_ARG
+    assert forward_shared(lib, need, shared=MISALIGNED) == _lib.MOE_ERR_INVALID_ARG
+    assert forward_shared(lib, need, S=-1) == _lib.MOE_ERR_INVALID_ARG
+    assert forward_shared(lib, need, S=_lib.MOE_MAX_SHARED + 1) == _lib.MOE_ERR_UNSUPPORTED
+    assert forward_shared(lib, 0, T=0) == _lib.MOE_OK
+    # S = 0 needs no shared pointers and exactly moe_forward's workspace
+    base = _lib.moe_workspace_size(256, 64, 128, 8, 2, _lib.MOE_BF16)
+    assert forward_shared(lib, base - 1, S=0, shared=None) == _lib.MOE_ERR_WORKSPACE
+
+
+def test_shared_ffn_and_combine_checks(lib):
+    call = lambda **kw: lib.moe_shared_ffn(kw.get("x", FAKE), kw.get("T", 64), 64, 128, kw.get("S", 2),
+                                           kw.get("w1", FAKE), FAKE, FAKE, FAKE, kw.get("h", FAKE), FAKE,
+                                           _lib.MOE_BF16, None)
+    assert call(x=None) == _lib.MOE_ERR_INVALID_ARG
+    assert call(w1=MISALIGNED) == _lib.MOE_ERR_INVALID_ARG
+    assert call(h=None) == _lib.MOE_ERR_INVALID_ARG
+    assert call(S=9) == _lib.MOE_ERR_UNSUPPORTED
+    assert call(S=0, x=None) == _lib.MOE_OK          # nothing to do
+    assert call(T=0, x=None) == _lib.MOE_OK
+    comb = lambda **kw: lib.moe_combine_shared(FAKE, FAKE, None, kw.get("ys", FAKE), kw.get("S", 2), 64, 2, 64,
+                                               _lib.MOE_BF16, FAKE, None)
+    assert comb(ys=None) == _lib.MOE_ERR_INVALID_ARG
+    assert comb(ys=MISALIGNED) == _lib.MOE_ERR_INVALID_ARG
+    assert comb(S=9) == _lib.MOE_ERR_UNSUPPORTED
+    assert comb(S=-1) == _lib.MOE_ERR_INVALID_ARG
+
+
+def test_reroute_checks(lib):
+    # workspace grows with the rounds; k + F must fit the router's selection and E
+    base = _lib.moe_forward_ex_workspace_size(4096, 768, 3072, 32, 1, 0, 0, _lib.MOE_BF16)
+    one = _lib.moe_forward_ex_workspace_size(4096, 768, 3072, 32, 1, 0, 1, _lib.MOE_BF16)
+    three = _lib.moe_forward_ex_workspace_size(4096, 768, 3072, 32, 1, 0, 3, _lib.MOE_BF16)
+    assert base < one < three
+    assert _lib.moe_forward_ex_workspace_size(4096, 768, 3072, 32, 2, 0, 7, _lib.MOE_BF16) == 0   # k + F > 8
+    assert _lib.moe_forward_ex_workspace_size(64, 64, 64, 3, 2, 0, 2, _lib.MOE_BF16) == 0         # k + F > E
+    assert _lib.moe_forward_ex_workspace_size(64, 64, 64, 3, 2, 0, -1, _lib.MOE_BF16) == 0
+    fb = _lib.moe_forward_ex_workspace_offset(4096, 768, 3072, 32, 1, 0, 2, _lib.MOE_BF16, "fallback_idx")
+    fg = _lib.moe_forward_ex_workspace_offset(4096, 768, 3072, 32, 1, 0, 2, _lib.MOE_BF16, "fallback_gate")
+    assert fg - fb >= 4096 * 2 * 4
+    need = _lib.moe_forward_ex_workspace_size(256, 64, 128, 8, 2, 0, 2, _lib.MOE_BF16)
+    assert forward_shared(lib, need - 1, S=0, shared=None, F=2, cap=10) == _lib.MOE_ERR_WORKSPACE
+    assert forward_shared(lib, need, S=0, shared=None, F=7, cap=10) == _lib.MOE_ERR_UNSUPPORTED
+    assert forward_shared(lib, need, S=0, shared=None, F=-2, cap=10) == _lib.MOE_ERR_INVALID_ARG
+    # step form
+    nws = _lib.moe_dispatch_reroute_workspace_size(1000, 2, 2, 8)
+    assert nws > 0 and _lib.moe_dispatch_reroute_workspace_size(1000, 2, 7, 8) == 0
+    call = lambda **kw: lib.moe_dispatch_reroute(
+        kw.get("idx", FAKE), kw.get("gate", None), 1000, 2, kw.get("F", 2), 8, 100, FAKE, FAKE, FAKE, FAKE, None,
+        kw.get("row_gate", None), kw.get("x", None), kw.get("xp", None), 64, _lib.MOE_BF16,
+        kw.get("ws", FAKE), kw.get("ws_bytes", nws), None)
+    assert call(ws_bytes=nws - 1) == _lib.MOE_ERR_WORKSPACE
+    assert call(ws=FAKE + 16) == _lib.MOE_ERR_WORKSPACE
+    assert call(row_gate=FAKE) == _lib.MOE_ERR_INVALID_ARG
+    assert call(idx=None) == _lib.MOE_ERR_INVALID_ARG
+    assert call(x=FAKE) == _lib.MOE_ERR_INVALID_ARG
+    assert call(F=7) == _lib.MOE_ERR_UNSUPPORTED
