@@ -306,6 +306,35 @@ def algorithmic_bytes(kernel, w, R, E_active, es):
     return None
 
 
+def copy_bandwidth(x_host, out_host, x_dev, out_dev, reps: int = 20):
+    """Host<->device copy rates of one step's input and output (pinned, each
+    direction alone, then both at once), GB/s: the ceiling of the end-to-end
+    number."""
+    import torch
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    res = {}
+    for name, streams in (("h2d", [s_in]), ("d2h", [s_out]), ("both", [s_in, s_out])):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for st in streams:
+            st.wait_event(e0)
+        for _ in range(reps):
+            if s_in in streams:
+                with torch.cuda.stream(s_in):
+                    x_dev.copy_(x_host, non_blocking=True)
+            if s_out in streams:
+                with torch.cuda.stream(s_out):
+                    out_host.copy_(out_dev, non_blocking=True)
+        for st in streams:
+            torch.cuda.current_stream().wait_stream(st)
+        e1.record()
+        torch.cuda.synchronize()
+        nbytes = reps * x_host.numel() * x_host.element_size() * len(streams)
+        res[name] = nbytes / (e0.elapsed_time(e1) / 1000.0) / 1e9
+    return res
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -426,6 +455,7 @@ def run_ours(args):
         dist.barrier()
     e2e_value = whole_job_tokens_per_s(world, e2e_steps, w.T, e2e_ms)
     io_bytes = x.numel() * x.element_size()
+    pcie = copy_bandwidth(x_hosts[0], out_hosts[0], pipe.x_dev[0], pipe.out_dev[0])
     # the device result of the last step equals the device-only forward
     ref_out = layer.forward(x)
     torch.cuda.synchronize()
@@ -484,7 +514,9 @@ def run_ours(args):
         "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
                 "d2h_bytes_per_step": io_bytes, "steps": e2e_steps,
-                "mode": "pinned host buffers; H2D, layer and D2H of consecutive steps overlap on three streams"},
+                "mode": "pinned host buffers; H2D, layer (a CUDA graph per lane) and D2H of consecutive steps "
+                        "overlap on three streams, three lanes",
+                "copy_gbs": pcie},
         "clocks": clocks,
         "gpu_launches": launches,
         "stats": {k: st[k] for k in ("aux_loss", "imbalance", "drop_rate", "rerouted")},

@@ -30,6 +30,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// GPU-scope acquire load / release store of a 64-bit flag (one CTA publishes
+// data, another waits for the flag before reading it)
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // programmatic dependent launch: every kernel is launched allowed to start
 // before the previous kernel on the stream has finished.  It calls

@@ -443,6 +443,141 @@ forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict_
     gather_chunk_rows(slot_s, a0, na, k, x, row_bytes, xp, out_zero_dropped);
 }
 
+// The scan fused into the permute: every CTA of chunk c derives what the
+// one-CTA scan would give it from the router's per-chunk histograms (its
+// bases: counts of each expert in chunks before c; the totals, capacity
+// clamp and offsets), so the dispatch is one launch.  CTA (0, 0) also
+// writes counts, offsets and the statistics.  Each CTA reads nchunk * E
+// histogram entries, so the host uses this only while that table is small.
+// Thread e < E owns expert e (E <= MOE_MAX_EXPERTS = kFwdThreads).
+static_assert(MOE_MAX_EXPERTS <= kFwdThreads, "one thread per expert");
+
+__global__ void __launch_bounds__(kFwdThreads)
+forward_dispatch_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, int T, int k, int E,
+                        int chunk_tokens, const int32_t* __restrict__ hist, const float* __restrict__ psum_part,
+                        int nchunk, int capacity, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                        moe_stats* __restrict__ st, int32_t* __restrict__ perm, int32_t* __restrict__ slot_of,
+                        float* __restrict__ row_gate, const uint8_t* __restrict__ x, int row_bytes,
+                        uint8_t* __restrict__ xp, uint8_t* __restrict__ out_zero_dropped) {
+    pdl_wait();
+    pdl_release();
+    __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
+    __shared__ int off_s[MOE_MAX_EXPERTS + 1];
+    __shared__ int base_s[MOE_MAX_EXPERTS];
+    __shared__ int kept_s[MOE_MAX_EXPERTS];
+    __shared__ int cnt_s[MOE_MAX_EXPERTS];
+    __shared__ float fp_s[MOE_MAX_EXPERTS];
+    __shared__ int slot_s[kFwdMaxChunk];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int chunk = blockIdx.x;
+    const bool lead = (blockIdx.x == 0 && blockIdx.y == 0);
+    const int A = T * k;
+    const int a0 = chunk * chunk_tokens * k;
+    const int na = min(chunk_tokens * k, A - a0);
+
+    if (tid < E) {
+        const int e = tid;
+        int pre = 0, tot = 0;
+        float ps = 0.f;
+#pragma unroll 8
+        for (int b = 0; b < nchunk; ++b) {
+            const int h = hist[size_t(b) * E + e];
+            tot += h;
+            pre += (b < chunk) ? h : 0;
+        }
+        if (lead && st != nullptr && psum_part != nullptr)
+            for (int b = 0; b < nchunk; ++b) ps += psum_part[size_t(b) * E + e];
+        base_s[e] = pre;
+        cnt_s[e] = tot;
+        kept_s[e] = capacity < 0 ? tot : min(tot, capacity);
+        fp_s[e] = (float(tot) / float(T)) * (ps / float(T));
+        if (lead) counts[e] = tot;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        constexpr int PER = MOE_MAX_EXPERTS / 32;
+        int local[PER];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            local[i] = e < E ? kept_s[e] : 0;
+            sum += local[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            if (e < E) off_s[e] = run;
+            run += local[i];
+        }
+        if (lane == 31) off_s[E] = incl;
+        if (lead && st != nullptr) {
+            // statistics, in a fixed summation order
+            float f = 0.f;
+            int mx = 0;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = lane * PER + i;
+                if (e < E) {
+                    f += fp_s[e];
+                    mx = max(mx, cnt_s[e]);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                f += __shfl_xor_sync(0xffffffffu, f, o);
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            if (lane == 31) {
+                const int R = incl;
+                st->aux_loss = float(E) * f;
+                st->imbalance = float(mx) / (float(A) / float(E));
+                st->drop_rate = float(A - R) / float(A);
+                st->rows_kept = R;
+                st->max_count = mx;
+                st->dropped = A - R;
+                st->rerouted = 0;
+            }
+        }
+    }
+    __syncthreads();
+    if (lead)
+        for (int e = tid; e <= E; e += kFwdThreads) offsets[e] = off_s[e];
+
+    int ex[kFwdRankRounds], rank[kFwdRankRounds];
+    const int per = chunk_stable_ranks(idx, a0, na, E, wcnt, ex, rank);
+    const bool writer = blockIdx.y == 0;
+#pragma unroll
+    for (int r = 0; r < kFwdRankRounds; ++r) {
+        const int i = warp * per + r * 32 + lane;
+        if (!((r * 32 < per) && i < na)) continue;
+        const int a = a0 + i;
+        const int e = ex[r];
+        int slot = -1;
+        if (e >= 0) {
+            const int g = base_s[e] + wcnt[warp][e] + rank[r];
+            if (g < off_s[e + 1] - off_s[e]) slot = off_s[e] + g;
+        }
+        slot_s[i] = slot;
+        if (writer) {
+            slot_of[a] = slot;
+            if (slot >= 0) {
+                perm[slot] = a;
+                if (row_gate != nullptr) row_gate[slot] = gate[a];
+            }
+        }
+    }
+    __syncthreads();
+    gather_chunk_rows(slot_s, a0, na, k, x, row_bytes, xp, out_zero_dropped);
+}
+
 // ---------------------------------------------------------------------------
 // Overflow rerouting (F rounds).  Round r = 1..F: every token with an
 // unserved slot offers its first unserved slot j to its r-th fallback

@@ -41,6 +41,7 @@ struct TileTable {
     int arow[kMaxGroups];        // first A row of each group
     int crow[kMaxGroups];        // first C row (and row_gate / out_rows index)
     int rows[kMaxGroups];        // rows of each group
+    int routed_tiles;            // start[E]: tiles of the routed groups
 };
 
 // Must be called by all threads of the CTA; ends with __syncthreads().
@@ -96,13 +97,27 @@ __device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ off
         if (lane == 31) tt.start[G] = incl;
     }
     __syncthreads();
+    if (threadIdx.x == 0) tt.routed_tiles = tt.start[E];
+    __syncthreads();
 }
 
 struct TileCoord {
     int e, mt, nt;   // e: group (routed expert, or E + shared expert)
 };
 
+// Position t of the walk -> tile.  With both routed and shared groups the
+// walk interleaves them in proportion (position t is routed tile
+// floor(t*Rt/N) when that count steps at t, else shared tile t - that
+// count; a bijection since Rt <= N), so the CTAs running at any moment mix
+// routed tiles, which stream their weight panels from HBM, with shared
+// tiles, whose panels stay in L2 across their many M tiles.
 __device__ __forceinline__ TileCoord decode_tile(const TileTable& tt, int G, int t) {
+    const int total = tt.start[G], rt = tt.routed_tiles;
+    if (rt > 0 && rt < total) {
+        const int r0 = int((long long)t * rt / total);
+        const int r1 = int((long long)(t + 1) * rt / total);
+        t = (r1 > r0) ? r0 : rt + (t - r0);
+    }
     int lo = 0, hi = G - 1;   // last g with start[g] <= t (groups with no tiles are skipped)
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -255,6 +270,83 @@ struct TcCfg {
     static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;   // + alignment slack
 };
 
+// Work split of one launch (G = gridDim.x CTAs).  Without partials
+// (classic): CTA b takes whole tiles b, b + G, b + 2G, ...  With partials
+// (stream-K hybrid): all but the last one to two waves of tiles go whole,
+// round-robin as in the classic split (CTAs running together share weight
+// panels and A rows through L2); the remaining tiles' k-block units are cut
+// into G contiguous ranges [b*U/G, (b+1)*U/G), so the tail of the launch is
+// spread over every SM instead of leaving most of them idle.  A range
+// splits at most its first and last tile.  The CTA that covers a split
+// tile's first k-block finishes it: the CTAs after it, which cover the rest
+// of that tile at the start of their ranges, write fp32 partial tiles to
+// partials[c] and publish flags[c] = epoch; the finisher waits for them
+// (bounded), adds them in CTA order and runs the epilogue.  A CTA ends its
+// range with the tile it finishes, so it waits for work the next CTAs did
+// first.
+struct StreamK {
+    float* partials;               // [gridDim.x][kTcBM][BN] fp32, or null: classic split
+    unsigned long long* flags;     // [gridDim.x]; a finisher clears the flags it consumed
+    unsigned long long epoch;      // unique per host launch call (never 0)
+};
+
+enum SegKind { kSegFull = 0, kSegFinish = 1, kSegPartial = 2 };
+
+struct Seg {
+    int pos;    // tile position of the walk (decode_tile maps it to a tile)
+    int kb0, kb1;
+    int kind;
+};
+
+// The segments of this CTA's work, in order; every warp role walks the same
+// sequence.
+struct SegWalk {
+    int total, KB, G;
+    int dp;            // tiles handed out whole, round-robin
+    long long U;       // k-block units of the split tail
+    int t;             // next whole tile
+    long long u, u1;   // split tail: unit cursor and end
+    __device__ __forceinline__ SegWalk(int total_, int KB_, bool sk) : total(total_), KB(KB_), G(int(gridDim.x)) {
+        dp = total;
+        if (sk) {
+            const int waves = total / G;
+            dp = waves >= 2 ? (waves - 1) * G : 0;
+        }
+        U = (long long)(total - dp) * KB;
+        t = int(blockIdx.x);
+        u = range_begin(int(blockIdx.x));
+        u1 = range_begin(int(blockIdx.x) + 1);
+    }
+    __device__ __forceinline__ long long range_begin(int c) const { return U * c / G; }
+    __device__ __forceinline__ bool next(Seg& sg) {
+        if (t < dp) {
+            sg.pos = t;
+            sg.kb0 = 0;
+            sg.kb1 = KB;
+            sg.kind = kSegFull;
+            t += G;
+            return true;
+        }
+        if (u >= u1) return false;
+        const int local = int(u / KB);
+        sg.pos = dp + local;
+        sg.kb0 = int(u - (long long)local * KB);
+        const long long rem = u1 - u;
+        sg.kb1 = (rem < (long long)(KB - sg.kb0)) ? sg.kb0 + int(rem) : KB;
+        sg.kind = (sg.kb0 > 0) ? kSegPartial : (sg.kb1 < KB ? kSegFinish : kSegFull);
+        u += sg.kb1 - sg.kb0;
+        return true;
+    }
+    // last CTA holding part of split tile `pos` (whose first k-block this CTA holds)
+    __device__ __forceinline__ int last_contributor(int pos) const {
+        const long long tile_end = (long long)(pos - dp + 1) * KB;
+        int c = int(blockIdx.x);
+        while (c + 1 < G && range_begin(c + 1) < tile_end) ++c;
+        return c;
+    }
+    __device__ __forceinline__ bool range_empty(int c) const { return range_begin(c) >= range_begin(c + 1); }
+};
+
 // tmA2 / tmB2 / bias2: the shared experts' A rows and parameters (used when sh.S > 0)
 template <int BN, int STAGES, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -263,7 +355,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                    const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
                    const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C, SharedGroups sh,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                   const __nv_bfloat16* __restrict__ bias2) {
+                   const __nv_bfloat16* __restrict__ bias2, StreamK skp) {
     using Cfg = TcCfg<BN, STAGES>;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN: whole 32-column epilogue chunks, MMA N <= 256");
     __shared__ TileTable tt;
@@ -271,6 +363,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
+    __shared__ int partial_ok;
     __shared__ float sbias[BN];
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
@@ -307,6 +400,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     const int G = E + sh.S;
     const int total = tt.start[G];
     const int KB = (K + kTcBK - 1) / kTcBK;
+    const bool sk = skp.partials != nullptr;
     volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
@@ -317,15 +411,17 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             int last_parity[STAGES];
             for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const TileCoord tc = decode_tile(tt, G, t);
+            SegWalk walk(total, KB, sk);
+            Seg sg;
+            while (ok && walk.next(sg)) {
+                const TileCoord tc = decode_tile(tt, G, sg.pos);
                 const bool shared_g = tc.e >= E;
                 const CUtensorMap* ma = shared_g ? &tmA2 : &tmA;
                 const CUtensorMap* mb = shared_g ? &tmB2 : &tmB;
                 const int widx = shared_g ? tc.e - E : tc.e;
                 const int row0 = tt.arow[tc.e] + tc.mt * kTcBM;
                 const int n0 = tc.nt * BN;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) { ok = false; break; }
                     uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
                     uint8_t* sb = sa + Cfg::kABytes;
@@ -355,11 +451,13 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            SegWalk walk(total, KB, sk);
+            Seg sg;
+            while (ok && walk.next(sg)) {
                 if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_p)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, abort_p)) { ok = false; break; }
                     tc_fence_after();
                     const uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
@@ -368,7 +466,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
 #pragma unroll
                     for (int kk = 0; kk < kTcBK / 16; ++kk)
                         umma_f16(d_tmem, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc,
-                                 (kb > 0 || kk > 0) ? 1u : 0u);
+                                 (kb > sg.kb0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty_bar[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -388,17 +486,20 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         const int etid = threadIdx.x - 64;   // 0..255
         const int q = warp & 3;              // TMEM lane quarter this warp may access
         const int half = (warp - 2) >> 2;    // which alternate 32-column chunks
+        const int row_in_tile = q * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool failed = false;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        SegWalk walk(total, KB, sk);
+        Seg sg;
+        while (walk.next(sg)) {
             // all epilogue warps stop together once any wait has given up, so
             // none is left behind at a named barrier
             if (named_bar_red_or(1, 32 * kTcEpiWarps, failed || *abort_p)) break;
-            const TileCoord tc = decode_tile(tt, G, t);
+            const TileCoord tc = decode_tile(tt, G, sg.pos);
             const bool shared_g = tc.e >= E;
             const int rows = tt.rows[tc.e];
-            const int r_in = tc.mt * kTcBM + q * 32 + lane;
+            const int r_in = tc.mt * kTcBM + row_in_tile;
             const bool valid = r_in < rows;
             const size_t grow = size_t(tt.crow[tc.e]) + r_in;
             // destination row: the grouped row, or (direct output of a routed
@@ -411,41 +512,118 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             // (the barrier above also ends every read of the previous tile's bias)
             for (int i = etid; i < BN; i += 32 * kTcEpiWarps)
                 sbias[i] = (n0 + i < N) ? __bfloat162float(bb[n0 + i]) : 0.f;
-            named_bar_sync(1, 32 * kTcEpiWarps);   // this tile's bias is visible
-            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_p)) {
-                failed = true;
-                continue;
-            }
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = half; c < BN / 32; c += 2) {
-                uint32_t r[32];
-                __syncwarp();
-                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
-                tmem_ld_wait();
-                const int nb = n0 + c * 32;
-                if (!valid || nb >= N) continue;
-                __nv_bfloat16* cp = C + crow * N + nb;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    if (nb + v * 8 >= N) break;
-                    float o[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float cval = __uint_as_float(r[v * 8 + i]) + sbias[c * 32 + v * 8 + i];
-                        o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
+            // the CTAs after this one that hold the rest of a tile it finishes
+            int c_last = int(blockIdx.x);
+            if (sg.kind == kSegFinish) {
+                c_last = walk.last_contributor(sg.pos);
+                if (etid == 0) {
+                    int ok_all = 1;
+                    for (int c = int(blockIdx.x) + 1; c <= c_last; ++c) {
+                        if (walk.range_empty(c)) continue;
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire_u64(skp.flags + c) != skp.epoch) {
+                            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                                set_error(MOE_ERR_TIMEOUT);
+                                ok_all = 0;
+                                break;
+                            }
+                        }
+                        if (!ok_all) break;
                     }
-                    uint4 u;
-                    u.x = pack_bf16x2(o[0], o[1]);
-                    u.y = pack_bf16x2(o[2], o[3]);
-                    u.z = pack_bf16x2(o[4], o[5]);
-                    u.w = pack_bf16x2(o[6], o[7]);
-                    *reinterpret_cast<uint4*>(cp + v * 8) = u;
+                    partial_ok = ok_all;
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+            named_bar_sync(1, 32 * kTcEpiWarps);   // bias and partial flags visible
+            if (sg.kind == kSegFinish && !partial_ok) failed = true;
+            // every epilogue warp takes the same barriers below whether or not
+            // its wait succeeded; a failed warp only skips the work
+            // (uniform per warp: the TMEM loads below are warp-collective)
+            const bool got = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_p));
+            if (!got) failed = true;
+            tc_fence_after();
+            if (sg.kind == kSegPartial) {
+                // raw fp32 accumulators of this CTA's share of the tile
+                float* dst = skp.partials + (size_t(blockIdx.x) * kTcBM + row_in_tile) * BN;
+                if (got) {
+#pragma unroll 1
+                    for (int c = half; c < BN / 32; c += 2) {
+                        uint32_t r[32];
+                        __syncwarp();
+                        tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            *reinterpret_cast<uint4*>(dst + c * 32 + v * 4) =
+                                make_uint4(r[v * 4], r[v * 4 + 1], r[v * 4 + 2], r[v * 4 + 3]);
+                    }
+                    __threadfence();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0 && got) mbar_arrive(&tempty_bar[acc]);
+                // every thread's partial is written and fenced; publish it
+                // only if no warp gave up
+                const bool any_failed = named_bar_red_or(1, 32 * kTcEpiWarps, !got);
+                if (etid == 0 && !any_failed) st_release_u64(skp.flags + blockIdx.x, skp.epoch);
+            } else {
+                if (got) {
+#pragma unroll 1
+                    for (int c = half; c < BN / 32; c += 2) {
+                        uint32_t r[32];
+                        __syncwarp();
+                        tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
+                        tmem_ld_wait();
+                        const int nb = n0 + c * 32;
+                        if (!valid || nb >= N) continue;
+                        float a[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
+                        if (sg.kind == kSegFinish) {
+                            for (int cc = int(blockIdx.x) + 1; cc <= c_last; ++cc) {
+                                if (walk.range_empty(cc)) continue;
+                                const float* src =
+                                    skp.partials + (size_t(cc) * kTcBM + row_in_tile) * BN + c * 32;
+#pragma unroll
+                                for (int v = 0; v < 8; ++v) {
+                                    const float4 pv = __ldcg(reinterpret_cast<const float4*>(src) + v);
+                                    a[v * 4] += pv.x;
+                                    a[v * 4 + 1] += pv.y;
+                                    a[v * 4 + 2] += pv.z;
+                                    a[v * 4 + 3] += pv.w;
+                                }
+                            }
+                        }
+                        __nv_bfloat16* cp = C + crow * N + nb;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            if (nb + v * 8 >= N) break;
+                            float o[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float cval = a[v * 8 + i] + sbias[c * 32 + v * 8 + i];
+                                o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
+                            }
+                            uint4 u;
+                            u.x = pack_bf16x2(o[0], o[1]);
+                            u.y = pack_bf16x2(o[2], o[3]);
+                            u.z = pack_bf16x2(o[4], o[5]);
+                            u.w = pack_bf16x2(o[6], o[7]);
+                            *reinterpret_cast<uint4*>(cp + v * 8) = u;
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0 && got) mbar_arrive(&tempty_bar[acc]);
+                if (sg.kind == kSegFinish) {
+                    // every partial is consumed: clear the contributors' flags so a
+                    // replay of this launch (same epoch, e.g. from a CUDA graph)
+                    // waits for fresh partials
+                    named_bar_sync(1, 32 * kTcEpiWarps);
+                    if (etid == 0 && partial_ok)
+                        for (int cc = int(blockIdx.x) + 1; cc <= c_last; ++cc) skp.flags[cc] = 0ull;
+                }
+            }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }

@@ -163,6 +163,13 @@ int check_reroute(int k, int E, int F) {
     return MOE_OK;
 }
 
+// bf16 tensor-core GEMM tile: 128 x 256 (the widest single-CTA MMA; narrower
+// tiles measured slower on every workload: more A re-reads per FLOP)
+constexpr int kTcBN = 256, kTcStages = 4;
+// stream-K scratch of the bf16 grouped FFN: one fp32 partial tile and one
+// flag per CTA, for grids of up to kSkMaxCtas CTAs
+constexpr int kSkMaxCtas = 160;
+
 // Scratch of a rerouting dispatch (F rounds, nchunk chunks).
 struct RerouteWs {
     int32_t* srv;     // [T*k]
@@ -207,6 +214,7 @@ struct WsLayout {
     size_t idx, gate, counts, offsets, perm, slot_of, row_gate, xp, h, yp;
     size_t fhist, fbase, fpsum;   // per-router-chunk arrays of the forward path
     size_t fb_idx, fb_gate, reroute;   // overflow rerouting (F > 0)
+    size_t sk_partials, sk_flags;      // stream-K scratch of the bf16 grouped FFN
     size_t total;
 };
 
@@ -247,6 +255,9 @@ WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype, int S = 0, int
     L.fb_idx = take(size_t(T) * F * 4);
     L.fb_gate = take(size_t(T) * F * 4);
     L.reroute = take(F > 0 ? reroute_ws_bytes(T, k, E, F, int(nchunk)) : 0);
+    const bool sk = dtype == MOE_BF16;
+    L.sk_partials = take(sk ? size_t(kSkMaxCtas) * kTcBM * kTcBN * sizeof(float) : 0);
+    L.sk_flags = take(sk ? size_t(kSkMaxCtas) * sizeof(unsigned long long) : 0);
     L.total = o;
     return L;
 }
@@ -297,10 +308,23 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Raises a kernel's dynamic shared memory limit once per device (later
+// calls, e.g. while a CUDA graph is being captured, only look it up).
+std::mutex g_attr_mu;
+std::vector<std::pair<const void*, int>> g_attr_done;   // (kernel, device) already set
+
 template <typename K>
 bool set_smem_attr(K kernel, size_t bytes) {
-    // cudaFuncSetAttribute is cheap and idempotent; it is per device, so set it every call
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) == cudaSuccess;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const void* key = reinterpret_cast<const void*>(kernel);
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    for (const auto& kd : g_attr_done)
+        if (kd.first == key && kd.second == dev) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) != cudaSuccess)
+        return false;
+    g_attr_done.emplace_back(key, dev);
+    return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -425,9 +449,6 @@ int run_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int
     return MOE_OK;
 }
 
-// bf16 tensor-core GEMM tile: 128 x 256 (the widest single-CTA MMA; narrower
-// tiles measured slower on every workload: more A re-reads per FLOP)
-constexpr int kTcBN = 256, kTcStages = 4;
 
 // The shared always-on experts of one FFN GEMM (host side): S groups of
 // `g.rows` rows each, A rows from `a` (a_rows rows in all), weights [S, N, K]
@@ -442,10 +463,13 @@ struct SharedArgs {
 
 // Routed groups: E experts over rows offsets[0..E] of `a` (a_rows rows;
 // routed_rows_ub bounds offsets[E]).  E may be 0 when only shared groups run.
+// every stream-K launch takes a fresh epoch (never 0, the cleared flag)
+std::atomic<unsigned long long> g_sk_epoch{0x9E3779B97F4A7C15ull};
+
 template <int BN, int STAGES, int MODE>
 int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
               const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
-              const SharedArgs& sa, int kernel_id, cudaStream_t s) {
+              const SharedArgs& sa, StreamK skp, int kernel_id, cudaStream_t s) {
     CUtensorMap tmA, tmB, tmA2, tmB2;
     if (sa.g.S > 0) {
         if (!make_map_2d(&tmA2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
@@ -469,13 +493,21 @@ int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const v
     const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kTcBM)) + E +
                             static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kTcBM);
     const long long tiles_ub = mt_ub * ceil_div(N, BN);
-    const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
+    int grid;
+    if (skp.partials != nullptr) {
+        // stream-K: one CTA per SM, each with an equal share of the k-block units
+        const long long units_ub = tiles_ub * ceil_div(a_cols, kTcBK);
+        grid = int(std::max(1ll, std::min<long long>(units_ub, std::min(num_sms(), kSkMaxCtas))));
+        skp.epoch = g_sk_epoch.fetch_add(1, std::memory_order_relaxed);
+    } else {
+        grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
+    }
     Launch L(kernel_id, s);
     cudaError_t launch_err;
     launch_err = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, s, tmA, tmB, offsets, E, N, a_cols,
                             static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
                             static_cast<__nv_bfloat16*>(c), sa.g, tmA2, tmB2,
-                            static_cast<const __nv_bfloat16*>(sa.bias));
+                            static_cast<const __nv_bfloat16*>(sa.bias), skp);
     return L.finish(launch_err);
 }
 
@@ -511,9 +543,10 @@ struct SharedExperts {
 // max_rows routed rows followed by S * T shared rows (shared expert s, token
 // t at row max_rows + s * T + t).  out_rows (nullable): fc2 writes routed
 // row r to row out_rows[r] of yp (the direct output of a k == 1 layer).
+// skp: stream-K scratch for the bf16 launches (partials null: whole tiles)
 int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
             const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp, int dtype,
-            const int32_t* out_rows, const SharedExperts& se, cudaStream_t s) {
+            const int32_t* out_rows, const SharedExperts& se, const StreamK& skp, cudaStream_t s) {
     const int h_rows = max_rows + se.S * se.T;
     SharedArgs s1, s2;
     if (se.S > 0) {
@@ -533,10 +566,10 @@ int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, 
     int rc;
     if (dtype == MOE_BF16) {
         rc = launch_tc<kTcBN, kTcStages, kFc1Gelu>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr,
-                                                   nullptr, h, s1, MOE_KERNEL_FFN1, s);
+                                                   nullptr, h, s1, skp, MOE_KERNEL_FFN1, s);
         if (rc != MOE_OK) return rc;
         return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate,
-                                                     out_rows, yp, s2, MOE_KERNEL_FFN2, s);
+                                                     out_rows, yp, s2, skp, MOE_KERNEL_FFN2, s);
     }
     rc = launch_simt<kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, s1, MOE_KERNEL_FFN1,
                                s);
@@ -550,12 +583,26 @@ int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, 
 // gather kernel over (chunk, G) CTAs.
 int permute_split(int nchunk) { return std::max(1, std::min(8, ceil_div(2 * num_sms(), nchunk))); }
 
+// the fused scan + permute kernel reads the whole per-chunk histogram table
+// in every CTA: used while that table is small
+constexpr long long kFusedScanMaxEntries = 16384;
+
 int run_forward_dispatch(const int32_t* idx, const float* gate, int T, int k, int E, int capacity, int chunk_tokens,
                          const int32_t* fhist, const float* fpsum, int32_t* fbase, int32_t* counts, int32_t* offsets,
                          int32_t* perm, int32_t* slot_of, uint8_t* drop_mask, float* row_gate, moe_stats* st,
                          const void* x, void* xp, int d, int dtype, void* out_zero_dropped, cudaStream_t s) {
     const int nchunk = ceil_div(T, chunk_tokens);
     int rc;
+    if (drop_mask == nullptr && static_cast<long long>(nchunk) * E <= kFusedScanMaxEntries) {
+        const int row_bytes = int(size_t(d) * elem_bytes(dtype));
+        Launch L(MOE_KERNEL_PERMUTE, s);
+        cudaError_t launch_err;
+        launch_err = launch_pdl(forward_dispatch_kernel, dim3(nchunk, permute_split(nchunk)), dim3(kFwdThreads), 0,
+                                s, idx, gate, T, k, E, chunk_tokens, fhist, fpsum, nchunk, capacity, counts, offsets,
+                                st, perm, slot_of, row_gate, static_cast<const uint8_t*>(x), row_bytes,
+                                static_cast<uint8_t*>(xp), static_cast<uint8_t*>(out_zero_dropped));
+        return L.finish(launch_err);
+    }
     {
         Launch L(MOE_KERNEL_SCAN, s);
         cudaError_t launch_err;
@@ -916,7 +963,7 @@ int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E,
         !aligned16(yp))
         return MOE_ERR_INVALID_ARG;
     return run_ffn(xp, offsets, max_rows, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype, nullptr,
-                   SharedExperts{}, static_cast<cudaStream_t>(stream));
+                   SharedExperts{}, StreamK{}, static_cast<cudaStream_t>(stream));
 }
 
 int moe_shared_ffn(const void* x, int T, int d, int ff, int S, const void* w1s, const void* b1s, const void* w2s,
@@ -938,7 +985,7 @@ int moe_shared_ffn(const void* x, int T, int d, int ff, int S, const void* w1s, 
     se.w2 = w2s;
     se.b2 = b2s;
     return run_ffn(nullptr, nullptr, 0, 0, d, ff, nullptr, nullptr, nullptr, nullptr, nullptr, h, ys, dtype,
-                   nullptr, se, static_cast<cudaStream_t>(stream));
+                   nullptr, se, StreamK{}, static_cast<cudaStream_t>(stream));
 }
 
 int moe_combine(const void* yp, const int32_t* slot_of, const float* topk_gate, int T, int k, int d, int dtype,
@@ -1045,8 +1092,13 @@ int moe_forward_ex(const void* x, const void* w_router, const float* logit_bias,
                                   perm, slot_of, nullptr, row_gate, stats, x, xp, d, dtype, direct ? out : nullptr,
                                   s);
     if (rc != MOE_OK) return rc;
+    StreamK skp{};
+    if (dtype == MOE_BF16) {
+        skp.partials = reinterpret_cast<float*>(w + L.sk_partials);
+        skp.flags = reinterpret_cast<unsigned long long*>(w + L.sk_flags);
+    }
     if ((rc = run_ffn(xp, offsets, A, E, d, ff, w1, b1, w2, b2, row_gate, h, direct ? out : yp, dtype,
-                      direct ? perm : nullptr, se, s)) != MOE_OK)
+                      direct ? perm : nullptr, se, skp, s)) != MOE_OK)
         return rc;
     if (!direct) {
         const void* ys = static_cast<const uint8_t*>(yp) + size_t(A) * d * elem_bytes(dtype);

@@ -159,13 +159,19 @@ class HostPipeline:
     """End-to-end forward passes from pinned host memory, pipelined.
 
     Each step copies its tokens host -> device, runs the layer and copies
-    the output device -> host.  The three run on their own streams with
-    `depth` device buffers, so the input copy of step i+1 and the output
-    copy of step i-1 overlap the layer of step i (PCIe is full duplex).
-    Every step's copies are still issued and completed.
+    the output device -> host.  The copies run on their own streams and the
+    layer on a third, with `depth` lanes (device input / output buffers and
+    a workspace each), so the input copy of step i+1 and the output copy of
+    step i-1 overlap the layer of step i (PCIe is full duplex).  Every
+    step's copies are still issued and completed.
+
+    With `graphs` (default) each lane's layer call is captured once into a
+    CUDA graph and replayed, so a step costs the host a few calls instead of
+    the layer's launch sequence; the layer calls of all lanes stay on one
+    stream, one after another.
     """
 
-    def __init__(self, layer: MoELayer, T: int, depth: int = 2):
+    def __init__(self, layer: MoELayer, T: int, depth: int = 3, graphs: bool = True):
         dev = layer.p.w1.device
         dt = TORCH_DTYPE[layer.p.dtype]
         self.layer = layer
@@ -175,9 +181,25 @@ class HostPipeline:
         self.s_out = torch.cuda.Stream(device=dev)
         self.x_dev = [torch.empty((T, layer.p.d), dtype=dt, device=dev) for _ in range(depth)]
         self.out_dev = [torch.empty((T, layer.p.d), dtype=dt, device=dev) for _ in range(depth)]
+        # one layer (own workspace) per lane, sharing the parameters
+        self.lanes = [MoELayer(layer.p, layer.k, layer.capacity, layer.reroute) for _ in range(depth)]
+        for ln in self.lanes:
+            ln.workspace(T)
         self.in_done = [torch.cuda.Event() for _ in range(depth)]
         self.run_done = [torch.cuda.Event() for _ in range(depth)]
         self.out_done = [torch.cuda.Event() for _ in range(depth)]
+        self.graphs = None
+        if graphs:
+            self.graphs = []
+            torch.cuda.synchronize(dev)
+            for b in range(depth):
+                self.lanes[b].forward(self.x_dev[b], out=self.out_dev[b])      # warm the launch path
+                torch.cuda.synchronize(dev)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    self.lanes[b].forward(self.x_dev[b], out=self.out_dev[b])
+                self.graphs.append(g)
+            torch.cuda.synchronize(dev)
 
     def run(self, x_hosts, out_hosts, start_event=None, end_event=None):
         """x_hosts[i] (pinned) -> layer -> out_hosts[i] (pinned), for every i."""
@@ -193,7 +215,11 @@ class HostPipeline:
             self.in_done[b].record(self.s_in)
             self.s_run.wait_event(self.in_done[b])
             self.s_run.wait_event(self.out_done[b])         # out_dev[b] already copied out
-            self.layer.forward(self.x_dev[b], out=self.out_dev[b], stream=self.s_run)
+            if self.graphs is not None:
+                with torch.cuda.stream(self.s_run):
+                    self.graphs[b].replay()
+            else:
+                self.lanes[b].forward(self.x_dev[b], out=self.out_dev[b], stream=self.s_run)
             self.run_done[b].record(self.s_run)
             self.s_out.wait_event(self.run_done[b])
             with torch.cuda.stream(self.s_out):
@@ -206,4 +232,3 @@ class HostPipeline:
         self.s_out.synchronize()
         self.s_in.synchronize()
         self.s_run.synchronize()
-

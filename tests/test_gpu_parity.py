@@ -405,7 +405,7 @@ def test_launch_counter_and_timing():
     launched = _lib.moe_launch_count() - n0
     t = _lib.moe_timing_read()
     _lib.moe_timing_enable(False)
-    # router, scan, permute+gather, ffn1, ffn2, combine (k = 2)
-    assert launched == 6
-    assert sum(n for _, n in t.values()) == 6
+    # router, dispatch (scan + permute + gather), ffn1, ffn2, combine (k = 2)
+    assert launched == 5
+    assert sum(n for _, n in t.values()) == 5
     assert all(ms > 0 for ms, n in t.values() if n)

@@ -175,5 +175,5 @@ def test_shared_launch_count():
     n0 = _lib.moe_launch_count()
     layer.forward(x)
     torch.cuda.synchronize()
-    # router, scan, permute+gather, ffn1 (routed + shared), ffn2 (routed + shared), combine
-    assert _lib.moe_launch_count() - n0 == 6
+    # router, dispatch (scan + permute + gather), ffn1 (routed + shared), ffn2 (routed + shared), combine
+    assert _lib.moe_launch_count() - n0 == 5
