@@ -356,6 +356,13 @@ MOE_API int moe_get_error(void* stream);
  * <= 1.5e-7), the bf16 tensor-core epilogue's form. */
 MOE_API int moe_debug_gelu(const float* x, float* y, int n, int variant, void* stream);
 
+/* Failure-path check: launches one kernel whose bounded wait on a barrier
+ * that nothing completes gives up after limit_ns (0 < limit_ns <= 2 s, the
+ * limit of the layer's own pipeline waits) and records MOE_ERR_TIMEOUT in
+ * the device error word, exactly as a stalled pipeline wait would; the
+ * context stays usable.  Read the status with moe_get_error. */
+MOE_API int moe_debug_wait_timeout(int64_t limit_ns, void* stream);
+
 /* Number of kernels this library has launched in this process. */
 MOE_API uint64_t moe_launch_count(void);
 

@@ -74,6 +74,7 @@ _SIGS = {
     "moe_combine_shared": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "moe_get_error": (_I, [_P]),
     "moe_debug_gelu": (_I, [_P, _P, _I, _I, _P]),
+    "moe_debug_wait_timeout": (_I, [ctypes.c_int64, _P]),
     "moe_launch_count": (ctypes.c_uint64, []),
     "moe_timing_enable": (_I, [_I]),
     "moe_timing_read": (_I, [_P, _P]),
@@ -270,3 +271,8 @@ def moe_timing_read():
     n = (ctypes.c_int64 * MOE_NUM_KERNELS)()
     _check(load().moe_timing_read(ctypes.cast(ms, _P), ctypes.cast(n, _P)), "moe_timing_read")
     return {name: (ms[i], int(n[i])) for i, name in enumerate(KERNEL_NAMES)}
+
+
+def moe_debug_wait_timeout(limit_ns: int, stream=None):
+    """One bounded wait that runs out; the device error word then holds MOE_ERR_TIMEOUT."""
+    _check(load().moe_debug_wait_timeout(int(limit_ns), _stream(stream)), "moe_debug_wait_timeout")

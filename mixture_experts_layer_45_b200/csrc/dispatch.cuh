@@ -970,6 +970,22 @@ combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, co
     }
 }
 
+// Exercises the bounded-wait path: waits on an mbarrier that nothing ever
+// completes, gives up after limit_ns and records MOE_ERR_TIMEOUT, like a
+// pipeline wait of the layer's kernels that runs out.
+__global__ void wait_timeout_probe_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns);
+    __syncthreads();
+}
+
 // y[i] = GELU(x[i]) with the form the fp32 path uses (variant 0, erff) or the
 // bf16 tensor-core epilogue uses (variant 1, A&S 7.1.26); for testing.
 __global__ void gelu_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int variant) {

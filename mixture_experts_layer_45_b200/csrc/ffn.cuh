@@ -270,83 +270,6 @@ struct TcCfg {
     static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;   // + alignment slack
 };
 
-// Work split of one launch (G = gridDim.x CTAs).  Without partials
-// (classic): CTA b takes whole tiles b, b + G, b + 2G, ...  With partials
-// (stream-K hybrid): all but the last one to two waves of tiles go whole,
-// round-robin as in the classic split (CTAs running together share weight
-// panels and A rows through L2); the remaining tiles' k-block units are cut
-// into G contiguous ranges [b*U/G, (b+1)*U/G), so the tail of the launch is
-// spread over every SM instead of leaving most of them idle.  A range
-// splits at most its first and last tile.  The CTA that covers a split
-// tile's first k-block finishes it: the CTAs after it, which cover the rest
-// of that tile at the start of their ranges, write fp32 partial tiles to
-// partials[c] and publish flags[c] = epoch; the finisher waits for them
-// (bounded), adds them in CTA order and runs the epilogue.  A CTA ends its
-// range with the tile it finishes, so it waits for work the next CTAs did
-// first.
-struct StreamK {
-    float* partials;               // [gridDim.x][kTcBM][BN] fp32, or null: classic split
-    unsigned long long* flags;     // [gridDim.x]; a finisher clears the flags it consumed
-    unsigned long long epoch;      // unique per host launch call (never 0)
-};
-
-enum SegKind { kSegFull = 0, kSegFinish = 1, kSegPartial = 2 };
-
-struct Seg {
-    int pos;    // tile position of the walk (decode_tile maps it to a tile)
-    int kb0, kb1;
-    int kind;
-};
-
-// The segments of this CTA's work, in order; every warp role walks the same
-// sequence.
-struct SegWalk {
-    int total, KB, G;
-    int dp;            // tiles handed out whole, round-robin
-    long long U;       // k-block units of the split tail
-    int t;             // next whole tile
-    long long u, u1;   // split tail: unit cursor and end
-    __device__ __forceinline__ SegWalk(int total_, int KB_, bool sk) : total(total_), KB(KB_), G(int(gridDim.x)) {
-        dp = total;
-        if (sk) {
-            const int waves = total / G;
-            dp = waves >= 2 ? (waves - 1) * G : 0;
-        }
-        U = (long long)(total - dp) * KB;
-        t = int(blockIdx.x);
-        u = range_begin(int(blockIdx.x));
-        u1 = range_begin(int(blockIdx.x) + 1);
-    }
-    __device__ __forceinline__ long long range_begin(int c) const { return U * c / G; }
-    __device__ __forceinline__ bool next(Seg& sg) {
-        if (t < dp) {
-            sg.pos = t;
-            sg.kb0 = 0;
-            sg.kb1 = KB;
-            sg.kind = kSegFull;
-            t += G;
-            return true;
-        }
-        if (u >= u1) return false;
-        const int local = int(u / KB);
-        sg.pos = dp + local;
-        sg.kb0 = int(u - (long long)local * KB);
-        const long long rem = u1 - u;
-        sg.kb1 = (rem < (long long)(KB - sg.kb0)) ? sg.kb0 + int(rem) : KB;
-        sg.kind = (sg.kb0 > 0) ? kSegPartial : (sg.kb1 < KB ? kSegFinish : kSegFull);
-        u += sg.kb1 - sg.kb0;
-        return true;
-    }
-    // last CTA holding part of split tile `pos` (whose first k-block this CTA holds)
-    __device__ __forceinline__ int last_contributor(int pos) const {
-        const long long tile_end = (long long)(pos - dp + 1) * KB;
-        int c = int(blockIdx.x);
-        while (c + 1 < G && range_begin(c + 1) < tile_end) ++c;
-        return c;
-    }
-    __device__ __forceinline__ bool range_empty(int c) const { return range_begin(c) >= range_begin(c + 1); }
-};
-
 // tmA2 / tmB2 / bias2: the shared experts' A rows and parameters (used when sh.S > 0)
 template <int BN, int STAGES, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -355,7 +278,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                    const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
                    const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C, SharedGroups sh,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                   const __nv_bfloat16* __restrict__ bias2, StreamK skp) {
+                   const __nv_bfloat16* __restrict__ bias2) {
     using Cfg = TcCfg<BN, STAGES>;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN: whole 32-column epilogue chunks, MMA N <= 256");
     __shared__ TileTable tt;
@@ -363,7 +286,6 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
-    __shared__ int partial_ok;
     __shared__ float sbias[BN];
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
@@ -400,7 +322,6 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     const int G = E + sh.S;
     const int total = tt.start[G];
     const int KB = (K + kTcBK - 1) / kTcBK;
-    const bool sk = skp.partials != nullptr;
     volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
@@ -411,17 +332,15 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             int last_parity[STAGES];
             for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
             bool ok = true;
-            SegWalk walk(total, KB, sk);
-            Seg sg;
-            while (ok && walk.next(sg)) {
-                const TileCoord tc = decode_tile(tt, G, sg.pos);
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const TileCoord tc = decode_tile(tt, G, t);
                 const bool shared_g = tc.e >= E;
                 const CUtensorMap* ma = shared_g ? &tmA2 : &tmA;
                 const CUtensorMap* mb = shared_g ? &tmB2 : &tmB;
                 const int widx = shared_g ? tc.e - E : tc.e;
                 const int row0 = tt.arow[tc.e] + tc.mt * kTcBM;
                 const int n0 = tc.nt * BN;
-                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) { ok = false; break; }
                     uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
                     uint8_t* sb = sa + Cfg::kABytes;
@@ -451,13 +370,11 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            SegWalk walk(total, KB, sk);
-            Seg sg;
-            while (ok && walk.next(sg)) {
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_p)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
-                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, abort_p)) { ok = false; break; }
                     tc_fence_after();
                     const uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
@@ -466,7 +383,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
 #pragma unroll
                     for (int kk = 0; kk < kTcBK / 16; ++kk)
                         umma_f16(d_tmem, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc,
-                                 (kb > sg.kb0 || kk > 0) ? 1u : 0u);
+                                 (kb > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty_bar[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -486,20 +403,17 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         const int etid = threadIdx.x - 64;   // 0..255
         const int q = warp & 3;              // TMEM lane quarter this warp may access
         const int half = (warp - 2) >> 2;    // which alternate 32-column chunks
-        const int row_in_tile = q * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool failed = false;
-        SegWalk walk(total, KB, sk);
-        Seg sg;
-        while (walk.next(sg)) {
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
             // all epilogue warps stop together once any wait has given up, so
             // none is left behind at a named barrier
             if (named_bar_red_or(1, 32 * kTcEpiWarps, failed || *abort_p)) break;
-            const TileCoord tc = decode_tile(tt, G, sg.pos);
+            const TileCoord tc = decode_tile(tt, G, t);
             const bool shared_g = tc.e >= E;
             const int rows = tt.rows[tc.e];
-            const int r_in = tc.mt * kTcBM + row_in_tile;
+            const int r_in = tc.mt * kTcBM + q * 32 + lane;
             const bool valid = r_in < rows;
             const size_t grow = size_t(tt.crow[tc.e]) + r_in;
             // destination row: the grouped row, or (direct output of a routed
@@ -512,118 +426,42 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             // (the barrier above also ends every read of the previous tile's bias)
             for (int i = etid; i < BN; i += 32 * kTcEpiWarps)
                 sbias[i] = (n0 + i < N) ? __bfloat162float(bb[n0 + i]) : 0.f;
-            // the CTAs after this one that hold the rest of a tile it finishes
-            int c_last = int(blockIdx.x);
-            if (sg.kind == kSegFinish) {
-                c_last = walk.last_contributor(sg.pos);
-                if (etid == 0) {
-                    int ok_all = 1;
-                    for (int c = int(blockIdx.x) + 1; c <= c_last; ++c) {
-                        if (walk.range_empty(c)) continue;
-                        const uint64_t t0 = globaltimer_ns();
-                        while (ld_acquire_u64(skp.flags + c) != skp.epoch) {
-                            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                                set_error(MOE_ERR_TIMEOUT);
-                                ok_all = 0;
-                                break;
-                            }
-                        }
-                        if (!ok_all) break;
-                    }
-                    partial_ok = ok_all;
-                }
-            }
-            named_bar_sync(1, 32 * kTcEpiWarps);   // bias and partial flags visible
-            if (sg.kind == kSegFinish && !partial_ok) failed = true;
-            // every epilogue warp takes the same barriers below whether or not
-            // its wait succeeded; a failed warp only skips the work
+            named_bar_sync(1, 32 * kTcEpiWarps);   // this tile's bias is visible
             // (uniform per warp: the TMEM loads below are warp-collective)
-            const bool got = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_p));
-            if (!got) failed = true;
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_p))) {
+                failed = true;
+                continue;
+            }
             tc_fence_after();
-            if (sg.kind == kSegPartial) {
-                // raw fp32 accumulators of this CTA's share of the tile
-                float* dst = skp.partials + (size_t(blockIdx.x) * kTcBM + row_in_tile) * BN;
-                if (got) {
 #pragma unroll 1
-                    for (int c = half; c < BN / 32; c += 2) {
-                        uint32_t r[32];
-                        __syncwarp();
-                        tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            *reinterpret_cast<uint4*>(dst + c * 32 + v * 4) =
-                                make_uint4(r[v * 4], r[v * 4 + 1], r[v * 4 + 2], r[v * 4 + 3]);
-                    }
-                    __threadfence();
-                }
-                tc_fence_before();
+            for (int c = half; c < BN / 32; c += 2) {
+                uint32_t r[32];
                 __syncwarp();
-                if (lane == 0 && got) mbar_arrive(&tempty_bar[acc]);
-                // every thread's partial is written and fenced; publish it
-                // only if no warp gave up
-                const bool any_failed = named_bar_red_or(1, 32 * kTcEpiWarps, !got);
-                if (etid == 0 && !any_failed) st_release_u64(skp.flags + blockIdx.x, skp.epoch);
-            } else {
-                if (got) {
-#pragma unroll 1
-                    for (int c = half; c < BN / 32; c += 2) {
-                        uint32_t r[32];
-                        __syncwarp();
-                        tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
-                        tmem_ld_wait();
-                        const int nb = n0 + c * 32;
-                        if (!valid || nb >= N) continue;
-                        float a[32];
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
+                tmem_ld_wait();
+                const int nb = n0 + c * 32;
+                if (!valid || nb >= N) continue;
+                __nv_bfloat16* cp = C + crow * N + nb;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
-                        if (sg.kind == kSegFinish) {
-                            for (int cc = int(blockIdx.x) + 1; cc <= c_last; ++cc) {
-                                if (walk.range_empty(cc)) continue;
-                                const float* src =
-                                    skp.partials + (size_t(cc) * kTcBM + row_in_tile) * BN + c * 32;
+                for (int v = 0; v < 4; ++v) {
+                    if (nb + v * 8 >= N) break;
+                    float o[8];
 #pragma unroll
-                                for (int v = 0; v < 8; ++v) {
-                                    const float4 pv = __ldcg(reinterpret_cast<const float4*>(src) + v);
-                                    a[v * 4] += pv.x;
-                                    a[v * 4 + 1] += pv.y;
-                                    a[v * 4 + 2] += pv.z;
-                                    a[v * 4 + 3] += pv.w;
-                                }
-                            }
-                        }
-                        __nv_bfloat16* cp = C + crow * N + nb;
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            if (nb + v * 8 >= N) break;
-                            float o[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const float cval = a[v * 8 + i] + sbias[c * 32 + v * 8 + i];
-                                o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
-                            }
-                            uint4 u;
-                            u.x = pack_bf16x2(o[0], o[1]);
-                            u.y = pack_bf16x2(o[2], o[3]);
-                            u.z = pack_bf16x2(o[4], o[5]);
-                            u.w = pack_bf16x2(o[6], o[7]);
-                            *reinterpret_cast<uint4*>(cp + v * 8) = u;
-                        }
+                    for (int i = 0; i < 8; ++i) {
+                        const float cval = __uint_as_float(r[v * 8 + i]) + sbias[c * 32 + v * 8 + i];
+                        o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
                     }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0 && got) mbar_arrive(&tempty_bar[acc]);
-                if (sg.kind == kSegFinish) {
-                    // every partial is consumed: clear the contributors' flags so a
-                    // replay of this launch (same epoch, e.g. from a CUDA graph)
-                    // waits for fresh partials
-                    named_bar_sync(1, 32 * kTcEpiWarps);
-                    if (etid == 0 && partial_ok)
-                        for (int cc = int(blockIdx.x) + 1; cc <= c_last; ++cc) skp.flags[cc] = 0ull;
+                    uint4 u;
+                    u.x = pack_bf16x2(o[0], o[1]);
+                    u.y = pack_bf16x2(o[2], o[3]);
+                    u.z = pack_bf16x2(o[4], o[5]);
+                    u.w = pack_bf16x2(o[6], o[7]);
+                    *reinterpret_cast<uint4*>(cp + v * 8) = u;
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
@@ -633,6 +471,231 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    }
+}
+
+// ===========================================================================
+// bf16 path on CTA pairs: tcgen05.mma.cta_group::2, 256 x 256 tiles.
+//
+// A cluster of two CTAs computes one 256-row x 256-column tile per step:
+// CTA r loads A rows [m0 + 128r, +128) and weight rows [n0 + 128r, +128)
+// (its halves of A and of the tile's N) into its own shared memory, both
+// loads counting on CTA 0's `full` barrier; CTA 0's MMA thread issues the
+// pair MMA and commits to both CTAs' `empty` / `tfull` barriers; each CTA's
+// epilogue reads its 128 accumulator rows (all 256 columns) from its own
+// tensor memory and signals CTA 0's `tempty` barrier.  Per CTA a k-block
+// moves 32 KB for 128 x 256 x 64 MACs (the single-CTA tile moves 48 KB), so
+// six stages fit in shared memory and the loads keep the tensor pipe fed
+// at large K.  Same warp roles, tile table (M tiles of 256 rows), bounded
+// waits and epilogue as ffn_tc_bf16_kernel.
+// ===========================================================================
+constexpr int kTc2BM = 256;          // rows per pair tile (128 per CTA)
+constexpr int kTc2BN = 256;          // columns per pair tile (128 weight rows per CTA)
+
+template <int STAGES>
+struct Tc2Cfg {
+    static constexpr uint32_t kABytes = 128 * kTcBK * 2;
+    static constexpr uint32_t kBBytes = (kTc2BN / 2) * kTcBK * 2;
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+    static constexpr uint32_t kTmemCols = 2 * kTc2BN;   // two accumulators
+    static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
+};
+
+template <int STAGES, int MODE>
+__global__ void __launch_bounds__(kTcThreads, 1)
+ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const int32_t* __restrict__ offsets, int E, int N, int K,
+                    const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
+                    const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C, SharedGroups sh,
+                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                    const __nv_bfloat16* __restrict__ bias2) {
+    using Cfg = Tc2Cfg<STAGES>;
+    constexpr int BN = kTc2BN;
+    __shared__ TileTable tt;
+    __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+    __shared__ float sbias[BN];
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();   // 0: issues the pair MMAs
+    const int pair = int(blockIdx.x >> 1), npairs = int(gridDim.x >> 1);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);    // CTA 0's copy counts both CTAs' loads
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull_bar[a], 1);
+            mbar_init(&tempty_bar[a], 2 * kTcEpiWarps);   // CTA 0's copy: every epilogue warp of the pair
+        }
+        mbar_init(&drain_bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (sh.S > 0) {
+            tma_prefetch_desc(&tmA2);
+            tma_prefetch_desc(&tmB2);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish_pair();
+        tc_fence_before();
+    }
+    const int ntn = (N + BN - 1) / BN;
+    build_tile_table(offsets, E, sh, kTc2BM, ntn, tt);   // contains __syncthreads()
+    cluster_sync();   // both CTAs' barriers are initialised before any cross-CTA arrive
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+    const int G = E + sh.S;
+    const int total = tt.start[G];
+    const int KB = (K + kTcBK - 1) / kTcBK;
+    volatile int* abort_p = &abort_flag;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs) ----------------
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = pair; t < total && ok; t += npairs) {
+                const TileCoord tc = decode_tile(tt, G, t);
+                const bool shared_g = tc.e >= E;
+                const CUtensorMap* ma = shared_g ? &tmA2 : &tmA;
+                const CUtensorMap* mb = shared_g ? &tmB2 : &tmB;
+                const int widx = shared_g ? tc.e - E : tc.e;
+                const int row0 = tt.arow[tc.e] + tc.mt * kTc2BM + 128 * int(rank);
+                const int n0 = tc.nt * BN + (BN / 2) * int(rank);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) { ok = false; break; }
+                    uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
+                    uint8_t* sb = sa + Cfg::kABytes;
+                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * Cfg::kStageBytes);
+                    tma_load_2d_pair(sa, ma, &full_bar[stage], kb * kTcBK, row0);
+                    tma_load_3d_pair(sb, mb, &full_bar[stage], kb * kTcBK, n0, widx);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------- pair MMA issuer (CTA 0) ----------------
+            constexpr uint32_t idesc = idesc_bf16_f32(kTc2BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = pair; t < total && ok; t += npairs) {
+                if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_p)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, abort_p)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
+                    const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sa));
+                    const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sa + Cfg::kABytes));
+#pragma unroll
+                    for (int kk = 0; kk < kTcBK / 16; ++kk)
+                        umma_f16_pair(d_tmem, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc,
+                                      (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit_pair(&empty_bar[stage], 0x3);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit_pair(&tfull_bar[acc], 0x3);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            // every pair MMA completes (in both CTAs' view) before teardown
+            umma_commit_pair(&drain_bar, 0x3);
+        }
+    } else {
+        // ---------------- epilogue (warps 2..9 of each CTA) ----------------
+        const int etid = threadIdx.x - 64;   // 0..255
+        const int q = warp & 3;              // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;    // which alternate 32-column chunks
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool failed = false;
+        for (int t = pair; t < total; t += npairs) {
+            if (named_bar_red_or(1, 32 * kTcEpiWarps, failed || *abort_p)) break;
+            const TileCoord tc = decode_tile(tt, G, t);
+            const bool shared_g = tc.e >= E;
+            const int rows = tt.rows[tc.e];
+            const int r_in = tc.mt * kTc2BM + 128 * int(rank) + q * 32 + lane;
+            const bool valid = r_in < rows;
+            const size_t grow = size_t(tt.crow[tc.e]) + r_in;
+            const size_t crow = (out_rows != nullptr && valid && !shared_g) ? size_t(out_rows[grow]) : grow;
+            const int n0 = tc.nt * BN;
+            float g = 1.f;
+            if (MODE == kFc2Gate && row_gate != nullptr && valid && !shared_g) g = row_gate[grow];
+            const __nv_bfloat16* bb = shared_g ? bias2 + size_t(tc.e - E) * N : bias + size_t(tc.e) * N;
+            for (int i = etid; i < BN; i += 32 * kTcEpiWarps)
+                sbias[i] = (n0 + i < N) ? __bfloat162float(bb[n0 + i]) : 0.f;
+            named_bar_sync(1, 32 * kTcEpiWarps);
+            // (uniform per warp: the TMEM loads below are warp-collective)
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_p))) {
+                failed = true;
+                continue;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = half; c < BN / 32; c += 2) {
+                uint32_t r[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
+                tmem_ld_wait();
+                const int nb = n0 + c * 32;
+                if (!valid || nb >= N) continue;
+                __nv_bfloat16* cp = C + crow * N + nb;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    if (nb + v * 8 >= N) break;
+                    float o[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float cval = __uint_as_float(r[v * 8 + i]) + sbias[c * 32 + v * 8 + i];
+                        o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
+                    }
+                    uint4 u;
+                    u.x = pack_bf16x2(o[0], o[1]);
+                    u.y = pack_bf16x2(o[2], o[3]);
+                    u.z = pack_bf16x2(o[4], o[5]);
+                    u.w = pack_bf16x2(o[6], o[7]);
+                    *reinterpret_cast<uint4*>(cp + v * 8) = u;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(&tempty_bar[acc]);
+                else mbar_arrive_remote(&tempty_bar[acc], 0);
+            }
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    // teardown: every pair MMA has completed (it reads both CTAs' shared
+    // memory and writes both tensor memories) before either CTA frees
+    // anything or exits
+    if (warp == 1 && lane == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+    }
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
     }
 }
 

@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -122,6 +123,27 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// The same with thread-block clusters of `cluster_x` CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, int cluster_x,
+                               cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = unsigned(cluster_x);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // helpers
 // ---------------------------------------------------------------------------
@@ -129,6 +151,17 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline size_t elem_bytes(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
 inline int ceil_div(long long a, long long b) { return int((a + b - 1) / b); }
+
+// CTA-pair FFN tiles: the heuristic's choice unless the environment
+// variable MOE_PAIR_TILES is "0" (never) or "1" (always)
+bool pair_tiles_enabled(bool heuristic) {
+    static const int forced = []() {
+        const char* v = std::getenv("MOE_PAIR_TILES");
+        if (v == nullptr || *v == 0) return -1;
+        return v[0] == '0' ? 0 : 1;
+    }();
+    return forced < 0 ? heuristic : forced == 1;
+}
 
 int num_sms() {
     int dev = 0, n = 0;
@@ -166,10 +199,6 @@ int check_reroute(int k, int E, int F) {
 // bf16 tensor-core GEMM tile: 128 x 256 (the widest single-CTA MMA; narrower
 // tiles measured slower on every workload: more A re-reads per FLOP)
 constexpr int kTcBN = 256, kTcStages = 4;
-// stream-K scratch of the bf16 grouped FFN: one fp32 partial tile and one
-// flag per CTA, for grids of up to kSkMaxCtas CTAs
-constexpr int kSkMaxCtas = 160;
-
 // Scratch of a rerouting dispatch (F rounds, nchunk chunks).
 struct RerouteWs {
     int32_t* srv;     // [T*k]
@@ -214,12 +243,15 @@ struct WsLayout {
     size_t idx, gate, counts, offsets, perm, slot_of, row_gate, xp, h, yp;
     size_t fhist, fbase, fpsum;   // per-router-chunk arrays of the forward path
     size_t fb_idx, fb_gate, reroute;   // overflow rerouting (F > 0)
-    size_t sk_partials, sk_flags;      // stream-K scratch of the bf16 grouped FFN
     size_t total;
 };
 
 // tokens per router CTA (= one dispatch chunk of the forward path)
-inline int router_chunk_tokens(int dtype) { return dtype == MOE_BF16 ? kRtBM : kRouterTM; }
+// Tokens per router CTA (= one dispatch chunk of the forward path).  bf16
+// uses 128-token tiles: smaller tiles (measured with 32 and 64) were slower,
+// since every router CTA streams all of W_r and pays the same fixed
+// load -> MMA -> epilogue latency.
+inline int router_chunk_tokens(int dtype, int /*T*/) { return dtype == MOE_BF16 ? kRtBM : kRouterTM; }
 
 size_t dispatch_ws_bytes(int A, int E) {
     const int nblk = std::max(1, ceil_div(A, kDispChunk));
@@ -248,16 +280,13 @@ WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype, int S = 0, int
     L.xp = take(A * d * es);
     L.h = take(HR * ff * es);
     L.yp = take(HR * d * es);
-    const size_t nchunk = size_t(std::max(1, ceil_div(T, router_chunk_tokens(dtype))));
+    const size_t nchunk = size_t(std::max(1, ceil_div(T, router_chunk_tokens(dtype, T))));
     L.fhist = take(nchunk * E * 4);
     L.fbase = take(nchunk * E * 4);
     L.fpsum = take(nchunk * E * 4);
     L.fb_idx = take(size_t(T) * F * 4);
     L.fb_gate = take(size_t(T) * F * 4);
     L.reroute = take(F > 0 ? reroute_ws_bytes(T, k, E, F, int(nchunk)) : 0);
-    const bool sk = dtype == MOE_BF16;
-    L.sk_partials = take(sk ? size_t(kSkMaxCtas) * kTcBM * kTcBN * sizeof(float) : 0);
-    L.sk_flags = take(sk ? size_t(kSkMaxCtas) * sizeof(unsigned long long) : 0);
     L.total = o;
     return L;
 }
@@ -357,30 +386,55 @@ int launch_router_ep(const void* x, const void* wr, const float* bias, int T, in
     return L.finish(launch_err);
 }
 
-template <int EP, int KMAX>
+template <int EP, int KMAX, int KSPLIT>
 int launch_router_tc(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
                      const RouterOut& o, cudaStream_t s) {
     CUtensorMap tmX, tmW;
-    if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), kRtBM)) return MOE_ERR_UNSUPPORTED;
+    const int tile_tok = router_chunk_tokens(MOE_BF16, T);
+    if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), uint32_t(tile_tok))) return MOE_ERR_UNSUPPORTED;
     if (!make_map_2d(&tmW, wr, uint64_t(d), uint64_t(E), EP)) return MOE_ERR_UNSUPPORTED;
-    auto kern = router_tc_kernel<EP, KMAX>;
-    const size_t smem = RtCfg<EP>::kSmemBytes;
+    auto kern = router_tc_kernel<EP, KMAX, KSPLIT>;
+    const size_t smem = RtCfg<EP, KSPLIT>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     Launch L(MOE_KERNEL_ROUTER, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(kern, dim3(ceil_div(T, kRtBM)), dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k,
-                            o.idx, o.gate, o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate);
+    const dim3 grid(ceil_div(T, tile_tok) * KSPLIT);
+    if (KSPLIT > 1)
+        launch_err = launch_pdl_cluster(kern, grid, dim3(kRtThreads), smem, KSPLIT, s, tmX, tmW, bias, T, d, E, k,
+                                        o.idx, o.gate, o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate,
+                                        tile_tok);
+    else
+        launch_err = launch_pdl(kern, grid, dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k, o.idx, o.gate,
+                                o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate, tile_tok);
     return L.finish(launch_err);
+}
+
+// Split K over a cluster when the token tiles alone would leave most SMs
+// idle: KSPLIT CTAs per tile (4 or 2) while tiles * KSPLIT fits the SMs and
+// each CTA keeps at least two k-blocks; only for E <= 64 (the partial
+// logits of the other CTAs must fit next to the stages in shared memory).
+template <int EP, int KMAX>
+int launch_router_tc_split(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
+                           const RouterOut& o, cudaStream_t s) {
+    if constexpr (EP <= 64) {
+        const int tiles = ceil_div(T, router_chunk_tokens(MOE_BF16, T));
+        const int kb = ceil_div(d, 64);
+        if (tiles * 4 <= num_sms() && kb >= 8)
+            return launch_router_tc<EP, KMAX, 4>(x, wr, bias, T, d, E, k, o, s);
+        if (tiles * 2 <= num_sms() && kb >= 4)
+            return launch_router_tc<EP, KMAX, 2>(x, wr, bias, T, d, E, k, o, s);
+    }
+    return launch_router_tc<EP, KMAX, 1>(x, wr, bias, T, d, E, k, o, s);
 }
 
 template <int KMAX>
 int launch_router_tc_k(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
                        const RouterOut& o, cudaStream_t s) {
-    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 128) return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 16) return launch_router_tc_split<16, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 32) return launch_router_tc_split<32, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 64) return launch_router_tc_split<64, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 128) return launch_router_tc_split<128, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    return launch_router_tc_split<256, KMAX>(x, wr, bias, T, d, E, k, o, s);
 }
 
 template <typename Tin>
@@ -463,13 +517,11 @@ struct SharedArgs {
 
 // Routed groups: E experts over rows offsets[0..E] of `a` (a_rows rows;
 // routed_rows_ub bounds offsets[E]).  E may be 0 when only shared groups run.
-// every stream-K launch takes a fresh epoch (never 0, the cleared flag)
-std::atomic<unsigned long long> g_sk_epoch{0x9E3779B97F4A7C15ull};
 
 template <int BN, int STAGES, int MODE>
 int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
               const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
-              const SharedArgs& sa, StreamK skp, int kernel_id, cudaStream_t s) {
+              const SharedArgs& sa, int kernel_id, cudaStream_t s) {
     CUtensorMap tmA, tmB, tmA2, tmB2;
     if (sa.g.S > 0) {
         if (!make_map_2d(&tmA2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
@@ -493,21 +545,54 @@ int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const v
     const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kTcBM)) + E +
                             static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kTcBM);
     const long long tiles_ub = mt_ub * ceil_div(N, BN);
-    int grid;
-    if (skp.partials != nullptr) {
-        // stream-K: one CTA per SM, each with an equal share of the k-block units
-        const long long units_ub = tiles_ub * ceil_div(a_cols, kTcBK);
-        grid = int(std::max(1ll, std::min<long long>(units_ub, std::min(num_sms(), kSkMaxCtas))));
-        skp.epoch = g_sk_epoch.fetch_add(1, std::memory_order_relaxed);
-    } else {
-        grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
-    }
+    const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
     launch_err = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, s, tmA, tmB, offsets, E, N, a_cols,
                             static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
                             static_cast<__nv_bfloat16*>(c), sa.g, tmA2, tmB2,
-                            static_cast<const __nv_bfloat16*>(sa.bias), skp);
+                            static_cast<const __nv_bfloat16*>(sa.bias));
+    return L.finish(launch_err);
+}
+
+// The CTA-pair variant (cta_group::2, 256 x 256 tiles): A map boxes of 128
+// rows, weight map boxes of 128 rows (half of the tile's N).
+constexpr int kTc2Stages = 6;
+
+template <int MODE>
+int launch_tc2(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
+               const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
+               const SharedArgs& sa, int kernel_id, cudaStream_t s) {
+    CUtensorMap tmA, tmB, tmA2, tmB2;
+    if (sa.g.S > 0) {
+        if (!make_map_2d(&tmA2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), 128)) return MOE_ERR_UNSUPPORTED;
+        if (!make_map_3d(&tmB2, sa.w, uint64_t(a_cols), uint64_t(N), uint64_t(sa.g.S), kTc2BN / 2))
+            return MOE_ERR_UNSUPPORTED;
+    }
+    if (E > 0) {
+        if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(a_rows), 128)) return MOE_ERR_UNSUPPORTED;
+        if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), kTc2BN / 2)) return MOE_ERR_UNSUPPORTED;
+    } else {
+        tmA = tmA2;
+        tmB = tmB2;
+    }
+    if (sa.g.S == 0) {
+        tmA2 = tmA;
+        tmB2 = tmB;
+    }
+    auto kern = ffn_tc2_bf16_kernel<kTc2Stages, MODE>;
+    const size_t smem = Tc2Cfg<kTc2Stages>::kSmemBytes;
+    if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
+    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kTc2BM)) + E +
+                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kTc2BM);
+    const long long tiles_ub = mt_ub * ceil_div(N, kTc2BN);
+    const int pairs = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms() / 2)));
+    Launch L(kernel_id, s);
+    cudaError_t launch_err;
+    launch_err = launch_pdl_cluster(kern, dim3(2 * pairs), dim3(kTcThreads), smem, 2, s, tmA, tmB, offsets, E, N,
+                                    a_cols, static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
+                                    static_cast<__nv_bfloat16*>(c), sa.g, tmA2, tmB2,
+                                    static_cast<const __nv_bfloat16*>(sa.bias));
     return L.finish(launch_err);
 }
 
@@ -543,10 +628,11 @@ struct SharedExperts {
 // max_rows routed rows followed by S * T shared rows (shared expert s, token
 // t at row max_rows + s * T + t).  out_rows (nullable): fc2 writes routed
 // row r to row out_rows[r] of yp (the direct output of a k == 1 layer).
-// skp: stream-K scratch for the bf16 launches (partials null: whole tiles)
+// use_pairs: bf16 fc2 on CTA pairs (256-row tiles), for layers whose experts
+// average enough rows that the doubled M tile wastes little
 int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
             const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp, int dtype,
-            const int32_t* out_rows, const SharedExperts& se, const StreamK& skp, cudaStream_t s) {
+            const int32_t* out_rows, const SharedExperts& se, bool use_pairs, cudaStream_t s) {
     const int h_rows = max_rows + se.S * se.T;
     SharedArgs s1, s2;
     if (se.S > 0) {
@@ -565,11 +651,17 @@ int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, 
     }
     int rc;
     if (dtype == MOE_BF16) {
+        // fc1 stays on single-CTA 128-row tiles: its K (= d) is short, so the
+        // pair kernel's doubled M padding costs more than its halved loads
+        // save (measured on the skewed and large workloads)
         rc = launch_tc<kTcBN, kTcStages, kFc1Gelu>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr,
-                                                   nullptr, h, s1, skp, MOE_KERNEL_FFN1, s);
+                                                   nullptr, h, s1, MOE_KERNEL_FFN1, s);
         if (rc != MOE_OK) return rc;
+        if (use_pairs)
+            return launch_tc2<kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, s2,
+                                        MOE_KERNEL_FFN2, s);
         return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate,
-                                                     out_rows, yp, s2, skp, MOE_KERNEL_FFN2, s);
+                                                     out_rows, yp, s2, MOE_KERNEL_FFN2, s);
     }
     rc = launch_simt<kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, s1, MOE_KERNEL_FFN1,
                                s);
@@ -963,7 +1055,7 @@ int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E,
         !aligned16(yp))
         return MOE_ERR_INVALID_ARG;
     return run_ffn(xp, offsets, max_rows, E, d, ff, w1, b1, w2, b2, row_gate, h, yp, dtype, nullptr,
-                   SharedExperts{}, StreamK{}, static_cast<cudaStream_t>(stream));
+                   SharedExperts{}, false, static_cast<cudaStream_t>(stream));
 }
 
 int moe_shared_ffn(const void* x, int T, int d, int ff, int S, const void* w1s, const void* b1s, const void* w2s,
@@ -985,7 +1077,7 @@ int moe_shared_ffn(const void* x, int T, int d, int ff, int S, const void* w1s, 
     se.w2 = w2s;
     se.b2 = b2s;
     return run_ffn(nullptr, nullptr, 0, 0, d, ff, nullptr, nullptr, nullptr, nullptr, nullptr, h, ys, dtype,
-                   nullptr, se, StreamK{}, static_cast<cudaStream_t>(stream));
+                   nullptr, se, false, static_cast<cudaStream_t>(stream));
 }
 
 int moe_combine(const void* yp, const int32_t* slot_of, const float* topk_gate, int T, int k, int d, int dtype,
@@ -1064,7 +1156,7 @@ int moe_forward_ex(const void* x, const void* w_router, const float* logit_bias,
     void* h = w + L.h;
     void* yp = w + L.yp;
     const int A = T * k;
-    const int chunk_tokens = router_chunk_tokens(dtype);
+    const int chunk_tokens = router_chunk_tokens(dtype, T);
     // rerouting only matters when a capacity can drop assignments
     const int F = capacity >= 0 ? reroute_rounds : 0;
     // top-1 without shared experts: every token has one contribution, so fc2
@@ -1092,13 +1184,11 @@ int moe_forward_ex(const void* x, const void* w_router, const float* logit_bias,
                                   perm, slot_of, nullptr, row_gate, stats, x, xp, d, dtype, direct ? out : nullptr,
                                   s);
     if (rc != MOE_OK) return rc;
-    StreamK skp{};
-    if (dtype == MOE_BF16) {
-        skp.partials = reinterpret_cast<float*>(w + L.sk_partials);
-        skp.flags = reinterpret_cast<unsigned long long*>(w + L.sk_flags);
-    }
+    // CTA pairs once the routed experts average at least 384 rows (256-row
+    // tiles then waste little on padding) or env MOE_PAIR_TILES forces it
+    const bool use_pairs = pair_tiles_enabled(static_cast<long long>(A) >= 384ll * E);
     if ((rc = run_ffn(xp, offsets, A, E, d, ff, w1, b1, w2, b2, row_gate, h, direct ? out : yp, dtype,
-                      direct ? perm : nullptr, se, skp, s)) != MOE_OK)
+                      direct ? perm : nullptr, se, use_pairs, s)) != MOE_OK)
         return rc;
     if (!direct) {
         const void* ys = static_cast<const uint8_t*>(yp) + size_t(A) * d * elem_bytes(dtype);
@@ -1122,6 +1212,12 @@ int moe_debug_gelu(const float* x, float* y, int n, int variant, void* stream) {
     if (!x || !y) return MOE_ERR_INVALID_ARG;
     gelu_probe_kernel<<<std::min(ceil_div(n, 256), 1024), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n,
                                                                                                      variant);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_debug_wait_timeout(int64_t limit_ns, void* stream) {
+    if (limit_ns <= 0 || static_cast<uint64_t>(limit_ns) > kWaitLimitNs) return MOE_ERR_INVALID_ARG;
+    wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(limit_ns));
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -214,3 +214,9 @@ def test_reroute_checks(lib):
     assert call(idx=None) == _lib.MOE_ERR_INVALID_ARG
     assert call(x=FAKE) == _lib.MOE_ERR_INVALID_ARG
     assert call(F=7) == _lib.MOE_ERR_UNSUPPORTED
+
+
+def test_wait_timeout_probe_checks_its_limit(lib):
+    assert lib.moe_debug_wait_timeout(0, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_debug_wait_timeout(-5, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_debug_wait_timeout(3_000_000_000, None) == _lib.MOE_ERR_INVALID_ARG   # above the 2 s cap

@@ -338,6 +338,11 @@ def test_forward_matches_oracle(w):
     (600, 64, 64, 256, 8, -1),       # the most experts and slots: 256 experts, top-8
     (2000, 256, 4096, 8, 1, -1),     # few tiles, long fc2 K, ragged rows
     (1500, 256, 2048, 6, 2, 300),    # k = 2 with capacity drops, long fc2 K
+    # >= 384 rows per expert: bf16 runs the CTA-pair (256-row tile) kernels
+    (4000, 72, 200, 4, 1, -1),       # pairs, ragged K and N tails, direct fc2 output
+    (5000, 128, 256, 8, 2, 900),     # pairs with capacity drops, k = 2
+    (6000, 64, 128, 4, 1, 1400),     # pairs, top-1 with drops (zeroed rows)
+    (3333, 192, 1088, 3, 1, -1),     # pairs, ragged last 256-row tile and N tail
 ])
 def test_forward_edge_cases(dtype, T, d, ff, E, k, cap):
     inp = wl.draw_custom(5, T=T, d=d, ff=ff, E=E, dtype=dtype, router_std=0.5)

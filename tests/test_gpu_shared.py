@@ -103,6 +103,7 @@ def test_forward_shared_matches_oracle(w):
     (777, 64, 128, 1, 1, -1, 8),       # the most shared experts, one routed expert
     (2000, 128, 256, 16, 1, 60, 2),    # top-1 with drops (no direct fc2 output with shared experts)
     (300, 136, 320, 4, 4, -1, 1),      # k = E
+    (3000, 64, 128, 2, 1, -1, 2),      # >= 384 rows per expert: CTA-pair kernels with shared groups
 ])
 def test_forward_shared_edge_cases(dtype, T, d, ff, E, k, cap, S):
     inp = wl.draw_custom(7, T=T, d=d, ff=ff, E=E, dtype=dtype, router_std=0.5, shared=S)
