@@ -314,17 +314,6 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mas
         : "memory");
 }
 
-// 16-byte store to the shared memory of CTA `rank` of the cluster, at the
-// offset `local` (a shared address of this CTA) names
-__device__ __forceinline__ void st_cluster_v4(uint32_t local, uint32_t rank, const uint32_t* v) {
-    asm volatile(
-        "{\n\t.reg .b32 ra;\n\t"
-        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-        "st.shared::cluster.v4.b32 [ra], {%2, %3, %4, %5};\n\t}\n" ::"r"(local),
-        "r"(rank), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
-        : "memory");
-}
-
 // arrive on the barrier at `bar`'s offset in CTA `rank` of the cluster
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
     asm volatile(

@@ -248,10 +248,10 @@ struct WsLayout {
 
 // tokens per router CTA (= one dispatch chunk of the forward path)
 // Tokens per router CTA (= one dispatch chunk of the forward path).  bf16
-// uses 128-token tiles: smaller tiles (measured with 32 and 64) were slower,
-// since every router CTA streams all of W_r and pays the same fixed
-// load -> MMA -> epilogue latency.
-inline int router_chunk_tokens(int dtype, int /*T*/) { return dtype == MOE_BF16 ? kRtBM : kRouterTM; }
+// uses 128-token tiles (32- and 64-token tiles and a split-K cluster of 4
+// CTAs per tile were measured no faster: every router CTA pays the same
+// fixed load -> MMA -> epilogue chain).
+inline int router_chunk_tokens(int dtype) { return dtype == MOE_BF16 ? kRtBM : kRouterTM; }
 
 size_t dispatch_ws_bytes(int A, int E) {
     const int nblk = std::max(1, ceil_div(A, kDispChunk));
@@ -280,7 +280,7 @@ WsLayout ws_layout(int T, int d, int ff, int E, int k, int dtype, int S = 0, int
     L.xp = take(A * d * es);
     L.h = take(HR * ff * es);
     L.yp = take(HR * d * es);
-    const size_t nchunk = size_t(std::max(1, ceil_div(T, router_chunk_tokens(dtype, T))));
+    const size_t nchunk = size_t(std::max(1, ceil_div(T, router_chunk_tokens(dtype))));
     L.fhist = take(nchunk * E * 4);
     L.fbase = take(nchunk * E * 4);
     L.fpsum = take(nchunk * E * 4);
@@ -386,55 +386,30 @@ int launch_router_ep(const void* x, const void* wr, const float* bias, int T, in
     return L.finish(launch_err);
 }
 
-template <int EP, int KMAX, int KSPLIT>
+template <int EP, int KMAX>
 int launch_router_tc(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
                      const RouterOut& o, cudaStream_t s) {
     CUtensorMap tmX, tmW;
-    const int tile_tok = router_chunk_tokens(MOE_BF16, T);
-    if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), uint32_t(tile_tok))) return MOE_ERR_UNSUPPORTED;
+    if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), kRtBM)) return MOE_ERR_UNSUPPORTED;
     if (!make_map_2d(&tmW, wr, uint64_t(d), uint64_t(E), EP)) return MOE_ERR_UNSUPPORTED;
-    auto kern = router_tc_kernel<EP, KMAX, KSPLIT>;
-    const size_t smem = RtCfg<EP, KSPLIT>::kSmemBytes;
+    auto kern = router_tc_kernel<EP, KMAX>;
+    const size_t smem = RtCfg<EP>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     Launch L(MOE_KERNEL_ROUTER, s);
     cudaError_t launch_err;
-    const dim3 grid(ceil_div(T, tile_tok) * KSPLIT);
-    if (KSPLIT > 1)
-        launch_err = launch_pdl_cluster(kern, grid, dim3(kRtThreads), smem, KSPLIT, s, tmX, tmW, bias, T, d, E, k,
-                                        o.idx, o.gate, o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate,
-                                        tile_tok);
-    else
-        launch_err = launch_pdl(kern, grid, dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k, o.idx, o.gate,
-                                o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate, tile_tok);
+    launch_err = launch_pdl(kern, dim3(ceil_div(T, kRtBM)), dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k,
+                            o.idx, o.gate, o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate);
     return L.finish(launch_err);
-}
-
-// Split K over a cluster when the token tiles alone would leave most SMs
-// idle: KSPLIT CTAs per tile (4 or 2) while tiles * KSPLIT fits the SMs and
-// each CTA keeps at least two k-blocks; only for E <= 64 (the partial
-// logits of the other CTAs must fit next to the stages in shared memory).
-template <int EP, int KMAX>
-int launch_router_tc_split(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
-                           const RouterOut& o, cudaStream_t s) {
-    if constexpr (EP <= 64) {
-        const int tiles = ceil_div(T, router_chunk_tokens(MOE_BF16, T));
-        const int kb = ceil_div(d, 64);
-        if (tiles * 4 <= num_sms() && kb >= 8)
-            return launch_router_tc<EP, KMAX, 4>(x, wr, bias, T, d, E, k, o, s);
-        if (tiles * 2 <= num_sms() && kb >= 4)
-            return launch_router_tc<EP, KMAX, 2>(x, wr, bias, T, d, E, k, o, s);
-    }
-    return launch_router_tc<EP, KMAX, 1>(x, wr, bias, T, d, E, k, o, s);
 }
 
 template <int KMAX>
 int launch_router_tc_k(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
                        const RouterOut& o, cudaStream_t s) {
-    if (E <= 16) return launch_router_tc_split<16, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 32) return launch_router_tc_split<32, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 64) return launch_router_tc_split<64, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 128) return launch_router_tc_split<128, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    return launch_router_tc_split<256, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 128) return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, o, s);
 }
 
 template <typename Tin>
@@ -1156,7 +1131,7 @@ int moe_forward_ex(const void* x, const void* w_router, const float* logit_bias,
     void* h = w + L.h;
     void* yp = w + L.yp;
     const int A = T * k;
-    const int chunk_tokens = router_chunk_tokens(dtype, T);
+    const int chunk_tokens = router_chunk_tokens(dtype);
     // rerouting only matters when a capacity can drop assignments
     const int F = capacity >= 0 ? reroute_rounds : 0;
     // top-1 without shared experts: every token has one contribution, so fc2

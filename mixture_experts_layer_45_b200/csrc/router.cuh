@@ -202,10 +202,8 @@ router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const 
 }
 
 // ===========================================================================
-// bf16 router on the tensor cores.  One CTA (or, with KSPLIT > 1, one
-// cluster of KSPLIT CTAs) per tile of tile_tok <= 128 tokens (the MMA is
-// always M = 128; rows past tile_tok are ignored), 192 threads:
-//   warp 0      TMA producer: x tile rows [t0, t0+tile_tok) and W_r, 64 columns of
+// bf16 router on the tensor cores.  One CTA per 128-token tile, 192 threads:
+//   warp 0      TMA producer: x tile rows [t0, t0+128) and W_r, 64 columns of
 //               K per stage (128B swizzle; rows past T and experts past E
 //               are zero-filled by the tensor maps)
 //   warp 1      TMEM allocator and MMA issuer: logits[128 x EP] in fp32
@@ -213,39 +211,29 @@ router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const 
 //               TMEM loads, register top-k (ties to the lower index), gates,
 //               then the per-expert probability column sums (shared-memory
 //               transpose, fixed summation order) and the expert histogram
-// Split K (KSPLIT CTAs of a cluster per tile, for batches too short to fill
-// the GPU with tiles): CTA r multiplies k-blocks [r*KB/KSPLIT, (r+1)*KB/
-// KSPLIT) into its own tensor memory; CTAs 1.. store their fp32 partial
-// logits into CTA 0's shared memory (distributed shared memory), a cluster
-// barrier orders the stores, and CTA 0 adds them in rank order before its
-// epilogue.  The chain load -> MMA -> epilogue of each CTA is KSPLIT times
-// shorter.
 // ===========================================================================
 constexpr int kRtBM = 128;
 constexpr int kRtThreads = 192;
 
-template <int EP, int KSPLIT = 1>
+template <int EP>
 struct RtCfg {
     static constexpr uint32_t kABytes = kRtBM * 64 * 2;
     static constexpr uint32_t kBBytes = EP * 64 * 2;
     static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = KSPLIT > 1 ? 4 : ((EP <= 64) ? 8 : (EP <= 128 ? 6 : 4));
+    static constexpr int kStages = (EP <= 64) ? 8 : (EP <= 128 ? 6 : 4);
     static constexpr uint32_t kTmemCols = EP < 32 ? 32 : EP;
-    static constexpr int kRedLd = ((EP + 31) / 32) * 32 + 4;   // floats per partial-logit row
-    static constexpr size_t kRedBytes = size_t(KSPLIT - 1) * kRtBM * kRedLd * sizeof(float);
-    static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + kRedBytes + 1024;
+    static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024;
 };
 
 // KMAX >= k + F: the selection also yields the F fallback experts (fb_idx /
 // fb_gate [T, F]), as in router_topk_kernel.
-template <int EP, int KMAX, int KSPLIT>
+template <int EP, int KMAX>
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ bias, int T, int d, int E, int k, int32_t* __restrict__ topk_idx,
                  float* __restrict__ topk_gate, float* __restrict__ prob_sum, float* __restrict__ psum_part,
-                 int32_t* __restrict__ hist, int F, int32_t* __restrict__ fb_idx, float* __restrict__ fb_gate,
-                 int tile_tok) {
-    using Cfg = RtCfg<EP, KSPLIT>;
+                 int32_t* __restrict__ hist, int F, int32_t* __restrict__ fb_idx, float* __restrict__ fb_gate) {
+    using Cfg = RtCfg<EP>;
     constexpr int S = Cfg::kStages;
     constexpr int NCH = (EP + 31) / 32;   // 32-column TMEM chunks
     __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], done_bar;
@@ -281,15 +269,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     pdl_wait();
     pdl_release();
     const uint32_t tmem_base = tmem_slot;
-    const int KBall = (d + 63) / 64;
-    const int tile = KSPLIT > 1 ? int(blockIdx.x) / KSPLIT : int(blockIdx.x);
-    const int rank = KSPLIT > 1 ? int(cluster_ctarank()) : 0;
-    const int kb_begin = KBall * rank / KSPLIT, kb_end = KBall * (rank + 1) / KSPLIT;
-    const int KB = kb_end - kb_begin;   // k-blocks of this CTA
-    // partial logits of CTAs 1.. (in CTA 0's shared memory, after the stages)
-    float* red = reinterpret_cast<float*>(smem + size_t(S) * Cfg::kStageBytes);
-    const int t0 = tile * tile_tok;
-    const uint32_t stage_tx = uint32_t(tile_tok) * 128u + Cfg::kBBytes;   // x box rows + W
+    const int KB = (d + 63) / 64;
+    const int t0 = blockIdx.x * kRtBM;
     volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
@@ -301,9 +282,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             for (int kb = 0; kb < KB; ++kb) {
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) break;
                 uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
-                mbar_arrive_expect_tx(&full_bar[stage], stage_tx);
-                tma_load_2d(sa, &tmX, &full_bar[stage], (kb_begin + kb) * 64, t0);
-                tma_load_2d(sa + Cfg::kABytes, &tmW, &full_bar[stage], (kb_begin + kb) * 64, 0);
+                mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
+                tma_load_2d(sa, &tmX, &full_bar[stage], kb * 64, t0);
+                tma_load_2d(sa + Cfg::kABytes, &tmW, &full_bar[stage], kb * 64, 0);
                 last_parity[stage] = int(phase);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
@@ -339,59 +320,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
         }
     } else {
-        // CTAs 1.. of a split-K cluster: hand the partial logits to CTA 0
-        const bool ok = mbar_wait(&done_bar, 0, abort_p);
-        tc_fence_after();
-        if constexpr (KSPLIT > 1) {
-            if (rank > 0) {
-                const int q = warp & 3;
-                const int row = q * 32 + lane;
-                const uint32_t dst = smem_u32(red + (size_t(rank - 1) * kRtBM + row) * Cfg::kRedLd);
-#pragma unroll 1
-                for (int c = 0; c < NCH; ++c) {
-                    uint32_t r[32];
-                    __syncwarp();
-                    tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
-                    tmem_ld_wait();
-                    if (!ok) continue;
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) st_cluster_v4(dst + uint32_t((c * 32 + v * 4) * 4), 0, r + v * 4);
-                }
-            }
-        }
-        tc_fence_before();
-    }
-    // the partial-logit stores of CTAs 1.. are visible in CTA 0 after this
-    if constexpr (KSPLIT > 1) cluster_sync();
-    if (warp >= 2 && rank == 0) {
         const int ew = warp - 2;      // 0..3
         const int q = warp & 3;       // TMEM lane quarter
         const int row = q * 32 + lane;
         const int t = t0 + row;
-        const bool valid = row < tile_tok && t < T;
+        const bool valid = t < T;
         const bool ok = mbar_wait(&done_bar, 0, abort_p);
         tc_fence_after();
-        // logits chunk c of this row: this CTA's accumulators plus, in rank
-        // order, the partials of the other CTAs of the cluster
-        auto load_logits = [&](int c, uint32_t (&r)[32]) {
-            __syncwarp();
-            tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
-            tmem_ld_wait();
-            if constexpr (KSPLIT > 1) {
-#pragma unroll 1
-                for (int j = 0; j < KSPLIT - 1; ++j) {
-                    const float* src = red + (size_t(j) * kRtBM + row) * Cfg::kRedLd + c * 32;
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const float4 pv = *reinterpret_cast<const float4*>(src + v * 4);
-                        r[v * 4] = __float_as_uint(__uint_as_float(r[v * 4]) + pv.x);
-                        r[v * 4 + 1] = __float_as_uint(__uint_as_float(r[v * 4 + 1]) + pv.y);
-                        r[v * 4 + 2] = __float_as_uint(__uint_as_float(r[v * 4 + 2]) + pv.z);
-                        r[v * 4 + 3] = __float_as_uint(__uint_as_float(r[v * 4 + 3]) + pv.w);
-                    }
-                }
-            }
-        };
         float m = -INFINITY, ssum = 0.f;
         float tv[KMAX];
         int ti[KMAX];
@@ -404,7 +339,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll 1
         for (int c = 0; c < NCH; ++c) {
             uint32_t r[32];
-            load_logits(c, r);
+            __syncwarp();
+            tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
+            tmem_ld_wait();
             float l[32];
             float cm = -INFINITY;
 #pragma unroll
@@ -467,7 +404,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll 1
             for (int c = 0; c < NCH; ++c) {
                 uint32_t r[32];
-                load_logits(c, r);
+                __syncwarp();
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
+                tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int e = c * 32 + i;
@@ -489,11 +428,11 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         tc_fence_before();
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E && rank == 0; e += kRtThreads) {
+    for (int e = threadIdx.x; e < E; e += kRtThreads) {
         const float tot = ((s_col[0][e] + s_col[1][e]) + s_col[2][e]) + s_col[3][e];
-        if (psum_part != nullptr) psum_part[size_t(tile) * E + e] = tot;
+        if (psum_part != nullptr) psum_part[size_t(blockIdx.x) * E + e] = tot;
         else if (prob_sum != nullptr) atomicAdd(prob_sum + e, tot);
-        if (hist != nullptr) hist[size_t(tile) * E + e] = s_hist[e];
+        if (hist != nullptr) hist[size_t(blockIdx.x) * E + e] = s_hist[e];
     }
     if (warp == 1) {
         tc_fence_after();
