@@ -213,7 +213,8 @@ MOE_API int moe_dispatch_noalloc(const int32_t* topk_idx, const float* topk_gate
  * number of rows xp, h and yp are allocated for (>= offsets[E], normally
  * T*k).  h is caller-provided scratch [max_rows, ff].  bf16 runs on the
  * tcgen05 tensor cores with fp32 accumulation in tensor memory; h and yp are
- * rounded to bf16.  f32 runs in fp32 FMA. */
+ * rounded to bf16.  f32 runs on the tensor cores as three-pass TF32 (each
+ * operand split into a TF32 part and its fp32 remainder; fp32-level error). */
 MOE_API int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows,
                     int E, int d, int ff,
                     const void* w1, const void* b1, const void* w2, const void* b2,

@@ -219,6 +219,24 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64
         : "memory");
 }
 
+// D(tmem) (+)= A(smem) * B(smem)^T, kind::tf32 (fp32 operands read as tf32,
+// fp32 accumulate)
+__device__ __forceinline__ void umma_tf32(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// generic-proxy shared-memory writes of this thread become visible to the
+// async proxy (tensor-core operand reads)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // arrive once on `bar` when every tcgen05 op issued so far by this thread completes
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -337,6 +355,16 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {
     d |= static_cast<uint64_t>(1) << 46;                        // version
     d |= static_cast<uint64_t>(2) << 61;                        // 128B swizzle
     return d;
+}
+
+// Instruction descriptor, kind::tf32: fp32 accumulator, tf32 A and B, both
+// K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+    return (1u << 4)                                   // D format: f32
+         | (2u << 7)                                   // A format: tf32
+         | (2u << 10)                                  // B format: tf32
+         | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both

@@ -311,29 +311,36 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 [rows, cols] row-major, box {64, box_rows}, 128B swizzle
-bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+// [rows, cols] row-major of dtype (bf16 or fp32), box {128 B of columns,
+// box_rows}, 128B swizzle
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                 int dtype = MOE_BF16) {
     EncodeTiledFn enc = encode_fn();
     if (enc == nullptr) return false;
+    const uint64_t es = elem_bytes(dtype);
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {uint32_t(kTcBK), box_rows};
+    const cuuint64_t strides[1] = {cols * es};
+    const cuuint32_t box[2] = {uint32_t(128 / es), box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return enc(m, dtype == MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [E, rows, cols], box {64, box_rows, 1}, 128B swizzle
-bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E, uint32_t box_rows) {
+// [E, rows, cols] of dtype, box {128 B of columns, box_rows, 1}, 128B swizzle
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t E, uint32_t box_rows,
+                 int dtype = MOE_BF16) {
     EncodeTiledFn enc = encode_fn();
     if (enc == nullptr) return false;
+    const uint64_t es = elem_bytes(dtype);
     const cuuint64_t dims[3] = {cols, rows, E};
-    const cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
-    const cuuint32_t box[3] = {uint32_t(kTcBK), box_rows, 1};
+    const cuuint64_t strides[2] = {cols * es, cols * rows * es};
+    const cuuint32_t box[3] = {uint32_t(128 / es), box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return enc(m, dtype == MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -571,21 +578,44 @@ int launch_tc2(const void* a, int a_cols, int a_rows, int routed_rows_ub, const 
     return L.finish(launch_err);
 }
 
+// fp32 on the tensor cores, three-pass TF32: 128 x 128 tiles, 3 stages
+constexpr int kTfBN = 128, kTfStages = 3;
+
 template <int MODE>
-int launch_simt(const void* a, int K, int routed_rows_ub, const void* w, int N, int E, const int32_t* offsets,
-                const void* bias, const float* row_gate, const int32_t* out_rows, void* c, const SharedArgs& sa,
-                int kernel_id, cudaStream_t s) {
-    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kSgBM)) + E +
-                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kSgBM);
-    const long long tiles_ub = mt_ub * ceil_div(N, kSgBN);
-    const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, 2ll * num_sms())));
+int launch_tf32x3(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
+                  const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
+                  const SharedArgs& sa, int kernel_id, cudaStream_t s) {
+    CUtensorMap tmA, tmB, tmA2, tmB2;
+    if (sa.g.S > 0) {
+        if (!make_map_2d(&tmA2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), kTcBM, MOE_F32))
+            return MOE_ERR_UNSUPPORTED;
+        if (!make_map_3d(&tmB2, sa.w, uint64_t(a_cols), uint64_t(N), uint64_t(sa.g.S), kTfBN, MOE_F32))
+            return MOE_ERR_UNSUPPORTED;
+    }
+    if (E > 0) {
+        if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(a_rows), kTcBM, MOE_F32)) return MOE_ERR_UNSUPPORTED;
+        if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), kTfBN, MOE_F32))
+            return MOE_ERR_UNSUPPORTED;
+    } else {
+        tmA = tmA2;
+        tmB = tmB2;
+    }
+    if (sa.g.S == 0) {
+        tmA2 = tmA;
+        tmB2 = tmB;
+    }
+    auto kern = ffn_tc_f32x3_kernel<kTfBN, kTfStages, MODE>;
+    const size_t smem = TfCfg<kTfBN, kTfStages>::kSmemBytes;
+    if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
+    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kTcBM)) + E +
+                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kTcBM);
+    const long long tiles_ub = mt_ub * ceil_div(N, kTfBN);
+    const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(ffn_simt_f32_kernel<MODE>, dim3(grid), dim3(kSgThreads), 0, s,
-                            static_cast<const float*>(a), offsets, E, N, K, static_cast<const float*>(w),
-                            static_cast<const float*>(bias), row_gate, out_rows, static_cast<float*>(c), sa.g,
-                            static_cast<const float*>(sa.a), static_cast<const float*>(sa.w),
-                            static_cast<const float*>(sa.bias));
+    launch_err = launch_pdl(kern, dim3(grid), dim3(kTfThreads), smem, s, tmA, tmB, offsets, E, N, a_cols,
+                            static_cast<const float*>(bias), row_gate, out_rows, static_cast<float*>(c), sa.g, tmA2,
+                            tmB2, static_cast<const float*>(sa.bias));
     return L.finish(launch_err);
 }
 
@@ -638,11 +668,11 @@ int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, 
         return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate,
                                                      out_rows, yp, s2, MOE_KERNEL_FFN2, s);
     }
-    rc = launch_simt<kFc1Gelu>(xp, d, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, s1, MOE_KERNEL_FFN1,
-                               s);
+    rc = launch_tf32x3<kFc1Gelu>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, s1,
+                                 MOE_KERNEL_FFN1, s);
     if (rc != MOE_OK) return rc;
-    return launch_simt<kFc2Gate>(h, ff, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, s2,
-                                 MOE_KERNEL_FFN2, s);
+    return launch_tf32x3<kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, s2,
+                                   MOE_KERNEL_FFN2, s);
 }
 
 // Dispatch of the fused forward path from the router's per-chunk histograms
