@@ -105,11 +105,29 @@ class Launch {
     cudaEvent_t start_ = nullptr;
 };
 
+// Every kernel of the library asks for the largest shared-memory carveout,
+// so consecutive kernels of a step never reconfigure an SM's L1/shared
+// split between them (set once per kernel and device).
+std::mutex g_carve_mu;
+std::vector<std::pair<const void*, int>> g_carve_done;
+
+inline void uniform_carveout(const void* kern) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return;
+    std::lock_guard<std::mutex> lk(g_carve_mu);
+    for (const auto& kd : g_carve_done)
+        if (kd.first == kern && kd.second == dev) return;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared));
+    cudaGetLastError();   // a refused hint is not an error of the launch
+    g_carve_done.emplace_back(kern, dev);
+}
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel on the stream drains; the kernels order their own
 // global reads with griddepcontrol.wait.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+    uniform_carveout(reinterpret_cast<const void*>(kern));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -127,6 +145,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, int cluster_x,
                                cudaStream_t s, Args&&... args) {
+    uniform_carveout(reinterpret_cast<const void*>(kern));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -633,6 +652,21 @@ struct SharedExperts {
 // max_rows routed rows followed by S * T shared rows (shared expert s, token
 // t at row max_rows + s * T + t).  out_rows (nullable): fc2 writes routed
 // row r to row out_rows[r] of yp (the direct output of a k == 1 layer).
+// fc2 tile width for layers whose experts hold about one 128-row tile each:
+// 192 instead of 256 columns when that keeps the expected tiles within one
+// wave while 256 would leave a quarter of the SMs idle (expected tiles
+// assume balanced experts; the tile table itself comes from the device)
+constexpr int kTcBNNarrow = 192, kTcStagesNarrow = 5;
+
+bool fc2_narrow_tiles(int max_rows, int E, int N, const SharedExperts& se) {
+    if (E <= 0) return false;
+    const long long per_expert = ceil_div(ceil_div(max_rows, E), kTcBM);
+    const long long mt = per_expert * E + static_cast<long long>(se.S) * ceil_div(se.T, kTcBM);
+    const long long wide = mt * ceil_div(N, kTcBN), narrow = mt * ceil_div(N, kTcBNNarrow);
+    const int sms = num_sms();
+    return 4 * wide < 3ll * sms && narrow <= sms && narrow > wide;
+}
+
 // use_pairs: bf16 fc2 on CTA pairs (256-row tiles), for layers whose experts
 // average enough rows that the doubled M tile wastes little
 int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
@@ -665,6 +699,12 @@ int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, 
         if (use_pairs)
             return launch_tc2<kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, s2,
                                         MOE_KERNEL_FFN2, s);
+        // fc2 of a layer with about one M tile per expert (switch-top1: 96
+        // tiles of 256 columns for 148 SMs): 192-column tiles put 4/3 as many
+        // SMs on the weight stream
+        if (fc2_narrow_tiles(max_rows, E, d, se))
+            return launch_tc<kTcBNNarrow, kTcStagesNarrow, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2,
+                                                                     row_gate, out_rows, yp, s2, MOE_KERNEL_FFN2, s);
         return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate,
                                                      out_rows, yp, s2, MOE_KERNEL_FFN2, s);
     }
