@@ -327,81 +327,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const bool valid = t < T;
         const bool ok = mbar_wait(&done_bar, 0, abort_p);
         tc_fence_after();
-        float m = -INFINITY, ssum = 0.f;
-        float tv[KMAX];
-        int ti[KMAX];
+        if constexpr (NCH <= 2) {
+            // E <= 64: the whole logits row stays in registers, so one
+            // tensor-memory read serves the max, the exponentials (computed
+            // once), the top-k and the probability column sums
+            float l[NCH][32];
+            float m = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            tv[j] = -INFINITY;
-            ti[j] = 0x7fffffff;
-        }
-        // pass 1: online softmax statistics and top-k over the logits row
-#pragma unroll 1
-        for (int c = 0; c < NCH; ++c) {
-            uint32_t r[32];
-            __syncwarp();
-            tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
-            tmem_ld_wait();
-            float l[32];
-            float cm = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int e = c * 32 + i;
-                float v = (e < E && ok) ? __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f) : -INFINITY;
-                if (v != v) v = -INFINITY;
-                l[i] = v;
-                cm = fmaxf(cm, v);
-            }
-            const float mn = fmaxf(m, cm);
-            if (mn != -INFINITY) {
-                float acc = (m == -INFINITY) ? 0.f : ssum * expf(m - mn);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) acc += (l[i] == -INFINITY) ? 0.f : expf(l[i] - mn);
-                ssum = acc;
-                m = mn;
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float v = l[i];
-                int ix = c * 32 + i;
-                if (v == -INFINITY || !(v > tv[KMAX - 1])) continue;
-#pragma unroll
-                for (int j = 0; j < KMAX; ++j) {
-                    if (v > tv[j]) {
-                        const float tf = tv[j];
-                        tv[j] = v;
-                        v = tf;
-                        const int tix = ti[j];
-                        ti[j] = ix;
-                        ix = tix;
-                    }
-                }
-            }
-        }
-        const float inv = 1.0f / ssum;
-        if (valid && ok) {
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                if (j < k + F) {
-                    // fewer than k + F finite logits cannot happen for k + F <= E with finite inputs;
-                    // guard so an all-NaN row still yields valid, distinct indices
-                    int e = ti[j];
-                    if (e >= E) e = j;
-                    const float g = (tv[j] == -INFINITY) ? 0.f : expf(tv[j] - m) * inv;
-                    if (j < k) {
-                        topk_idx[size_t(t) * k + j] = e;
-                        topk_gate[size_t(t) * k + j] = g;
-                        atomicAdd(&s_hist[e], 1);
-                    } else {
-                        fb_idx[size_t(t) * F + (j - k)] = e;
-                        fb_gate[size_t(t) * F + (j - k)] = g;
-                    }
-                }
-            }
-        }
-        // pass 2: per-expert sums of this tile's probabilities (fixed order)
-        if (prob_sum != nullptr || psum_part != nullptr) {
-#pragma unroll 1
             for (int c = 0; c < NCH; ++c) {
                 uint32_t r[32];
                 __syncwarp();
@@ -410,19 +342,181 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int e = c * 32 + i;
-                    float p = 0.f;
-                    if (valid && ok && e < E) {
-                        float v = __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f);
-                        p = (v != v) ? 0.f : expf(v - m) * inv;
-                    }
-                    s_tr[ew][lane][i] = p;
+                    float v = (e < E && ok) ? __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f) : -INFINITY;
+                    if (v != v) v = -INFINITY;
+                    l[c][i] = v;
+                    m = fmaxf(m, v);
                 }
-                __syncwarp();
-                float cs = 0.f;
+            }
+            // exponentials and their sum (four partial sums for shorter chains)
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < 32; ++i) cs += s_tr[ew][i][lane];
-                s_col[q][c * 32 + lane] = cs;
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float ex = (l[c][i] == -INFINITY) ? 0.f : __expf(l[c][i] - m);
+                    ps[i & 3] += ex;
+                    l[c][i] = ex;   // l now holds the exponentials; the logits order is kept in tv/ti below
+                }
+            const float inv = 1.0f / ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            // top-k by exponential (monotone in the logit; exact ties keep
+            // the lower index since later equal values do not displace)
+            float tv[KMAX];
+            int ti[KMAX];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                tv[j] = -1.f;
+                ti[j] = 0x7fffffff;
+            }
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float v = (c * 32 + i < E) ? l[c][i] : -1.f;
+                    int ix = c * 32 + i;
+                    if (!(v > tv[KMAX - 1])) continue;
+#pragma unroll
+                    for (int j = 0; j < KMAX; ++j) {
+                        if (v > tv[j]) {
+                            const float tf = tv[j];
+                            tv[j] = v;
+                            v = tf;
+                            const int tix = ti[j];
+                            ti[j] = ix;
+                            ix = tix;
+                        }
+                    }
+                }
+            if (valid && ok) {
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    if (j < k + F) {
+                        int e = ti[j];
+                        if (e >= E) e = j;
+                        const float g = (tv[j] < 0.f) ? 0.f : tv[j] * inv;
+                        if (j < k) {
+                            topk_idx[size_t(t) * k + j] = e;
+                            topk_gate[size_t(t) * k + j] = g;
+                            atomicAdd(&s_hist[e], 1);
+                        } else {
+                            fb_idx[size_t(t) * F + (j - k)] = e;
+                            fb_gate[size_t(t) * F + (j - k)] = g;
+                        }
+                    }
+                }
+            }
+            if (prob_sum != nullptr || psum_part != nullptr) {
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        s_tr[ew][lane][i] = (valid && ok && c * 32 + i < E) ? l[c][i] * inv : 0.f;
+                    __syncwarp();
+                    float cs = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) cs += s_tr[ew][i][lane];
+                    s_col[q][c * 32 + lane] = cs;
+                    __syncwarp();
+                }
+            }
+        } else {
+            float m = -INFINITY, ssum = 0.f;
+            float tv[KMAX];
+            int ti[KMAX];
+    #pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                tv[j] = -INFINITY;
+                ti[j] = 0x7fffffff;
+            }
+            // pass 1: online softmax statistics and top-k over the logits row
+    #pragma unroll 1
+            for (int c = 0; c < NCH; ++c) {
+                uint32_t r[32];
                 __syncwarp();
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
+                tmem_ld_wait();
+                float l[32];
+                float cm = -INFINITY;
+    #pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int e = c * 32 + i;
+                    float v = (e < E && ok) ? __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f) : -INFINITY;
+                    if (v != v) v = -INFINITY;
+                    l[i] = v;
+                    cm = fmaxf(cm, v);
+                }
+                const float mn = fmaxf(m, cm);
+                if (mn != -INFINITY) {
+                    float acc = (m == -INFINITY) ? 0.f : ssum * expf(m - mn);
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) acc += (l[i] == -INFINITY) ? 0.f : expf(l[i] - mn);
+                    ssum = acc;
+                    m = mn;
+                }
+    #pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float v = l[i];
+                    int ix = c * 32 + i;
+                    if (v == -INFINITY || !(v > tv[KMAX - 1])) continue;
+    #pragma unroll
+                    for (int j = 0; j < KMAX; ++j) {
+                        if (v > tv[j]) {
+                            const float tf = tv[j];
+                            tv[j] = v;
+                            v = tf;
+                            const int tix = ti[j];
+                            ti[j] = ix;
+                            ix = tix;
+                        }
+                    }
+                }
+            }
+            const float inv = 1.0f / ssum;
+            if (valid && ok) {
+    #pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    if (j < k + F) {
+                        // fewer than k + F finite logits cannot happen for k + F <= E with finite inputs;
+                        // guard so an all-NaN row still yields valid, distinct indices
+                        int e = ti[j];
+                        if (e >= E) e = j;
+                        const float g = (tv[j] == -INFINITY) ? 0.f : expf(tv[j] - m) * inv;
+                        if (j < k) {
+                            topk_idx[size_t(t) * k + j] = e;
+                            topk_gate[size_t(t) * k + j] = g;
+                            atomicAdd(&s_hist[e], 1);
+                        } else {
+                            fb_idx[size_t(t) * F + (j - k)] = e;
+                            fb_gate[size_t(t) * F + (j - k)] = g;
+                        }
+                    }
+                }
+            }
+            // pass 2: per-expert sums of this tile's probabilities (fixed order)
+            if (prob_sum != nullptr || psum_part != nullptr) {
+    #pragma unroll 1
+                for (int c = 0; c < NCH; ++c) {
+                    uint32_t r[32];
+                    __syncwarp();
+                    tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
+                    tmem_ld_wait();
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int e = c * 32 + i;
+                        float p = 0.f;
+                        if (valid && ok && e < E) {
+                            float v = __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f);
+                            p = (v != v) ? 0.f : expf(v - m) * inv;
+                        }
+                        s_tr[ew][lane][i] = p;
+                    }
+                    __syncwarp();
+                    float cs = 0.f;
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) cs += s_tr[ew][i][lane];
+                    s_col[q][c * 32 + lane] = cs;
+                    __syncwarp();
+                }
             }
         }
         tc_fence_before();
