@@ -516,6 +516,41 @@ struct SharedArgs {
     SharedGroups g{};
 };
 
+// The four operand maps of a grouped-FFN launch: routed A rows and weights,
+// shared-expert A rows and weights (each side falls back to the other when
+// it has no groups, so every map handed to the kernel is valid).
+struct FfnMaps {
+    CUtensorMap a, b, a2, b2;
+};
+
+bool make_ffn_maps(FfnMaps& m, const void* a, int a_cols, int a_rows, const void* w, int N, int E,
+                   const SharedArgs& sa, uint32_t a_box_rows, uint32_t w_box_rows, int dtype) {
+    if (sa.g.S > 0) {
+        if (!make_map_2d(&m.a2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), a_box_rows, dtype)) return false;
+        if (!make_map_3d(&m.b2, sa.w, uint64_t(a_cols), uint64_t(N), uint64_t(sa.g.S), w_box_rows, dtype))
+            return false;
+    }
+    if (E > 0) {
+        if (!make_map_2d(&m.a, a, uint64_t(a_cols), uint64_t(a_rows), a_box_rows, dtype)) return false;
+        if (!make_map_3d(&m.b, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), w_box_rows, dtype)) return false;
+    } else {
+        m.a = m.a2;
+        m.b = m.b2;
+    }
+    if (sa.g.S == 0) {
+        m.a2 = m.a;
+        m.b2 = m.b;
+    }
+    return true;
+}
+
+// Upper bound of a launch's tiles (the real count comes from the device offsets)
+long long ffn_tiles_ub(int routed_rows_ub, int E, const SharedArgs& sa, int BM, int N, int BN) {
+    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, BM)) + E +
+                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, BM);
+    return mt_ub * ceil_div(N, BN);
+}
+
 // Routed groups: E experts over rows offsets[0..E] of `a` (a_rows rows;
 // routed_rows_ub bounds offsets[E]).  E may be 0 when only shared groups run.
 
@@ -523,35 +558,18 @@ template <int BN, int STAGES, int MODE>
 int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
               const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
               const SharedArgs& sa, int kernel_id, cudaStream_t s) {
-    CUtensorMap tmA, tmB, tmA2, tmB2;
-    if (sa.g.S > 0) {
-        if (!make_map_2d(&tmA2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
-        if (!make_map_3d(&tmB2, sa.w, uint64_t(a_cols), uint64_t(N), uint64_t(sa.g.S), BN))
-            return MOE_ERR_UNSUPPORTED;
-    }
-    if (E > 0) {
-        if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(a_rows), kTcBM)) return MOE_ERR_UNSUPPORTED;
-        if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), BN)) return MOE_ERR_UNSUPPORTED;
-    } else {
-        tmA = tmA2;
-        tmB = tmB2;
-    }
-    if (sa.g.S == 0) {
-        tmA2 = tmA;
-        tmB2 = tmB;
-    }
+    FfnMaps mp;
+    if (!make_ffn_maps(mp, a, a_cols, a_rows, w, N, E, sa, kTcBM, BN, MOE_BF16)) return MOE_ERR_UNSUPPORTED;
     auto kern = ffn_tc_bf16_kernel<BN, STAGES, MODE>;
     const size_t smem = TcCfg<BN, STAGES>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
-    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kTcBM)) + E +
-                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kTcBM);
-    const long long tiles_ub = mt_ub * ceil_div(N, BN);
+    const long long tiles_ub = ffn_tiles_ub(routed_rows_ub, E, sa, kTcBM, N, BN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, s, tmA, tmB, offsets, E, N, a_cols,
+    launch_err = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, s, mp.a, mp.b, offsets, E, N, a_cols,
                             static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
-                            static_cast<__nv_bfloat16*>(c), sa.g, tmA2, tmB2,
+                            static_cast<__nv_bfloat16*>(c), sa.g, mp.a2, mp.b2,
                             static_cast<const __nv_bfloat16*>(sa.bias));
     return L.finish(launch_err);
 }
@@ -564,35 +582,18 @@ template <int MODE>
 int launch_tc2(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
                const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
                const SharedArgs& sa, int kernel_id, cudaStream_t s) {
-    CUtensorMap tmA, tmB, tmA2, tmB2;
-    if (sa.g.S > 0) {
-        if (!make_map_2d(&tmA2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), 128)) return MOE_ERR_UNSUPPORTED;
-        if (!make_map_3d(&tmB2, sa.w, uint64_t(a_cols), uint64_t(N), uint64_t(sa.g.S), kTc2BN / 2))
-            return MOE_ERR_UNSUPPORTED;
-    }
-    if (E > 0) {
-        if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(a_rows), 128)) return MOE_ERR_UNSUPPORTED;
-        if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), kTc2BN / 2)) return MOE_ERR_UNSUPPORTED;
-    } else {
-        tmA = tmA2;
-        tmB = tmB2;
-    }
-    if (sa.g.S == 0) {
-        tmA2 = tmA;
-        tmB2 = tmB;
-    }
+    FfnMaps mp;
+    if (!make_ffn_maps(mp, a, a_cols, a_rows, w, N, E, sa, 128, kTc2BN / 2, MOE_BF16)) return MOE_ERR_UNSUPPORTED;
     auto kern = ffn_tc2_bf16_kernel<kTc2Stages, MODE>;
     const size_t smem = Tc2Cfg<kTc2Stages>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
-    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kTc2BM)) + E +
-                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kTc2BM);
-    const long long tiles_ub = mt_ub * ceil_div(N, kTc2BN);
+    const long long tiles_ub = ffn_tiles_ub(routed_rows_ub, E, sa, kTc2BM, N, kTc2BN);
     const int pairs = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms() / 2)));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl_cluster(kern, dim3(2 * pairs), dim3(kTcThreads), smem, 2, s, tmA, tmB, offsets, E, N,
+    launch_err = launch_pdl_cluster(kern, dim3(2 * pairs), dim3(kTcThreads), smem, 2, s, mp.a, mp.b, offsets, E, N,
                                     a_cols, static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
-                                    static_cast<__nv_bfloat16*>(c), sa.g, tmA2, tmB2,
+                                    static_cast<__nv_bfloat16*>(c), sa.g, mp.a2, mp.b2,
                                     static_cast<const __nv_bfloat16*>(sa.bias));
     return L.finish(launch_err);
 }
@@ -604,37 +605,18 @@ template <int MODE>
 int launch_tf32x3(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
                   const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
                   const SharedArgs& sa, int kernel_id, cudaStream_t s) {
-    CUtensorMap tmA, tmB, tmA2, tmB2;
-    if (sa.g.S > 0) {
-        if (!make_map_2d(&tmA2, sa.a, uint64_t(a_cols), uint64_t(sa.a_rows), kTcBM, MOE_F32))
-            return MOE_ERR_UNSUPPORTED;
-        if (!make_map_3d(&tmB2, sa.w, uint64_t(a_cols), uint64_t(N), uint64_t(sa.g.S), kTfBN, MOE_F32))
-            return MOE_ERR_UNSUPPORTED;
-    }
-    if (E > 0) {
-        if (!make_map_2d(&tmA, a, uint64_t(a_cols), uint64_t(a_rows), kTcBM, MOE_F32)) return MOE_ERR_UNSUPPORTED;
-        if (!make_map_3d(&tmB, w, uint64_t(a_cols), uint64_t(N), uint64_t(E), kTfBN, MOE_F32))
-            return MOE_ERR_UNSUPPORTED;
-    } else {
-        tmA = tmA2;
-        tmB = tmB2;
-    }
-    if (sa.g.S == 0) {
-        tmA2 = tmA;
-        tmB2 = tmB;
-    }
+    FfnMaps mp;
+    if (!make_ffn_maps(mp, a, a_cols, a_rows, w, N, E, sa, kTcBM, kTfBN, MOE_F32)) return MOE_ERR_UNSUPPORTED;
     auto kern = ffn_tc_f32x3_kernel<kTfBN, kTfStages, MODE>;
     const size_t smem = TfCfg<kTfBN, kTfStages>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
-    const long long mt_ub = static_cast<long long>(ceil_div(routed_rows_ub, kTcBM)) + E +
-                            static_cast<long long>(sa.g.S) * ceil_div(sa.g.rows, kTcBM);
-    const long long tiles_ub = mt_ub * ceil_div(N, kTfBN);
+    const long long tiles_ub = ffn_tiles_ub(routed_rows_ub, E, sa, kTcBM, N, kTfBN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(kern, dim3(grid), dim3(kTfThreads), smem, s, tmA, tmB, offsets, E, N, a_cols,
-                            static_cast<const float*>(bias), row_gate, out_rows, static_cast<float*>(c), sa.g, tmA2,
-                            tmB2, static_cast<const float*>(sa.bias));
+    launch_err = launch_pdl(kern, dim3(grid), dim3(kTfThreads), smem, s, mp.a, mp.b, offsets, E, N, a_cols,
+                            static_cast<const float*>(bias), row_gate, out_rows, static_cast<float*>(c), sa.g, mp.a2,
+                            mp.b2, static_cast<const float*>(sa.bias));
     return L.finish(launch_err);
 }
 
