@@ -345,6 +345,55 @@ MOE_API int moe_shared_ffn(const void* x, int T, int d, int ff, int S,
 MOE_API int moe_combine_shared(const void* yp, const int32_t* slot_of, const float* topk_gate,
                        const void* ys, int S, int T, int k, int d, int dtype, void* out, void* stream);
 
+/* ---- end-to-end pipeline from host memory --------------------------------
+ * A pipeline runs the layer (moe_forward_ex) on a sequence of token batches
+ * that live in host memory: per step, the batch is copied host -> device,
+ * the layer runs, and the output is copied device -> host.  The two copies
+ * and the layer run on three streams the pipeline owns, over `depth` lanes
+ * (one device input, output and workspace each), so the input copy of
+ * step i+1 and the output copy of step i-1 overlap the layer of step i
+ * (PCIe is full duplex).  With MOE_PIPELINE_GRAPHS each lane's layer call
+ * is captured once into a CUDA graph at creation and replayed per step.
+ * The host loop is native: a step costs about ten CUDA runtime calls.
+ *
+ * moe_pipeline_create:
+ *   layer parameters, S, reroute_rounds, T, d, ff, E, k, capacity, dtype:
+ *     as moe_forward_ex (device pointers, caller-owned, kept by the
+ *     pipeline: they must stay valid and unchanged until destroy);
+ *   depth: lanes, 1 <= depth <= MOE_PIPELINE_MAX_DEPTH;
+ *   x_dev[depth], out_dev[depth]: device buffers [T, d] of dtype;
+ *   ws[depth]: device workspaces of ws_bytes each, ws_bytes >=
+ *     moe_forward_ex_workspace_size(T, d, ff, E, k, S, reroute_rounds,
+ *     dtype), 256-byte aligned.  All caller-owned; creation zeroes the
+ *     input buffers and runs the layer once per lane (warm-up).
+ *   flags: 0 or MOE_PIPELINE_GRAPHS;
+ *   out: receives the handle.
+ * Errors: MOE_ERR_INVALID_ARG / MOE_ERR_WORKSPACE before any CUDA call,
+ * moe_forward_ex's own argument errors from the warm-up, MOE_ERR_CUDA.
+ *
+ * moe_pipeline_run: steps i = 0..n-1 read x_host[i] (T*d elements of dtype)
+ * and write out_host[i]; returns once every output is in host memory.
+ * Host buffers should be pinned (page-locked) for the copies to overlap;
+ * pageable memory gives the same results, with staged copies.  Entries may
+ * repeat (the same buffer in several steps).  elapsed_ms (may be NULL)
+ * receives the device time from before the first copy to after the last.
+ * Not to be called concurrently on one pipeline.
+ *
+ * moe_pipeline_destroy: waits for the pipeline's streams and frees its
+ * streams, events and graphs (not the caller's buffers); NULL is a no-op. */
+#define MOE_PIPELINE_GRAPHS     1
+#define MOE_PIPELINE_MAX_DEPTH  8
+typedef struct moe_pipeline moe_pipeline;
+MOE_API int moe_pipeline_create(const void* w_router, const float* logit_bias,
+                        const void* w1, const void* b1, const void* w2, const void* b2,
+                        int S, const void* w1s, const void* b1s, const void* w2s, const void* b2s,
+                        int reroute_rounds, int T, int d, int ff, int E, int k, int capacity, int dtype,
+                        int depth, void* const* x_dev, void* const* out_dev, void* const* ws, size_t ws_bytes,
+                        int flags, moe_pipeline** out);
+MOE_API int moe_pipeline_run(moe_pipeline* p, const void* const* x_host, void* const* out_host, int n,
+                     float* elapsed_ms);
+MOE_API int moe_pipeline_destroy(moe_pipeline* p);
+
 /* ---- errors, counters, timing -------------------------------------------
  * moe_get_error: synchronises `stream`, then reads and clears the current
  * device's error word.  Returns MOE_OK, MOE_ERR_BAD_ROUTING,

@@ -28,6 +28,8 @@ MOE_BF16 = 1
 MOE_MAX_EXPERTS = 256
 MOE_MAX_TOPK = 8
 MOE_MAX_SHARED = 8
+MOE_PIPELINE_GRAPHS = 1
+MOE_PIPELINE_MAX_DEPTH = 8
 
 KERNEL_NAMES = ["router", "count", "scan", "permute", "gather", "ffn1", "ffn2", "combine", "stats", "reroute"]
 MOE_NUM_KERNELS = len(KERNEL_NAMES)
@@ -72,6 +74,10 @@ _SIGS = {
                                   ctypes.c_size_t, _P]),
     "moe_shared_ffn": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P]),
     "moe_combine_shared": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "moe_pipeline_create": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                                 _I, _P, _P, _P, ctypes.c_size_t, _I, _P]),
+    "moe_pipeline_run": (_I, [_P, _P, _P, _I, _P]),
+    "moe_pipeline_destroy": (_I, [_P]),
     "moe_get_error": (_I, [_P]),
     "moe_debug_gelu": (_I, [_P, _P, _I, _I, _P]),
     "moe_debug_wait_timeout": (_I, [ctypes.c_int64, _P]),
@@ -263,6 +269,42 @@ def moe_launch_count() -> int:
 
 def moe_timing_enable(enable: bool):
     _check(load().moe_timing_enable(1 if enable else 0), "moe_timing_enable")
+
+
+def _ptr_array(items):
+    return (ctypes.c_void_p * max(1, len(items)))(*[_ptr(t) for t in items])
+
+
+def moe_pipeline_create(w_router, logit_bias, w1, b1, w2, b2, S, w1s, b1s, w2s, b2s, reroute_rounds, T, d, ff, E,
+                        k, capacity, dtype, x_dev, out_dev, ws, ws_bytes, flags=MOE_PIPELINE_GRAPHS) -> int:
+    """Returns the pipeline handle (an integer); x_dev, out_dev and ws are
+    equal-length lists of device tensors (one per lane)."""
+    depth = len(x_dev)
+    if len(out_dev) != depth or len(ws) != depth:
+        raise ValueError("x_dev, out_dev and ws need one entry per lane")
+    handle = ctypes.c_void_p()
+    _check(load().moe_pipeline_create(_ptr(w_router), _ptr(logit_bias), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), S,
+                                      _ptr(w1s), _ptr(b1s), _ptr(w2s), _ptr(b2s), reroute_rounds, T, d, ff, E, k,
+                                      capacity, dtype, depth, _ptr_array(x_dev), _ptr_array(out_dev),
+                                      _ptr_array(ws), ws_bytes, flags, ctypes.byref(handle)),
+           "moe_pipeline_create")
+    return handle.value
+
+
+def moe_pipeline_run(handle: int, x_host, out_host) -> float:
+    """Runs len(x_host) steps (host tensors in, host tensors out); returns the
+    device time in milliseconds from before the first copy to after the last."""
+    if len(x_host) != len(out_host):
+        raise ValueError("one output buffer per input batch")
+    ms = ctypes.c_float(0.0)
+    _check(load().moe_pipeline_run(handle, _ptr_array(x_host), _ptr_array(out_host), len(x_host),
+                                   ctypes.byref(ms)),
+           "moe_pipeline_run")
+    return ms.value
+
+
+def moe_pipeline_destroy(handle: int):
+    _check(load().moe_pipeline_destroy(handle), "moe_pipeline_destroy")
 
 
 def moe_timing_read():

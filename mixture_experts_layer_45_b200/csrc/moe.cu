@@ -2,8 +2,10 @@
 //
 // Every entry point validates its arguments before touching the GPU, then
 // enqueues kernels on the caller's stream.  Nothing here synchronises the
-// host except moe_get_error and moe_timing_read, and nothing allocates
-// device memory: scratch comes from the caller's workspace.
+// host except moe_get_error, moe_timing_read and the pipeline's run and
+// destroy, and nothing allocates device memory: scratch comes from the
+// caller's workspace.  The pipeline (pipeline.cuh) owns only streams,
+// events and graphs.
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
@@ -1276,3 +1278,5 @@ int moe_timing_read(double* ms_per_kernel, int64_t* launches_per_kernel) {
 }
 
 }  // extern "C"
+
+#include "pipeline.cuh"

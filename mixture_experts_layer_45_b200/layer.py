@@ -156,79 +156,57 @@ class MoELayer:
 
 
 class HostPipeline:
-    """End-to-end forward passes from pinned host memory, pipelined.
+    """End-to-end forward passes from pinned host memory, pipelined
+    (libmoe's native pipeline, moe_pipeline_*).
 
     Each step copies its tokens host -> device, runs the layer and copies
     the output device -> host.  The copies run on their own streams and the
     layer on a third, with `depth` lanes (device input / output buffers and
     a workspace each), so the input copy of step i+1 and the output copy of
     step i-1 overlap the layer of step i (PCIe is full duplex).  Every
-    step's copies are still issued and completed.
-
-    With `graphs` (default) each lane's layer call is captured once into a
-    CUDA graph and replayed, so a step costs the host a few calls instead of
-    the layer's launch sequence; the layer calls of all lanes stay on one
-    stream, one after another.
+    step's copies are still issued and completed.  With `graphs` (default)
+    each lane's layer call is captured once into a CUDA graph and replayed;
+    the per-step host loop runs in the library.
     """
 
     def __init__(self, layer: MoELayer, T: int, depth: int = 3, graphs: bool = True):
-        dev = layer.p.w1.device
-        dt = TORCH_DTYPE[layer.p.dtype]
+        p = layer.p
+        dev = p.w1.device
+        dt = TORCH_DTYPE[p.dtype]
         self.layer = layer
         self.depth = depth
-        self.s_in = torch.cuda.Stream(device=dev)
-        self.s_run = torch.cuda.Stream(device=dev)
-        self.s_out = torch.cuda.Stream(device=dev)
-        self.x_dev = [torch.empty((T, layer.p.d), dtype=dt, device=dev) for _ in range(depth)]
-        self.out_dev = [torch.empty((T, layer.p.d), dtype=dt, device=dev) for _ in range(depth)]
-        # one layer (own workspace) per lane, sharing the parameters
-        self.lanes = [MoELayer(layer.p, layer.k, layer.capacity, layer.reroute) for _ in range(depth)]
-        for ln in self.lanes:
-            ln.workspace(T)
-        self.in_done = [torch.cuda.Event() for _ in range(depth)]
-        self.run_done = [torch.cuda.Event() for _ in range(depth)]
-        self.out_done = [torch.cuda.Event() for _ in range(depth)]
-        self.graphs = None
-        if graphs:
-            self.graphs = []
-            torch.cuda.synchronize(dev)
-            for b in range(depth):
-                self.lanes[b].forward(self.x_dev[b], out=self.out_dev[b])      # warm the launch path
-                torch.cuda.synchronize(dev)
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    self.lanes[b].forward(self.x_dev[b], out=self.out_dev[b])
-                self.graphs.append(g)
-            torch.cuda.synchronize(dev)
+        self.T = T
+        self.x_dev = [torch.empty((T, p.d), dtype=dt, device=dev) for _ in range(depth)]
+        self.out_dev = [torch.empty((T, p.d), dtype=dt, device=dev) for _ in range(depth)]
+        n = _lib.moe_forward_ex_workspace_size(T, p.d, p.ff, p.E, layer.k, p.S, layer.reroute, p.dtype)
+        if n == 0:
+            raise ValueError("invalid layer sizes")
+        self.ws = [torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(depth)]
+        self.handle = None
+        with torch.cuda.device(dev):
+            self.handle = _lib.moe_pipeline_create(
+                p.w_router, p.logit_bias, p.w1, p.b1, p.w2, p.b2, p.S, p.shared_w1, p.shared_b1, p.shared_w2,
+                p.shared_b2, layer.reroute, T, p.d, p.ff, p.E, layer.k, layer.capacity, p.dtype, self.x_dev,
+                self.out_dev, self.ws, n, _lib.MOE_PIPELINE_GRAPHS if graphs else 0)
 
-    def run(self, x_hosts, out_hosts, start_event=None, end_event=None):
-        """x_hosts[i] (pinned) -> layer -> out_hosts[i] (pinned), for every i."""
-        if start_event is not None:
-            start_event.record(self.s_in)
-            self.s_run.wait_event(start_event)
-            self.s_out.wait_event(start_event)
-        for i, (xh, oh) in enumerate(zip(x_hosts, out_hosts)):
-            b = i % self.depth
-            self.s_in.wait_event(self.run_done[b])          # x_dev[b] no longer read
-            with torch.cuda.stream(self.s_in):
-                self.x_dev[b].copy_(xh, non_blocking=True)
-            self.in_done[b].record(self.s_in)
-            self.s_run.wait_event(self.in_done[b])
-            self.s_run.wait_event(self.out_done[b])         # out_dev[b] already copied out
-            if self.graphs is not None:
-                with torch.cuda.stream(self.s_run):
-                    self.graphs[b].replay()
-            else:
-                self.lanes[b].forward(self.x_dev[b], out=self.out_dev[b], stream=self.s_run)
-            self.run_done[b].record(self.s_run)
-            self.s_out.wait_event(self.run_done[b])
-            with torch.cuda.stream(self.s_out):
-                oh.copy_(self.out_dev[b], non_blocking=True)
-            self.out_done[b].record(self.s_out)
-        if end_event is not None:
-            self.s_run.wait_stream(self.s_out)
-            self.s_in.wait_stream(self.s_out)
-            end_event.record(self.s_out)
-        self.s_out.synchronize()
-        self.s_in.synchronize()
-        self.s_run.synchronize()
+    def run(self, x_hosts, out_hosts) -> float:
+        """x_hosts[i] (pinned) -> layer -> out_hosts[i] (pinned), for every i;
+        returns the device milliseconds from the first copy in to the last
+        copy out."""
+        for xh, oh in zip(x_hosts, out_hosts):
+            if xh.shape != (self.T, self.layer.p.d) or oh.shape != xh.shape or xh.dtype != self.x_dev[0].dtype \
+                    or oh.dtype != xh.dtype or not (xh.is_contiguous() and oh.is_contiguous()) \
+                    or xh.is_cuda or oh.is_cuda:
+                raise ValueError("host batches must be contiguous CPU tensors of the pipeline's shape and dtype")
+        return _lib.moe_pipeline_run(self.handle, list(x_hosts), list(out_hosts))
+
+    def close(self):
+        if self.handle is not None:
+            _lib.moe_pipeline_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -220,3 +220,38 @@ def test_wait_timeout_probe_checks_its_limit(lib):
     assert lib.moe_debug_wait_timeout(0, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_wait_timeout(-5, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_wait_timeout(3_000_000_000, None) == _lib.MOE_ERR_INVALID_ARG   # above the 2 s cap
+
+
+def test_pipeline_checks(lib):
+    """moe_pipeline_create / run / destroy reject bad arguments before any CUDA call."""
+    T, d, ff, E, k = 256, 64, 128, 8, 2
+    need = lib.moe_forward_ex_workspace_size(T, d, ff, E, k, 0, 0, _lib.MOE_BF16)
+    arr = lambda *v: (ctypes.c_void_p * len(v))(*v)
+    handle = ctypes.c_void_p(FAKE)
+
+    def create(depth=2, x=None, o=None, ws=None, ws_bytes=need, flags=_lib.MOE_PIPELINE_GRAPHS, out=True, T=T,
+               E=E):
+        x = arr(*([FAKE] * depth)) if x is None else x
+        o = arr(*([FAKE] * depth)) if o is None else o
+        ws = arr(*([FAKE] * depth)) if ws is None else ws
+        return lib.moe_pipeline_create(FAKE, None, FAKE, FAKE, FAKE, FAKE, 0, None, None, None, None, 0, T, d, ff,
+                                       E, k, -1, _lib.MOE_BF16, depth, x, o, ws, ws_bytes, flags,
+                                       ctypes.byref(handle) if out else None)
+
+    assert create(out=False) == _lib.MOE_ERR_INVALID_ARG
+    assert handle.value == FAKE                                          # untouched without an out pointer
+    assert create(depth=0) == _lib.MOE_ERR_INVALID_ARG
+    assert create(depth=_lib.MOE_PIPELINE_MAX_DEPTH + 1) == _lib.MOE_ERR_INVALID_ARG
+    assert handle.value is None                                          # cleared on every other failure
+    assert create(flags=2) == _lib.MOE_ERR_INVALID_ARG
+    assert create(T=0) == _lib.MOE_ERR_INVALID_ARG
+    assert create(E=_lib.MOE_MAX_EXPERTS + 1) == _lib.MOE_ERR_INVALID_ARG           # sizes the layer rejects
+    assert create(x=arr(FAKE, None)) == _lib.MOE_ERR_INVALID_ARG
+    assert create(o=arr(FAKE, MISALIGNED)) == _lib.MOE_ERR_INVALID_ARG
+    assert create(ws_bytes=need - 1) == _lib.MOE_ERR_WORKSPACE
+    assert create(ws=arr(FAKE, FAKE + 16)) == _lib.MOE_ERR_WORKSPACE    # not 256-byte aligned
+    assert lib.moe_pipeline_run(None, None, None, 0, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_run(FAKE, None, None, -1, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_run(FAKE, None, None, 2, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_run(FAKE, arr(FAKE, None), arr(FAKE, FAKE), 2, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_destroy(None) == _lib.MOE_OK

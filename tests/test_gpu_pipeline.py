@@ -1,10 +1,10 @@
 """End-to-end pipeline and CUDA-graph replay of the layer on the GPU.
 
-The pipelined host path (HostPipeline: pinned host buffers, three streams,
-one CUDA graph per lane) must return exactly what the device forward
-returns, and a captured forward, replayed on new inputs, must equal the
-eager call bit for bit (the grouped FFN's split tiles publish and clear
-their flags on every replay).
+The pipelined host path (the library's moe_pipeline_*: pinned host
+buffers, three streams, one CUDA graph per lane, a native host loop) must
+return exactly what the device forward returns, with and without graphs,
+for any number of steps and lanes; and a captured forward, replayed on new
+inputs, must equal the eager call bit for bit.
 """
 import numpy as np
 import pytest
@@ -35,8 +35,9 @@ def scaled_inputs(x, n):
     return [(x.float() * (0.5 + 0.25 * i)).to(x.dtype) for i in range(n)]
 
 
-@pytest.mark.parametrize("shared,reroute", [(0, 0), (1, 1)])
-def test_host_pipeline_matches_device_forward(shared, reroute):
+@pytest.mark.parametrize("shared,reroute,depth,graphs", [(0, 0, 3, True), (1, 1, 3, True), (0, 0, 2, False),
+                                                         (0, 1, 1, True)])
+def test_host_pipeline_matches_device_forward(shared, reroute, depth, graphs):
     w = wl.workload("switch-top1", dtype="bf16", cf=1.0, shared=shared)
     inp = wl.draw_inputs(w)
     params = MoEParams.from_arrays(inp, _lib.MOE_BF16, DEV)
@@ -45,12 +46,36 @@ def test_host_pipeline_matches_device_forward(shared, reroute):
     xs = scaled_inputs(x, 5)
     x_hosts = [xi.cpu().pin_memory() for xi in xs]
     out_hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in xs]
-    pipe = HostPipeline(layer, w.T)
-    pipe.run(x_hosts, out_hosts)
+    pipe = HostPipeline(layer, w.T, depth=depth, graphs=graphs)
+    ms = pipe.run(x_hosts, out_hosts)
+    assert ms > 0.0
     assert _lib.moe_get_error() == _lib.MOE_OK
     for xi, oh in zip(xs, out_hosts):
         ref = layer.forward(xi).cpu()
         assert torch.equal(bits(oh), bits(ref))
+    # a second run on the same pipeline, buffers repeated across steps, pageable output
+    outs2 = [torch.empty(x.shape, dtype=x.dtype) for _ in range(2)]
+    pipe.run([x_hosts[4], x_hosts[0], x_hosts[4]], [outs2[0], outs2[1], outs2[0]])
+    assert torch.equal(bits(outs2[0]), bits(out_hosts[4])) and torch.equal(bits(outs2[1]), bits(out_hosts[0]))
+    assert pipe.run([], []) >= 0.0
+    pipe.close()
+
+
+def test_host_pipeline_f32_and_ragged_tokens():
+    T, d, ff, E, k = 1000, 72, 200, 5, 2
+    inp = wl.draw_custom(4, T=T, d=d, ff=ff, E=E, dtype="f32", router_std=0.5, shared=1)
+    params = MoEParams.from_arrays(inp, _lib.MOE_F32, DEV)
+    layer = MoELayer(params, k, 300, reroute=1)
+    x = to_device(inp["x"], _lib.MOE_F32, DEV)
+    xs = scaled_inputs(x, 4)
+    x_hosts = [xi.cpu().pin_memory() for xi in xs]
+    out_hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in xs]
+    pipe = HostPipeline(layer, T, depth=3)
+    pipe.run(x_hosts, out_hosts)
+    assert _lib.moe_get_error() == _lib.MOE_OK
+    for xi, oh in zip(xs, out_hosts):
+        assert torch.equal(oh, layer.forward(xi).cpu())
+    pipe.close()
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
