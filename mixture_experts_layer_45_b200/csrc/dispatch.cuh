@@ -349,50 +349,63 @@ __device__ __forceinline__ int chunk_stable_ranks(const int32_t* __restrict__ id
 }
 
 // Gather of a chunk's grouped rows: xp[slot] = x[token] for every kept
-// assignment (slot_s[i] >= 0), and, with out_zero_dropped, zero output rows
-// for dropped ones (k == 1 direct output).  The chunk's rows are split over
-// the gridDim.y CTAs of the chunk, flattened into 16-byte pieces with eight
-// independent loads in flight per thread.
+// assignment (slot_s[i] >= 0, i = the assignment's index in the chunk), and,
+// with out_zero_dropped, a zero output row for every token with no kept
+// slot (k == 1 direct output).  The walk is over the chunk's tokens, not
+// its assignments, so a token's row is read once and stored to each of its
+// kept slots.  The chunk's tokens are split over the gridDim.y CTAs of the
+// chunk (CTA y takes tokens y, y + Y, ...), flattened into 16-byte pieces
+// with eight independent loads in flight per thread.  a0 and na are
+// multiples of k (whole tokens).
 __device__ __forceinline__ void gather_chunk_rows(const int* slot_s, int a0, int na, int k,
                                                   const uint8_t* __restrict__ x, int row_bytes,
                                                   uint8_t* __restrict__ xp, uint8_t* __restrict__ out_zero_dropped) {
     const int tid = threadIdx.x;
     const int vecs = row_bytes >> 4;
     const int Y = int(gridDim.y), y = int(blockIdx.y);
-    const int my_rows = (na - y + Y - 1) / Y;
-    const int pieces = my_rows * vecs;
+    const int t0 = a0 / k;
+    const int nt = na / k;
+    const int my_tokens = (nt - y + Y - 1) / Y;
+    const int pieces = my_tokens * vecs;
     constexpr int U = 8;
     for (int p0 = tid; p0 < pieces; p0 += kFwdThreads * U) {
         uint4 val[U];
-        int row[U], vv[U], kind[U];   // kind 1: xp row, 2: zeroed output row of a dropped token
+        int tl[U], vv[U], kind[U];   // kind 1: store to the token's kept slots, 2: zero its output row
+        int first[U];                // the token's first slot (its only one for k = 1)
 #pragma unroll
         for (int j = 0; j < U; ++j) {
             const int pc = p0 + j * kFwdThreads;
             kind[j] = 0;
-            row[j] = 0;
+            tl[j] = 0;
             vv[j] = 0;
+            first[j] = -1;
             if (pc < pieces) {
                 const int il = pc / vecs;
                 vv[j] = pc - il * vecs;
-                const int i = y + Y * il;
-                const int slot = slot_s[i];
-                const int t = (a0 + i) / k;
-                if (slot >= 0) {
-                    val[j] = __ldg(reinterpret_cast<const uint4*>(x + size_t(t) * row_bytes) + vv[j]);
-                    row[j] = slot;
+                tl[j] = y + Y * il;
+                first[j] = slot_s[tl[j] * k];
+                bool kept = first[j] >= 0;
+                for (int c = 1; c < k; ++c) kept |= slot_s[tl[j] * k + c] >= 0;
+                if (kept) {
+                    val[j] = __ldg(reinterpret_cast<const uint4*>(x + size_t(t0 + tl[j]) * row_bytes) + vv[j]);
                     kind[j] = 1;
                 } else if (out_zero_dropped != nullptr) {
                     val[j] = make_uint4(0u, 0u, 0u, 0u);
-                    row[j] = t;
                     kind[j] = 2;
                 }
             }
         }
 #pragma unroll
         for (int j = 0; j < U; ++j) {
-            if (kind[j] == 1) reinterpret_cast<uint4*>(xp + size_t(row[j]) * row_bytes)[vv[j]] = val[j];
-            else if (kind[j] == 2)
-                reinterpret_cast<uint4*>(out_zero_dropped + size_t(row[j]) * row_bytes)[vv[j]] = val[j];
+            if (kind[j] == 1) {
+                if (first[j] >= 0) reinterpret_cast<uint4*>(xp + size_t(first[j]) * row_bytes)[vv[j]] = val[j];
+                for (int c = 1; c < k; ++c) {
+                    const int slot = slot_s[tl[j] * k + c];
+                    if (slot >= 0) reinterpret_cast<uint4*>(xp + size_t(slot) * row_bytes)[vv[j]] = val[j];
+                }
+            } else if (kind[j] == 2) {
+                reinterpret_cast<uint4*>(out_zero_dropped + size_t(t0 + tl[j]) * row_bytes)[vv[j]] = val[j];
+            }
         }
     }
 }
@@ -891,10 +904,13 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
     *reinterpret_cast<uint4*>(p) = u;
 }
 
-// One warp per token; each lane handles 16-byte pieces of the row, four at a
-// time, so 4 * k independent loads are in flight before the adds.  With
-// S > 0 shared experts, ys [S, Tn, d] holds their outputs and each adds its
-// row of token t with weight 1 after the routed slots.
+// One warp per token, the warps striding over the tokens (the grid is what
+// fits on the GPU at once); each lane handles 16-byte pieces of the row,
+// four at a time, so 4 * k independent loads are in flight before the adds.
+// Lane j < k holds slot j's row and gate, loaded one token ahead so the
+// next token's indices arrive while this token's rows load.  With S > 0
+// shared experts, ys [S, Tn, d] holds their outputs and each adds its row
+// of token t with weight 1 after the routed slots.
 template <typename T>
 __global__ void __launch_bounds__(256)
 combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
@@ -906,14 +922,27 @@ combine_kernel(const T* __restrict__ yp, const int32_t* __restrict__ slot_of, co
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int lane = threadIdx.x & 31;
     const int pieces = d / EPV;
-    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < Tn; t += warps_total) {
+    auto fetch = [&](int tt, int& sl, float& wv) {
+        sl = -1;
+        wv = 1.f;
+        if (tt < Tn && lane < k) {
+            sl = slot_of[size_t(tt) * k + lane];
+            if (gate != nullptr) wv = gate[size_t(tt) * k + lane];
+        }
+    };
+    int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    int next_slot;
+    float next_w;
+    fetch(t, next_slot, next_w);
+    for (; t < Tn; t += warps_total) {
         int slot[MOE_MAX_TOPK];
         float w[MOE_MAX_TOPK];
 #pragma unroll
         for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-            slot[j] = (j < k) ? slot_of[size_t(t) * k + j] : -1;
-            w[j] = (j < k && gate != nullptr) ? gate[size_t(t) * k + j] : 1.f;
+            slot[j] = __shfl_sync(0xffffffffu, next_slot, j);
+            w[j] = __shfl_sync(0xffffffffu, next_w, j);
         }
+        fetch(t + warps_total, next_slot, next_w);
         for (int c0 = lane; c0 < pieces; c0 += 32 * U) {
             float acc[U][EPV];
 #pragma unroll

@@ -384,6 +384,29 @@ bool set_smem_attr(K kernel, size_t bytes) {
     return true;
 }
 
+// CTAs of `kernel` (`threads` per CTA, no dynamic shared memory) that fit on
+// one SM at once; cached per (kernel, device); 1 if the query fails.
+std::mutex g_occ_mu;
+std::vector<std::pair<std::pair<const void*, int>, int>> g_occ_done;
+
+template <typename K>
+int resident_blocks(K kernel, int threads) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    const void* key = reinterpret_cast<const void*>(kernel);
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    for (const auto& kd : g_occ_done)
+        if (kd.first.first == key && kd.first.second == dev) return kd.second;
+    uniform_carveout(key);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = 1;
+    }
+    g_occ_done.push_back({{key, dev}, n});
+    return n;
+}
+
 // ---------------------------------------------------------------------------
 // step launchers (arguments already validated)
 // ---------------------------------------------------------------------------
@@ -797,7 +820,10 @@ int run_reroute_dispatch(const int32_t* idx, const float* gate, const int32_t* f
 // ys (nullable when S == 0): [S, T, d] shared-expert outputs added with weight 1
 int run_combine(const void* yp, const int32_t* slot_of, const float* gate, int T, int k, int d, int dtype, void* out,
                 const void* ys, int S, cudaStream_t s) {
-    const int grid = std::max(1, std::min(ceil_div(T, 8), num_sms() * 16));
+    // warps stride over the tokens: no more CTAs than fit on the GPU at once
+    const int per_sm = dtype == MOE_BF16 ? resident_blocks(combine_kernel<__nv_bfloat16>, 256)
+                                         : resident_blocks(combine_kernel<float>, 256);
+    const int grid = std::max(1, std::min(ceil_div(T, 8), num_sms() * per_sm));
     Launch L(MOE_KERNEL_COMBINE, s);
     cudaError_t launch_err;
     if (dtype == MOE_BF16)
