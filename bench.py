@@ -299,11 +299,31 @@ def algorithmic_bytes(kernel, w, R, E_active, es):
                 + R * 4)
     if kernel == "router":
         return T * d * es + E * d * es + T * k * 8 + E * 4
+    if kernel == "permute":
+        # the dispatch: x read once per token, xp written once per kept row,
+        # the routing arrays (idx, gate, slot_of) and perm / row_gate; with a
+        # direct top-1 output it also zeroes the dropped tokens' output rows
+        direct = k == 1 and S == 0
+        return T * d * es + R * d * es + T * k * 12 + R * 8 + ((T - R) * d * es if direct else 0)
     if kernel == "gather":
         return 2 * R * d * es + R * 4
     if kernel == "combine":
         return (R + S * T) * d * es + T * d * es + T * k * 4
     return None
+
+
+def add_memory_rooflines(kernels, w, R, E_active, es, hbm_gbs):
+    """GB/s and fraction of the HBM copy peak of the memory-bound kernels
+    (router, dispatch, combine), from their algorithmic bytes per launch and
+    their event-timed launch durations (launch gaps included)."""
+    for name in ("router", "permute", "combine"):
+        kn = kernels.get(name)
+        nbytes = algorithmic_bytes(name, w, R, E_active, es)
+        if kn is None or nbytes is None or not kn["ms_per_launch"]:
+            continue
+        gbs = nbytes / (kn["ms_per_launch"] / 1000.0) / 1e9
+        kn.update({"algorithmic_bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm_gbs})
+    return kernels
 
 
 def copy_bandwidth(x_host, out_host, x_dev, out_dev, reps: int = 20):
@@ -471,6 +491,7 @@ def run_ours(args):
     for name, (ms, n) in kt.items():
         if n:
             kernels[name] = {"launches": n, "ms_per_launch": ms / n, "share": ms / tot_k if tot_k else None}
+    add_memory_rooflines(kernels, w, R, E_active, es, peaks["hbm_gbs"])
     modelled = [kn for kn in kernels if algorithmic_bytes(kn, w, R, E_active, es) is not None]
     dom = max(modelled, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
     ffn_ms = sum(kernels[k]["ms_per_launch"] for k in ("ffn1", "ffn2") if k in kernels)
