@@ -32,9 +32,10 @@ host once each.  Shared experts and overflow rerouting are not part of
 this path.
 
 A second form, `ShardedExpertsMoE`, splits every expert instead of the
-set of experts (the MoEShard pages: "row- and column-wise decomposition of
-expert matrices", each GPU taking an equal share of every expert whatever
-the routing skew, no token dropped for balance).  Rank g holds the hidden
+set of experts (the MoEShard pages, abstract: each expert's weight matrices
+cut by rows and by columns across the GPUs, so that every GPU does an
+equal share of every expert whatever the routing skew and no token is
+dropped for balance).  Rank g holds the hidden
 units [g*ff/G, (g+1)*ff/G) of every expert: those columns of fc1 (rows of
 W1 and b1) and the matching rows of fc2 (columns of W2); b2 lives on rank
 0.  Every rank routes and dispatches the same replicated batch, runs the
