@@ -72,3 +72,28 @@ def test_traffic_is_read_for_the_bench_workload():
     w = wl.workload("switch-top1")
     assert bench.committed_traffic("ffn1", bench.workload_tag(w)) == 164175104.0
     assert bench.committed_traffic("ffn1", "no-such-workload") is None
+
+
+def test_defaults_meet_the_run_contract():
+    a = bench.parse_args([])
+    assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1 and a.impl == "ours"
+    assert bench.get_workload(a).name == "switch-top1"
+
+
+def test_reference_arm_line(capsys, monkeypatch):
+    """`--impl reference` times the oracle on the host cores and prints the
+    contract's line; under a multi-rank launch only rank 0 does so."""
+    import json
+    monkeypatch.setenv("RANK", "0")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "tokens/s"
+    assert line["value"] > 0 and line["higher_is_better"] is True and line["steps"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"].startswith("switch-top1 T=4096")
+    monkeypatch.setenv("RANK", "1")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    assert capsys.readouterr().out == ""
