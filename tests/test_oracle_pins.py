@@ -161,6 +161,61 @@ def test_drop_rate_closed_form_and_monotone():
     assert drops[1.0] > 0        # the untrained router overflows some expert at cf 1.0
 
 
+# A hand-built top-2 routing of T = 10 tokens over E = 4 experts.  Counting
+# by hand: expert 0 is in rows 0-7 (8), expert 1 in rows 0, 3, 5, 8, 9 (5),
+# expert 2 in rows 1, 4, 7, 8 (4), expert 3 in rows 2, 6, 9 (3); 20 = T*k.
+_HAND_IDX = np.array([[0, 1], [0, 2], [0, 3], [0, 1], [0, 2], [0, 1], [0, 3], [0, 2], [1, 2], [3, 1]])
+_HAND_COUNTS = [8, 5, 4, 3]
+
+
+def check_imbalance_closed_form():
+    """The notebook's imbalance ratio ("Capacity factor") is the largest
+    count over the balanced load T*k/E.  Hand-worked: T*k/E = 10*2/4 = 5,
+    so 8/5 = 1.6 (a T/E denominator would give 3.2).  Round-robin routing
+    loads every expert with exactly T*k/E assignments: 1.0."""
+    np.testing.assert_array_equal(moe_ref.token_count_per_expert(_HAND_IDX, 4), _HAND_COUNTS)
+    assert moe_ref.imbalance(np.array(_HAND_COUNTS), 10, 2, 4) == pytest.approx(1.6, abs=1e-15)
+    st = moe_ref.layer_stats(_HAND_IDX, np.full((10, 4), 0.25), 4, -1)
+    assert st["imbalance"] == pytest.approx(1.6, abs=1e-15) and st["max_count"] == 8
+    for T, k, E in ((64, 2, 8), (96, 1, 32), (40, 2, 4)):
+        rr = (np.arange(T * k) % E).reshape(T, k)
+        assert moe_ref.imbalance(moe_ref.token_count_per_expert(rr, E), T, k, E) == 1.0
+
+
+def test_imbalance_closed_form():
+    check_imbalance_closed_form()
+
+
+def check_layer_stats_drops_are_capacity_check():
+    """Without rerouting, the statistics' drop count and rate are the
+    notebook's capacity_check ("Capacity factor"): sum(max(counts - cap, 0))
+    and that over counts.sum() = T*k.  Hand-worked on _HAND_IDX: cap 4 drops
+    (8-4) + (5-4) = 5 of 20 (0.25), cap 5 drops 3 (0.15), cap 2 drops
+    6+3+2+1 = 12 (0.6), no limit drops nothing."""
+    gates = np.full((10, 4), 0.25)
+    for cap, dropped in ((4, 5), (5, 3), (2, 12), (8, 0), (0, 20), (-1, 0)):
+        st = moe_ref.layer_stats(_HAND_IDX, gates, 4, cap)
+        closed = sum(max(c - cap, 0) for c in _HAND_COUNTS) if cap >= 0 else 0
+        assert closed == dropped
+        assert st["dropped"] == dropped and st["rows_kept"] == 20 - dropped
+        assert st["drop_rate"] == pytest.approx(dropped / 20, abs=1e-15)
+        assert st["drop_rate"] == pytest.approx(moe_ref.drop_rate(_HAND_COUNTS, cap), abs=1e-15)
+    # and on a seeded routing, against the dispatch's own drop mask
+    w = wl.workload("switch-top1", dtype="f32")
+    inp = wl.draw_router_inputs(w)
+    r = moe_ref.route(inp["x"], inp["w_router"], w.k)
+    for cf in (1.0, 1.5):
+        cap = moe_ref.capacity(w.T, w.k, w.E, cf)
+        st = moe_ref.layer_stats(r["topk_idx"], r["gates"], w.E, cap)
+        counts = moe_ref.token_count_per_expert(r["topk_idx"], w.E)
+        assert st["drop_rate"] == pytest.approx(moe_ref.drop_rate(counts, cap), abs=1e-15)
+        assert st["dropped"] == int(moe_ref.dispatch(r["topk_idx"], w.E, cap)["drop_mask"].sum())
+
+
+def test_layer_stats_drops_are_capacity_check():
+    check_layer_stats_drops_are_capacity_check()
+
+
 # ---------------------------------------------------------------------------
 # GELU, expert FFN, combine
 # ---------------------------------------------------------------------------
@@ -595,11 +650,28 @@ def _offers_always_first_fallback(ranked_idx, served, k, r):
     return _ORIG_OFFERS(ranked_idx, served, k, 1)
 
 
+def _imbalance_over_T(counts, T, k, E):
+    return float(np.max(counts) / (T / E))
+
+
+def _layer_stats_drop_rate_over_T(topk_idx, gates, E, cap, slot_of=None):
+    st = _ORIG_LAYER_STATS(topk_idx, gates, E, cap, slot_of)
+    st["drop_rate"] = st["dropped"] / np.asarray(topk_idx).shape[0]
+    return st
+
+
+def _layer_stats_dropped_counts_kept(topk_idx, gates, E, cap, slot_of=None):
+    st = _ORIG_LAYER_STATS(topk_idx, gates, E, cap, slot_of)
+    st["dropped"] = st["rows_kept"]
+    return st
+
+
 _ORIG_ROUTE = moe_ref.route
 _ORIG_DISPATCH = moe_ref.dispatch
 _ORIG_AUX = moe_ref.switch_aux_loss
 _ORIG_SHARED_OUT = moe_ref.shared_expert_outputs
 _ORIG_OFFERS = moe_ref.reroute_offers
+_ORIG_LAYER_STATS = moe_ref.layer_stats
 
 MUTATIONS = {
     "tanh-gelu": ("gelu", _tanh_gelu, lambda: check_gelu(moe_ref.gelu)),
@@ -624,6 +696,11 @@ MUTATIONS = {
     "reroute-offers-reversed": ("reroute_offers", _offers_reverse_token_order, check_reroute_hand_example_top1),
     "reroute-no-deeper-fallback": ("reroute_offers", _offers_always_first_fallback,
                                    check_reroute_hand_example_top1),
+    "imbalance-over-T-not-Tk": ("imbalance", _imbalance_over_T, check_imbalance_closed_form),
+    "layer-drop-rate-over-T": ("layer_stats", _layer_stats_drop_rate_over_T,
+                               check_layer_stats_drops_are_capacity_check),
+    "layer-dropped-is-kept": ("layer_stats", _layer_stats_dropped_counts_kept,
+                              check_layer_stats_drops_are_capacity_check),
 }
 
 
