@@ -7,9 +7,10 @@
 One step = one whole forward pass of the layer (router -> dispatch ->
 grouped expert FFN -> combine -> statistics) over one batch of the
 workload's synthetic tokens, inputs resident in HBM.  The default workload
-is the Switch-style top-1 layer (T=4096, d=768, ff=3072, 32 experts, bf16,
-capacity factor 1.0).  L2 is flushed (a 256 MiB write) before every step,
-outside the per-step device timing.
+is the largest single-GPU one, the large top-2 layer (T=8192, d=4096,
+ff=14336, 8 experts, bf16, no capacity limit), where the expert FFN is
+bound by the tensor cores.  L2 is flushed (a 256 MiB write) before every
+step, outside the per-step device timing.
 
 With N > 1 (torchrun, one process per GPU) every rank runs an independent
 replica of the same layer: there is no data-path collective.  The timed
@@ -48,7 +49,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="switch-top1")
+    ap.add_argument("--workload", default="large-top2")
     ap.add_argument("--dtype", default=None, help="bf16 or f32 (switch-top1 only; default bf16)")
     ap.add_argument("--cf", type=float, default=None, help="capacity factor (switch-top1: 1.0 or 1.5)")
     ap.add_argument("--shared", type=int, default=0, help="shared always-on experts added to the workload")
@@ -57,6 +58,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget for the oracle baseline")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (profiling runs: keeps device memory to one layer)")
     return ap.parse_args(argv)
 
 
@@ -196,21 +199,38 @@ def blas_threads():
         return None
 
 
-def oracle_sample_inputs(w, sample_T):
+# float64 work of one oracle pass over a sample, kept near this many flops so
+# a pass takes about a second on a host's cores whatever the workload
+ORACLE_FLOPS_PER_PASS = 32e9
+
+
+def oracle_sample_tokens(w, most: int) -> int:
+    """Tokens of the oracle's sample: at most `most`, fewer where each token
+    costs more (the expert FFN is 4*k*d*ff flops per token), at least 16;
+    a power of two."""
+    per_token = 4.0 * (w.k + w.shared) * w.d * w.ff
+    n = max(16, min(most, w.T, int(ORACLE_FLOPS_PER_PASS // per_token)))
+    return 1 << (n.bit_length() - 1)
+
+
+def oracle_sample_inputs(w, sample_T, drawn=None):
     """A bounded sample of the workload: its first sample_T tokens (the same
-    seeded draws), with the capacity recomputed for the sample's size."""
+    seeded draws), with the capacity recomputed for the sample's size.  The
+    arrays are widened to float64 once here, outside any timing (the oracle
+    computes in float64; bf16 and fp32 values are exact in it)."""
+    import numpy as np
     from mixture_experts_layer_45_b200 import workloads as wl
-    inp = wl.draw_inputs(w)
-    inp = dict(inp)
+    inp = dict(wl.draw_inputs(w) if drawn is None else drawn)
     inp["x"] = inp["x"][:sample_T]
+    inp = {key: (None if v is None else np.asarray(v, np.float64)) for key, v in inp.items()}
     from oracle import moe_ref
     cap = moe_ref.capacity(sample_T, w.k, w.E, w.cf)
     return inp, cap
 
 
-def time_oracle(w, seconds: float, sample_T: int):
+def time_oracle(w, seconds: float, sample_T: int, drawn=None):
     from oracle import moe_ref
-    inp, cap = oracle_sample_inputs(w, sample_T)
+    inp, cap = oracle_sample_inputs(w, sample_T, drawn)
     moe_ref.moe_layer(inp, w.k, cap)          # warm-up
     t0 = time.perf_counter()
     n = 0
@@ -223,14 +243,15 @@ def time_oracle(w, seconds: float, sample_T: int):
     return n * sample_T / dt, n, dt
 
 
-def cpu_baseline(w, seconds: float):
-    sample_T = min(w.T, 1024)
-    tps, n, dt = time_oracle(w, seconds, sample_T)
+def cpu_baseline(w, seconds: float, drawn=None):
+    sample_T = oracle_sample_tokens(w, 1024)
+    tps, n, dt = time_oracle(w, seconds, sample_T, drawn)
     cores = len(os.sched_getaffinity(0))
     return {"value": tps, "unit": "tokens/s", "cores": cores, "blas_threads": blas_threads(),
             "kind": "oracle",
             "sample": f"{n} float64 oracle passes over the first {sample_T} tokens of {workload_label(w)} "
-                      f"(capacity recomputed for the sample), {dt:.1f} s wall"}
+                      f"(capacity recomputed for the sample; inputs widened to float64 before timing), "
+                      f"{dt:.1f} s wall"}
 
 
 def run_reference(args):
@@ -239,7 +260,7 @@ def run_reference(args):
         return 0
     w = get_workload(args)
     from oracle import moe_ref
-    sample_T = min(w.T, 512)
+    sample_T = oracle_sample_tokens(w, 512)
     inp, cap = oracle_sample_inputs(w, sample_T)
     for _ in range(args.warmup):
         moe_ref.moe_layer(inp, w.k, cap)
@@ -355,6 +376,46 @@ def copy_bandwidth(x_host, out_host, x_dev, out_dev, reps: int = 20):
     return res
 
 
+def run_e2e(args, layer, x, w, world, dev):
+    """End to end through the public API: pinned host in, pinned host out,
+    every step's input copied in and output copied back inside the timed
+    region; consecutive steps overlap on three streams (HostPipeline, the
+    library's native pipeline)."""
+    import torch
+    import torch.distributed as dist
+    from mixture_experts_layer_45_b200.layer import HostPipeline
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 100))
+    nbuf = 4
+    x_hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in range(nbuf)]
+    for xh in x_hosts:
+        xh.copy_(x.cpu())
+    out_hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in range(nbuf)]
+    pipe = HostPipeline(layer, w.T)
+    xs = [x_hosts[i % nbuf] for i in range(e2e_steps)]
+    outs = [out_hosts[i % nbuf] for i in range(e2e_steps)]
+    pipe.run(xs[:20], outs[:20])                              # warm-up (the first runs copy slower)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max_ms(pipe.run(xs, outs), dev)
+    if world > 1:
+        dist.barrier()
+    e2e_value = whole_job_tokens_per_s(world, e2e_steps, w.T, e2e_ms)
+    io_bytes = x.numel() * x.element_size()
+    pcie = copy_bandwidth(x_hosts[0], out_hosts[0], pipe.x_dev[0], pipe.out_dev[0])
+    # the device result of the last step equals the device-only forward
+    ref_out = layer.forward(x)
+    torch.cuda.synchronize()
+    if not torch.equal(outs[-1].to(dev).view(torch.int16) if x.dtype == torch.bfloat16 else outs[-1].to(dev),
+                       ref_out.view(torch.int16) if x.dtype == torch.bfloat16 else ref_out):
+        raise RuntimeError("end-to-end output differs from the device forward")
+    return {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
+            "d2h_bytes_per_step": io_bytes, "steps": e2e_steps,
+            "mode": "pinned host buffers; H2D, layer (a CUDA graph per lane) and D2H of consecutive steps "
+                    "overlap on three streams, three lanes; native host loop (moe_pipeline_run)",
+            "copy_gbs": pcie}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -449,36 +510,9 @@ def run_ours(args):
     kt = _lib.moe_timing_read()
     _lib.moe_timing_enable(False)
 
-    # ---- end to end through the public API: pinned host in, pinned host out,
-    # every step's input copied in and output copied back inside the timed
-    # region; consecutive steps overlap on three streams (HostPipeline, the
-    # library's native pipeline)
-    from mixture_experts_layer_45_b200.layer import HostPipeline
-    e2e_steps = args.e2e_steps or max(3, min(args.steps, 100))
-    nbuf = 4
-    x_hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in range(nbuf)]
-    for xh in x_hosts:
-        xh.copy_(x.cpu())
-    out_hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in range(nbuf)]
-    pipe = HostPipeline(layer, w.T)
-    xs = [x_hosts[i % nbuf] for i in range(e2e_steps)]
-    outs = [out_hosts[i % nbuf] for i in range(e2e_steps)]
-    pipe.run(xs[:20], outs[:20])                              # warm-up (the first runs copy slower)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e2e_ms = reduce_max_ms(pipe.run(xs, outs), dev)
-    if world > 1:
-        dist.barrier()
-    e2e_value = whole_job_tokens_per_s(world, e2e_steps, w.T, e2e_ms)
-    io_bytes = x.numel() * x.element_size()
-    pcie = copy_bandwidth(x_hosts[0], out_hosts[0], pipe.x_dev[0], pipe.out_dev[0])
-    # the device result of the last step equals the device-only forward
-    ref_out = layer.forward(x)
-    torch.cuda.synchronize()
-    if not torch.equal(outs[-1].to(dev).view(torch.int16) if x.dtype == torch.bfloat16 else outs[-1].to(dev),
-                       ref_out.view(torch.int16) if x.dtype == torch.bfloat16 else ref_out):
-        raise RuntimeError("end-to-end output differs from the device forward")
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, layer, x, w, world, dev)
 
     if rank != 0:
         if world > 1:
@@ -500,14 +534,24 @@ def run_ours(args):
     ffn_tflops = ffn_flops / (ffn_ms / 1000.0) / 1e12 if ffn_ms else None
     dom_bytes = algorithmic_bytes(dom, w, R, E_active, es)
     dom_s = kernels[dom]["ms_per_launch"] / 1000.0
-    # a kernel timed inside a long run meets the power cap: use the sustained tensor peak there
-    tensor_peak = peaks["bf16_tflops"] if total_ms < 2000 else peaks["bf16_tflops_sustained"]
+    # The tensor peak: the burst figure (a GEMM timed alone, before the power
+    # cap acts) unless the clocks record shows the power cap during the timed
+    # region or the region is seconds long; then the sustained figure, which
+    # was itself measured under the cap.
+    clocks = sampler.summary() if sampler else None
+    capped = bool(clocks and "sw_power_cap" in (clocks.get("reasons") or []))
+    sustained = capped or total_ms >= 2000
+    tensor_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     flops_dom = 2.0 * ffn_rows * w.d * w.ff
     ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if dom in ("ffn1", "ffn2") and w.dtype == "bf16" and flops_dom / max(dom_bytes, 1) > ridge:
         achieved = flops_dom / dom_s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": achieved / tensor_peak}
+                "frac": achieved / tensor_peak,
+                "peak_kind": ("sustained (sw_power_cap during the timed region)" if capped else
+                              "sustained (timed region >= 2 s)" if sustained else "burst"),
+                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                "algorithmic_flops_per_launch": flops_dom}
     else:
         achieved = dom_bytes / dom_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -515,7 +559,6 @@ def run_ours(args):
     roof.update({"kernel": dom, "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes,
                  "traffic": committed_traffic(dom, workload_tag(w))})
 
-    clocks = sampler.summary() if sampler else None
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": warm, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -527,20 +570,17 @@ def run_ours(args):
                    "kernel_timing": "second pass of the same steps with CUDA events around each launch",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": roof,
-        "ffn": {"tflops": ffn_tflops, "frac_of_bf16_peak": (ffn_tflops / peaks["bf16_tflops"]) if ffn_tflops
-                else None, "flops_per_step": ffn_flops, "ms_per_step": ffn_ms},
+        "ffn": {"tflops": ffn_tflops, "frac_of_bf16_peak": (ffn_tflops / tensor_peak) if ffn_tflops else None,
+                "frac_of_burst": (ffn_tflops / peaks["bf16_tflops"]) if ffn_tflops else None,
+                "flops_per_step": ffn_flops, "ms_per_step": ffn_ms},
         "kernels": kernels,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
-                "d2h_bytes_per_step": io_bytes, "steps": e2e_steps,
-                "mode": "pinned host buffers; H2D, layer (a CUDA graph per lane) and D2H of consecutive steps "
-                        "overlap on three streams, three lanes; native host loop (moe_pipeline_run)",
-                "copy_gbs": pcie},
+        "e2e": e2e,
         "clocks": clocks,
         "gpu_launches": launches,
         "stats": {k: st[k] for k in ("aux_loss", "imbalance", "drop_rate", "rerouted")},
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, drawn=inp)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -75,9 +75,29 @@ def test_traffic_is_read_for_the_bench_workload():
 
 
 def test_defaults_meet_the_run_contract():
+    """No flags: one GPU, at least 3 warm-up steps, and the largest
+    single-GPU workload (the large top-2 layer, tensor-bound FFN)."""
     a = bench.parse_args([])
-    assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1 and a.impl == "ours"
-    assert bench.get_workload(a).name == "switch-top1"
+    assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1 and a.impl == "ours" and not a.no_e2e
+    w = bench.get_workload(a)
+    assert (w.name, w.T, w.d, w.ff, w.E, w.k, w.dtype, w.cf) == ("large-top2", 8192, 4096, 14336, 8, 2, "bf16",
+                                                                 None)
+    assert bench.workload_tag(w) == "large-top2-bf16-cfnone"
+
+
+def test_oracle_sample_is_bounded_by_flops():
+    """The oracle's timed sample: a power of two, at most the cap, fewer
+    tokens where each costs more (about 32 GFLOP of float64 per pass)."""
+    big = wl.workload("large-top2")                 # 4*2*4096*14336 = 470 MFLOP per token
+    assert bench.oracle_sample_tokens(big, 1024) == 64
+    sw = wl.workload("switch-top1")                 # 9.4 MFLOP per token
+    assert bench.oracle_sample_tokens(sw, 1024) == 1024 and bench.oracle_sample_tokens(sw, 512) == 512
+    tiny = wl.workload("dense-top2-f32")
+    assert bench.oracle_sample_tokens(tiny, 1024) == 1024
+    for w in wl.all_workloads():
+        n = bench.oracle_sample_tokens(w, 1024)
+        assert 16 <= n <= 1024 and n & (n - 1) == 0
+        assert n == 16 or n * 4 * w.k * w.d * w.ff <= bench.ORACLE_FLOPS_PER_PASS
 
 
 def test_reference_arm_line(capsys, monkeypatch):
@@ -85,7 +105,7 @@ def test_reference_arm_line(capsys, monkeypatch):
     contract's line; under a multi-rank launch only rank 0 does so."""
     import json
     monkeypatch.setenv("RANK", "0")
-    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    assert bench.main(["--impl", "reference", "--workload", "switch-top1", "--steps", "1", "--warmup", "0"]) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "tokens/s"
     assert line["value"] > 0 and line["higher_is_better"] is True and line["steps"] == 1
@@ -95,5 +115,5 @@ def test_reference_arm_line(capsys, monkeypatch):
                            "d2h_bytes_per_step": 0}
     assert line["config"]["workload"].startswith("switch-top1 T=4096")
     monkeypatch.setenv("RANK", "1")
-    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0   # no draw, no output
     assert capsys.readouterr().out == ""
