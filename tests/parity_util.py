@@ -80,3 +80,38 @@ def sample_rows(T: int, n: int, seed: int = 0, must=()) -> np.ndarray:
     rows.update(int(m) for m in must if 0 <= m < T)
     rows.update([0, T - 1])
     return np.array(sorted(rows))
+
+
+def tile_covering_rows(offsets, perm, k: int, T: int, tile: int = 128, seed: int = 0, shared: int = 0) -> np.ndarray:
+    """Output tokens whose rows together reach every `tile`-row M tile of the
+    grouped FFN.
+
+    For each expert group (grouped rows offsets[e] .. offsets[e+1]-1, tiles
+    starting at offsets[e]) one random row of every tile and the group's last
+    row are taken, each mapped to its token perm[row] // k.  Tiles of 2*tile
+    rows (the CTA-pair kernel) are unions of two such tiles, so they are
+    reached too; a token's output row depends on every N tile of both GEMMs.
+    With shared experts (each a group of all T tokens in order) one token of
+    every `tile`-token block is added as well.
+    """
+    rng = np.random.default_rng(seed)
+    offsets = np.asarray(offsets, np.int64)
+    perm = np.asarray(perm, np.int64)
+    toks = set()
+    for e in range(len(offsets) - 1):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        for t0 in range(lo, hi, tile):
+            t1 = min(t0 + tile, hi)
+            toks.add(int(perm[int(rng.integers(t0, t1))] // k))
+        if hi > lo:
+            toks.add(int(perm[hi - 1] // k))
+    if shared:
+        for t0 in range(0, T, tile):
+            toks.add(int(rng.integers(t0, min(t0 + tile, T))))
+    return np.array(sorted(toks), dtype=np.int64)
+
+
+def m_tiles(offsets, tile: int = 128) -> int:
+    """M tiles of `tile` rows over the expert groups of the grouped layout."""
+    offsets = np.asarray(offsets, np.int64)
+    return int(sum(-(-int(offsets[e + 1] - offsets[e]) // tile) for e in range(len(offsets) - 1)))

@@ -296,7 +296,12 @@ def test_forward_matches_oracle(w):
         dsp0 = moe_ref.dispatch(idx_np, w.E, cap)
         hot = np.nonzero(idx_np[:, 0] == np.bincount(idx_np.ravel()).argmax())[0][:8]
         dropped = np.nonzero((dsp0["slot_of"].reshape(w.T, w.k) < 0).any(1))[0][:8]
-        rows = pu.sample_rows(w.T, 96, seed=w.seed, must=list(hot) + list(dropped))
+        # one row of every 128-row M tile of every expert group (so every
+        # 256-row CTA-pair tile too), plus random, hot-expert and dropped rows
+        tiles = pu.tile_covering_rows(dsp0["offsets"], dsp0["perm"], w.k, w.T, seed=w.seed)
+        rows = pu.sample_rows(w.T, 96, seed=w.seed, must=list(hot) + list(dropped) + list(tiles))
+        print(f"{w.name}: {len(rows)} sampled output rows reach all {pu.m_tiles(dsp0['offsets'])} "
+              f"128-row M tiles ({pu.m_tiles(dsp0['offsets'], 256)} 256-row tiles)")
         ref, dsp, r = oracle_on_gpu_routing(inp, w, idx_np, rows)
         got = out_np[rows]
     err = pu.max_rel_err(got, ref)

@@ -66,7 +66,12 @@ def test_forward_shared_matches_oracle(w):
     dropped = np.nonzero((dsp0["slot_of"].reshape(w.T, w.k) < 0).all(1))[0][:16]
     if cap >= 0:
         assert len(dropped) > 0 or w.cf is None or w.cf > 1.0
-    rows = pu.sample_rows(w.T, 96 if w.T > 2048 else w.T, seed=w.seed, must=list(dropped))
+    # every 128-row M tile of every routed and shared group (so every
+    # 256-row CTA-pair tile too), plus random and dropped rows
+    tiles = pu.tile_covering_rows(dsp0["offsets"], dsp0["perm"], w.k, w.T, seed=w.seed, shared=w.shared)
+    rows = pu.sample_rows(w.T, 96 if w.T > 2048 else w.T, seed=w.seed, must=list(dropped) + list(tiles))
+    print(f"{w.name} S={w.shared}: {len(rows)} sampled output rows reach all "
+          f"{pu.m_tiles(dsp0['offsets']) + w.shared * -(-w.T // 128)} 128-row M tiles")
     ref, dsp, r = oracle_rows(inp, idx, w.k, w.E, cap, rows)
     err = pu.max_rel_err(out[rows], ref)
     assert err <= pu.TOL[w.dtype], err

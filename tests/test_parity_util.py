@@ -55,3 +55,26 @@ def test_error_bound_is_small_relative_to_logits():
 def test_max_rel_err():
     assert pu.max_rel_err([1.0, 2.0], [1.0, 2.0]) == 0.0
     assert pu.max_rel_err([1.0, 2.1], [1.0, 2.0]) == pytest.approx(0.05)
+
+
+@pytest.mark.parametrize("k,E,T", [(2, 64, 3000), (1, 8, 1000), (2, 8, 4096)])
+def test_tile_covering_rows_reach_every_m_tile(k, E, T):
+    rng = np.random.default_rng(T)
+    # skewed routing: expert 0 takes most rows, some experts are empty
+    p = np.r_[0.5, np.full(E - 1, 0.5 / (E - 1))]
+    idx = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)])
+    d = moe_ref.dispatch(idx, E, -1)
+    toks = pu.tile_covering_rows(d["offsets"], d["perm"], k, T, seed=1)
+    slot = d["slot_of"].reshape(T, k)
+    rows_reached = set(int(r) for r in slot[toks].ravel() if r >= 0)
+    for tile in (128, 256):
+        reached = set()
+        for e in range(E):
+            lo, hi = int(d["offsets"][e]), int(d["offsets"][e + 1])
+            for t0 in range(lo, hi, tile):
+                if any(t0 <= r < min(t0 + tile, hi) for r in rows_reached):
+                    reached.add((e, t0))
+        assert len(reached) == pu.m_tiles(d["offsets"], tile)
+    # shared groups: one token of every 128-token block
+    toks_s = pu.tile_covering_rows(d["offsets"], d["perm"], k, T, seed=1, shared=2)
+    assert set(toks_s // 128) == set(range(-(-T // 128)))
