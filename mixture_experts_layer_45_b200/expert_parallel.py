@@ -106,15 +106,54 @@ def received_expert_ids(recv_counts: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# the collectives
+# ---------------------------------------------------------------------------
+
+class Exchange:
+    """The two collectives of the multi-GPU forms on a torch.distributed
+    group: all-to-all(-v) and a sum all-reduce.
+
+    A backend that moves device tensors (NCCL) gets them as they are.  A
+    backend that moves host tensors only (gloo) gets each exchanged tensor
+    copied to host memory and the result copied back, so the same forms run
+    over gloo, e.g. several processes sharing one GPU."""
+
+    def __init__(self, group=None, host_staged=None):
+        self.group = group
+        if host_staged is None:
+            host_staged = dist.get_backend(group) == "gloo"
+        self.host_staged = host_staged
+
+    def all_to_all(self, out: torch.Tensor, inp: torch.Tensor, out_splits=None, in_splits=None) -> None:
+        if not (self.host_staged and (out.is_cuda or inp.is_cuda)):
+            dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
+            return
+        h_out = torch.empty(out.shape, dtype=out.dtype)
+        dist.all_to_all_single(h_out, inp.cpu(), out_splits, in_splits, group=self.group)
+        out.copy_(h_out)
+
+    def all_reduce_sum(self, t: torch.Tensor) -> None:
+        if not (self.host_staged and t.is_cuda):
+            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group)
+            return
+        h = t.cpu()
+        dist.all_reduce(h, op=dist.ReduceOp.SUM, group=self.group)
+        t.copy_(h)
+
+
+# ---------------------------------------------------------------------------
 # the choreography
 # ---------------------------------------------------------------------------
 
-def ep_forward(x: torch.Tensor, steps, E: int, k: int, capacity: int, group=None) -> torch.Tensor:
+def ep_forward(x: torch.Tensor, steps, E: int, k: int, capacity: int, group=None,
+               exchange: Exchange = None) -> torch.Tensor:
     """One expert-parallel forward pass of this rank's tokens x [T, d].
 
     `steps` provides route / dispatch / ffn / combine (see LibmoeSteps);
-    the collectives run on `group` (default: the world)."""
+    the collectives run on `group` (default: the world) through `exchange`
+    (default: Exchange(group))."""
     G = dist.get_world_size(group)
+    xc = exchange if exchange is not None else Exchange(group)
     T, d = x.shape
     dev = x.device
     el = E // G
@@ -130,14 +169,14 @@ def ep_forward(x: torch.Tensor, steps, E: int, k: int, capacity: int, group=None
     # 2. counts, then rows and gates
     send_c = torch.from_numpy(dest_counts(offs, E, G).reshape(-1)).to(dev)
     recv_c = torch.empty(G * el, dtype=torch.int32, device=dev)
-    dist.all_to_all_single(recv_c, send_c, group=group)
+    xc.all_to_all(recv_c, send_c)
     rc = recv_c.cpu().numpy().reshape(G, el)
     recv_splits = [int(v) for v in rc.sum(axis=1)]
     Rr = sum(recv_splits)
     xr = torch.empty((Rr, d), dtype=x.dtype, device=dev)
     gr = torch.empty((Rr,), dtype=torch.float32, device=dev)
-    dist.all_to_all_single(xr, dsp["xp"][:R].contiguous(), recv_splits, splits, group=group)
-    dist.all_to_all_single(gr, dsp["row_gate"][:R].contiguous(), recv_splits, splits, group=group)
+    xc.all_to_all(xr, dsp["xp"][:R].contiguous(), recv_splits, splits)
+    xc.all_to_all(gr, dsp["row_gate"][:R].contiguous(), recv_splits, splits)
 
     # 3. the local experts on the received rows
     yr = torch.empty((Rr, d), dtype=x.dtype, device=dev)
@@ -150,17 +189,19 @@ def ep_forward(x: torch.Tensor, steps, E: int, k: int, capacity: int, group=None
     # 4. rows home, then each token's sum (a token whose slots were all
     # dropped sums nothing: 0)
     yb = torch.empty((R, d), dtype=x.dtype, device=dev)
-    dist.all_to_all_single(yb, yr, splits, recv_splits, group=group)
+    xc.all_to_all(yb, yr, splits, recv_splits)
     if R == 0:
         yb = torch.zeros((1, d), dtype=x.dtype, device=dev)
     return steps.combine(yb, dsp["slot_of"], T, k)
 
 
-def sharded_forward(x: torch.Tensor, steps, E: int, k: int, capacity: int, group=None) -> torch.Tensor:
+def sharded_forward(x: torch.Tensor, steps, E: int, k: int, capacity: int, group=None,
+                    exchange: Exchange = None) -> torch.Tensor:
     """One forward pass of the replicated batch x [T, d] with every expert's
     hidden units split over the ranks of `group`: each rank's grouped FFN
     gives gated partial rows from its slice, an all-reduce sums them, and
     the combine (gates already applied) gives the replicated output."""
+    xc = exchange if exchange is not None else Exchange(group)
     T, d = x.shape
     idx, gate = steps.route(x)
     dsp = steps.dispatch(idx, gate, T, k, E, capacity, x)
@@ -169,7 +210,7 @@ def sharded_forward(x: torch.Tensor, steps, E: int, k: int, capacity: int, group
         return steps.combine(torch.zeros((1, d), dtype=x.dtype, device=x.device), dsp["slot_of"], T, k)
     yp = steps.ffn(dsp["xp"], dsp["offsets"], dsp["row_gate"], T * k)
     part = yp[:R]
-    dist.all_reduce(part, op=dist.ReduceOp.SUM, group=group)
+    xc.all_reduce_sum(part)
     return steps.combine(yp, dsp["slot_of"], T, k)
 
 
