@@ -193,7 +193,11 @@ MOE_API int moe_dispatch(const int32_t* topk_idx, const float* topk_gate,
  * MOE_ERR_WORKSPACE (and print why to stderr) before launching anything.
  * The first call on a device looks up the array's device address for that
  * device (cudaGetSymbolAddress, with that device current); make that first
- * call before any stream capture.  All calls share the one array and it
+ * call before any stream capture.  The address is kept with the CUDA
+ * context it belongs to: after a device reset (cudaDeviceReset) or a
+ * re-created primary context, the next call on that device sees a new
+ * context and looks the address up again, so that call too belongs before
+ * any capture.  All calls share the one array and it
  * keeps the last call's contents (every entry a call reads is written
  * earlier in that call, so nothing needs clearing): calls whose executions
  * overlap on the GPU, on different streams or host threads, race on it and
@@ -440,6 +444,22 @@ MOE_API int moe_timing_enable(int enable);
  * the last read; then clears the record.  Arrays have MOE_NUM_KERNELS
  * entries; either may be NULL. */
 MOE_API int moe_timing_read(double* ms_per_kernel, int64_t* launches_per_kernel);
+
+/* Profiler annotations (the blog "MoE Parallelism for Inference", section
+ * on profiling: look at the router step and the expert passes separately).
+ * When on, every entry point that enqueues GPU work opens an NVTX range
+ * named after itself ("moe_forward", "moe_dispatch", ...), and every kernel
+ * launch inside it a nested range "moe.kernel.<step>" (router, count, scan,
+ * permute, gather, ffn1, ffn2, combine, stats, reroute), so that a timeline
+ * from Nsight Systems, or from torch.profiler recording NVTX, shows the
+ * steps apart.  The ranges mark host time: when the launches were issued.
+ * Off by default; on when the environment variable MOE_NVTX is "1" at the
+ * library's first check, or after moe_trace_enable(1).  With no profiler
+ * attached a range costs next to nothing; off, one atomic load.
+ * moe_trace_enable returns the previous setting (0 or 1) and never fails;
+ * moe_trace_enabled returns the current one.  Host only: no GPU needed. */
+MOE_API int moe_trace_enable(int enable);
+MOE_API int moe_trace_enabled(void);
 
 #ifdef __cplusplus
 }

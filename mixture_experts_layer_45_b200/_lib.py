@@ -84,6 +84,8 @@ _SIGS = {
     "moe_launch_count": (ctypes.c_uint64, []),
     "moe_timing_enable": (_I, [_I]),
     "moe_timing_read": (_I, [_P, _P]),
+    "moe_trace_enable": (_I, [_I]),
+    "moe_trace_enabled": (_I, []),
 }
 EXPORTED = sorted(_SIGS)
 
@@ -265,6 +267,15 @@ def moe_debug_gelu(x, y, n, variant, stream=None):
 
 def moe_launch_count() -> int:
     return int(load().moe_launch_count())
+
+
+def moe_trace_enable(enable: bool) -> bool:
+    """Turn the library's NVTX ranges on or off; returns the previous setting."""
+    return bool(load().moe_trace_enable(1 if enable else 0))
+
+
+def moe_trace_enabled() -> bool:
+    return bool(load().moe_trace_enabled())
 
 
 def moe_timing_enable(enable: bool):

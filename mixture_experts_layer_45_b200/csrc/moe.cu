@@ -14,6 +14,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "dispatch.cuh"
 #include "ffn.cuh"
@@ -22,6 +24,50 @@
 using namespace moe;
 
 namespace {
+
+// ---------------------------------------------------------------------------
+// NVTX ranges: one around every entry point that enqueues work and one
+// around every kernel launch, so that a profiler timeline (Nsight Systems,
+// or torch.profiler recording NVTX) shows the router, the dispatch, the two
+// FFN GEMMs and the combine apart.  Off unless the environment variable
+// MOE_NVTX is "1" when the library first checks, or moe_trace_enable(1) is
+// called; off, a range costs one relaxed atomic load.
+// ---------------------------------------------------------------------------
+std::atomic<int> g_trace{-1};
+
+bool trace_on() {
+    int v = g_trace.load(std::memory_order_relaxed);
+    if (v < 0) {
+        const char* e = std::getenv("MOE_NVTX");
+        int want = (e != nullptr && e[0] == '1') ? 1 : 0;
+        int expected = -1;
+        g_trace.compare_exchange_strong(expected, want, std::memory_order_relaxed);
+        v = g_trace.load(std::memory_order_relaxed);
+    }
+    return v == 1;
+}
+
+class TraceRange {
+  public:
+    explicit TraceRange(const char* name) : on_(trace_on()) {
+        if (on_) nvtxRangePushA(name);
+    }
+    ~TraceRange() {
+        if (on_) nvtxRangePop();
+    }
+    TraceRange(const TraceRange&) = delete;
+    TraceRange& operator=(const TraceRange&) = delete;
+
+  private:
+    bool on_;
+};
+
+const char* kernel_range_name(int kernel) {
+    static const char* const names[MOE_NUM_KERNELS] = {
+        "moe.kernel.router", "moe.kernel.count", "moe.kernel.scan", "moe.kernel.permute", "moe.kernel.gather",
+        "moe.kernel.ffn1",   "moe.kernel.ffn2",  "moe.kernel.combine", "moe.kernel.stats", "moe.kernel.reroute"};
+    return (kernel >= 0 && kernel < MOE_NUM_KERNELS && names[kernel]) ? names[kernel] : "moe.kernel";
+}
 
 // ---------------------------------------------------------------------------
 // launch counter and optional per-kernel event timing
@@ -73,7 +119,7 @@ cudaEvent_t take_event_locked() {
 // and, in finish(), checks the launch, counts it and records the stop event.
 class Launch {
   public:
-    Launch(int kernel, cudaStream_t s) : kernel_(kernel), stream_(s) {
+    Launch(int kernel, cudaStream_t s) : trace_(kernel_range_name(kernel)), kernel_(kernel), stream_(s) {
         if (g_timing.enabled) {
             std::lock_guard<std::mutex> lk(g_timing.mu);
             start_ = take_event_locked();
@@ -102,6 +148,7 @@ class Launch {
     }
 
   private:
+    TraceRange trace_;
     int kernel_;
     cudaStream_t stream_;
     cudaEvent_t start_ = nullptr;
@@ -859,18 +906,46 @@ static __device__ __align__(256) uint8_t g_dispatch_scratch[kNoallocScratchBytes
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
 
-// Device address of g_dispatch_scratch on the current device (looked up on
-// the first call for that device, with that device current).
+// The driver's cuCtxGetCurrent, reached through the runtime (the library
+// does not link the driver library); null if the driver does not offer it.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+    static const CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<CtxGetCurrentFn>(p);
+    }();
+    return fn;
+}
+
+CUcontext current_context() {
+    CUcontext c = nullptr;
+    const CtxGetCurrentFn f = ctx_get_current();
+    if (f == nullptr || f(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+// Device address of g_dispatch_scratch on the current device, looked up
+// with that device current on the first call for it and kept with the
+// context it belongs to.  A device reset or a re-created primary context
+// gives the device a new context (and the module a new load), so the
+// address is looked up again on the next call rather than reused.
 int noalloc_scratch(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    const CUcontext ctx = current_context();
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || ctx != g_noalloc_ctx[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
         g_noalloc_ptr[dev] = p;
+        g_noalloc_ctx[dev] = current_context();   // the runtime has made the context current by now
     }
     *out = g_noalloc_ptr[dev];
     return MOE_OK;
@@ -950,6 +1025,7 @@ size_t moe_dispatch_workspace_size(int T, int k, int E) {
 
 int moe_router_topk(const void* x, const void* w_router, const float* logit_bias, int T, int d, int E, int k,
                     int dtype, int32_t* topk_idx, float* topk_gate, float* prob_sum, void* stream) {
+    TraceRange trace_("moe_router_topk");
     int rc = check_sizes(T, d, 8, E, k, dtype, false);
     if (rc != MOE_OK) return rc;
     if (T == 0) {
@@ -968,6 +1044,7 @@ int moe_dispatch(const int32_t* topk_idx, const float* topk_gate, int T, int k, 
                  int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of, uint8_t* drop_mask,
                  float* row_gate, const void* x, void* xp, int d, int dtype, void* ws, size_t ws_bytes,
                  void* stream) {
+    TraceRange trace_("moe_dispatch");
     const bool want_rows = (x != nullptr || xp != nullptr);
     const int rc = want_rows ? check_sizes(T, d, 8, E, k, dtype, false) : check_sizes(T, 8, 8, E, k, MOE_F32, false);
     if (rc != MOE_OK) return rc;
@@ -990,6 +1067,7 @@ int moe_dispatch(const int32_t* topk_idx, const float* topk_gate, int T, int k, 
 int moe_dispatch_noalloc(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E, int capacity,
                          int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of, uint8_t* drop_mask,
                          float* row_gate, const void* x, void* xp, int d, int dtype, void* stream) {
+    TraceRange trace_("moe_dispatch_noalloc");
     const bool want_rows = (x != nullptr || xp != nullptr);
     const int rc = want_rows ? check_sizes(T, d, 8, E, k, dtype, false) : check_sizes(T, 8, 8, E, k, MOE_F32, false);
     if (rc != MOE_OK) return rc;
@@ -1056,6 +1134,7 @@ int moe_dispatch_reroute(const int32_t* ranked_idx, const float* ranked_gate, in
                          int capacity, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of,
                          uint8_t* drop_mask, float* row_gate, const void* x, void* xp, int d, int dtype, void* ws,
                          size_t ws_bytes, void* stream) {
+    TraceRange trace_("moe_dispatch_reroute");
     const bool want_rows = (x != nullptr || xp != nullptr);
     int rc = want_rows ? check_sizes(T, d, 8, E, k, dtype, false) : check_sizes(T, 8, 8, E, k, MOE_F32, false);
     if (rc != MOE_OK) return rc;
@@ -1102,6 +1181,7 @@ int moe_dispatch_reroute(const int32_t* ranked_idx, const float* ranked_gate, in
 int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
                     const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp,
                     int dtype, void* stream) {
+    TraceRange trace_("moe_grouped_ffn");
     const int rc = check_sizes(max_rows, d, ff, E, 1, dtype, true);
     if (rc != MOE_OK) return rc;
     if (max_rows == 0) return MOE_OK;
@@ -1115,6 +1195,7 @@ int moe_grouped_ffn(const void* xp, const int32_t* offsets, int max_rows, int E,
 
 int moe_shared_ffn(const void* x, int T, int d, int ff, int S, const void* w1s, const void* b1s, const void* w2s,
                    const void* b2s, void* h, void* ys, int dtype, void* stream) {
+    TraceRange trace_("moe_shared_ffn");
     int rc = check_sizes(T, d, ff, 1, 1, dtype, true);
     if (rc != MOE_OK) return rc;
     if ((rc = check_shared(T, 0, S)) != MOE_OK) return rc;
@@ -1137,6 +1218,7 @@ int moe_shared_ffn(const void* x, int T, int d, int ff, int S, const void* w1s, 
 
 int moe_combine(const void* yp, const int32_t* slot_of, const float* topk_gate, int T, int k, int d, int dtype,
                 void* out, void* stream) {
+    TraceRange trace_("moe_combine");
     const int rc = check_sizes(T, d, 8, k, k, dtype, false);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1147,6 +1229,7 @@ int moe_combine(const void* yp, const int32_t* slot_of, const float* topk_gate, 
 
 int moe_combine_shared(const void* yp, const int32_t* slot_of, const float* topk_gate, const void* ys, int S, int T,
                        int k, int d, int dtype, void* out, void* stream) {
+    TraceRange trace_("moe_combine_shared");
     int rc = check_sizes(T, d, 8, k, k, dtype, false);
     if (rc != MOE_OK) return rc;
     if ((rc = check_shared(T, k, S)) != MOE_OK) return rc;
@@ -1158,6 +1241,7 @@ int moe_combine_shared(const void* yp, const int32_t* slot_of, const float* topk
 
 int moe_layer_stats(const int32_t* counts, const int32_t* offsets, const float* prob_sum, int T, int k, int E,
                     moe_stats* stats, void* stream) {
+    TraceRange trace_("moe_layer_stats");
     const int rc = check_sizes(T, 8, 8, E, k, MOE_F32, false);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_ERR_INVALID_ARG;   // the statistics divide by T
@@ -1169,6 +1253,7 @@ int moe_forward(const void* x, const void* w_router, const float* logit_bias, co
                 const void* w2, const void* b2, int T, int d, int ff, int E, int k, int capacity, int dtype,
                 void* out, moe_stats* stats, int32_t* topk_idx_out, float* topk_gate_out, void* ws,
                 size_t ws_bytes, void* stream) {
+    TraceRange trace_("moe_forward");
     return moe_forward_ex(x, w_router, logit_bias, w1, b1, w2, b2, 0, nullptr, nullptr, nullptr, nullptr, 0, T, d,
                           ff, E, k, capacity, dtype, out, stats, topk_idx_out, topk_gate_out, ws, ws_bytes, stream);
 }
@@ -1178,6 +1263,7 @@ int moe_forward_ex(const void* x, const void* w_router, const float* logit_bias,
                    const void* b2s, int reroute_rounds, int T, int d, int ff, int E, int k, int capacity, int dtype,
                    void* out, moe_stats* stats, int32_t* topk_idx_out, float* topk_gate_out, void* ws,
                    size_t ws_bytes, void* stream) {
+    TraceRange trace_("moe_forward_ex");
     int rc = check_sizes(T, d, ff, E, k, dtype, true);
     if (rc != MOE_OK) return rc;
     if ((rc = check_shared(T, k, S)) != MOE_OK) return rc;
@@ -1290,6 +1376,14 @@ int moe_timing_enable(int enable) {
     g_timing.enabled = enable != 0;
     return MOE_OK;
 }
+
+int moe_trace_enable(int enable) {
+    const int prev = trace_on() ? 1 : 0;
+    g_trace.store(enable ? 1 : 0, std::memory_order_relaxed);
+    return prev;
+}
+
+int moe_trace_enabled(void) { return trace_on() ? 1 : 0; }
 
 int moe_timing_read(double* ms_per_kernel, int64_t* launches_per_kernel) {
     std::lock_guard<std::mutex> lk(g_timing.mu);

@@ -196,6 +196,7 @@ int moe_pipeline_run(moe_pipeline* p, const void* const* x_host, void* const* ou
     if (p == nullptr || n < 0 || (n > 0 && (x_host == nullptr || out_host == nullptr))) return MOE_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i)
         if (x_host[i] == nullptr || out_host[i] == nullptr) return MOE_ERR_INVALID_ARG;
+    TraceRange trace_("moe_pipeline_run");
     DeviceGuard guard(p->device);
     if (!guard.ok) return MOE_ERR_CUDA;
     bool ok = cudaEventRecord(p->t0, p->s_in) == cudaSuccess && cudaStreamWaitEvent(p->s_run, p->t0, 0) == cudaSuccess &&

@@ -255,3 +255,20 @@ def test_pipeline_checks(lib):
     assert lib.moe_pipeline_run(FAKE, None, None, 2, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_pipeline_run(FAKE, arr(FAKE, None), arr(FAKE, FAKE), 2, None) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_pipeline_destroy(None) == _lib.MOE_OK
+
+
+def test_nvtx_ranges_default_off_and_switch(lib, monkeypatch):
+    """The profiler ranges are off unless asked for; the switch returns the
+    previous setting; calls that reject their arguments still work with the
+    ranges on (no GPU needed)."""
+    if os.environ.get("MOE_NVTX") == "1":
+        pytest.skip("MOE_NVTX=1 in this environment")
+    assert _lib.moe_trace_enabled() is False
+    assert _lib.moe_trace_enable(True) is False
+    try:
+        assert _lib.moe_trace_enabled() is True
+        rc = lib.moe_combine(None, None, None, 4, 1, 8, _lib.MOE_F32, None, None)
+        assert rc == _lib.MOE_ERR_INVALID_ARG
+    finally:
+        assert _lib.moe_trace_enable(False) is True
+    assert _lib.moe_trace_enabled() is False

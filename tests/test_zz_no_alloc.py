@@ -75,3 +75,32 @@ def test_noalloc_dispatch_rejects_sizes_beyond_its_limit():
         _lib.moe_dispatch_noalloc(dummy, None, T, 2, 8, -1, dummy, dummy, dummy, dummy, None, None, None, None,
                                   8, _lib.MOE_F32)
     assert ei.value.status == _lib.MOE_ERR_WORKSPACE
+
+
+def test_noalloc_dispatch_at_its_exact_limit():
+    """T*k exactly MOE_NOALLOC_MAX_ASSIGNMENTS with the most experts: the
+    per-chunk histograms and bases then fill the fixed scratch to its last
+    byte.  The call is accepted and agrees bit for bit with moe_dispatch."""
+    A = _lib.MOE_NOALLOC_MAX_ASSIGNMENTS
+    E, k, d = _lib.MOE_MAX_EXPERTS, 2, 64
+    T = A // k
+    rng = np.random.default_rng(9)
+    p = rng.dirichlet(np.ones(E) * 0.5)
+    first = rng.choice(E, size=T, p=p)
+    second = (first + 1 + rng.integers(0, E - 1, size=T)) % E          # a different expert
+    idx = torch.from_numpy(np.stack([first, second], 1).astype(np.int32)).to(DEV)
+    gate = torch.from_numpy(rng.random((T, k)).astype(np.float32)).to(DEV)
+    x = torch.from_numpy(rng.normal(size=(T, d)).astype(np.float32)).to(DEV, torch.bfloat16)
+    cap = int(T * k / E)                                                 # capacity factor 1.0: drops
+    a = _outputs(T, k, E, d, _lib.MOE_BF16)
+    _lib.moe_dispatch_noalloc(idx, gate, T, k, E, cap, a["counts"], a["offsets"], a["perm"], a["slot_of"],
+                              a["drop"], a["row_gate"], x, a["xp"], d, _lib.MOE_BF16)
+    b = _outputs(T, k, E, d, _lib.MOE_BF16)
+    nws = _lib.moe_dispatch_workspace_size(T, k, E)
+    ws = torch.empty(nws, dtype=torch.uint8, device=DEV)
+    _lib.moe_dispatch(idx, gate, T, k, E, cap, b["counts"], b["offsets"], b["perm"], b["slot_of"], b["drop"],
+                      b["row_gate"], x, b["xp"], d, _lib.MOE_BF16, ws, nws)
+    assert _lib.moe_get_error() == _lib.MOE_OK
+    for key in a:
+        assert torch.equal(a[key].view(torch.uint8), b[key].view(torch.uint8)), key
+    assert int(a["counts"].sum()) == A and int(a["drop"].sum()) > 0
