@@ -76,25 +76,39 @@ __device__ __forceinline__ float gelu_erf(float v) {
     return 0.5f * v * (1.0f + erff(v * 0.70710678118654752440f));
 }
 
-// erf(z) by Abramowitz & Stegun, Handbook of Mathematical Functions, eq.
-// 7.1.26: erf(a) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-a^2),
-// t = 1 / (1 + p a), a >= 0, |error| <= 1.5e-7; odd in z.  Branch-free, one
-// exponential and one reciprocal: used where the result is rounded to bf16.
-__device__ __forceinline__ float erf_as7126(float z) {
-    const float a = fabsf(z);
-    const float t = __fdividef(1.0f, fmaf(0.3275911f, a, 1.0f));
-    float poly = fmaf(1.061405429f, t, -1.453152027f);
-    poly = fmaf(poly, t, 1.421413741f);
-    poly = fmaf(poly, t, -0.284496736f);
-    poly = fmaf(poly, t, 0.254829592f);
-    poly *= t;
-    const float r = fmaf(-poly, __expf(-a * a), 1.0f);
-    return copysignf(r, z);
+// The hardware's approximate reciprocal and base-2 exponential (PTX
+// rcp.approx.ftz.f32 and ex2.approx.ftz.f32).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
-// GELU with the A&S erf (bf16 tensor-core epilogue)
+// GELU(v) = v * Phi(v), Phi(v) = (1 + erf(v / sqrt 2)) / 2, with erf by
+// Abramowitz & Stegun, Handbook of Mathematical Functions, eq. 7.1.26:
+// 1 - erf(a) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-a^2),
+// t = 1 / (1 + p a), a >= 0, |error| <= 1.5e-7.  With a = |v| / sqrt 2:
+// q = (1 - erf(a)) / 2 = (b1 t + ... + b5 t^5) 2^(-v^2 log2(e) / 2),
+// b_i = a_i / 2, t = 1 / (1 + (p / sqrt 2) |v|); and since erf is odd,
+// Phi(v) = 1 - q for v >= 0 and q for v < 0.  One reciprocal and one
+// exponential, no division by sqrt 2 and no sign transfer: used in the
+// bf16 tensor-core epilogue, where the result is rounded to bf16.
 __device__ __forceinline__ float gelu_as(float v) {
-    return 0.5f * v * (1.0f + erf_as7126(v * 0.70710678118654752440f));
+    constexpr float kP = 0.2316418883f;              // p / sqrt 2, p = 0.3275911
+    constexpr float kE = -0.72134752044448169f;      // -log2(e) / 2
+    const float t = rcp_approx(fmaf(kP, fabsf(v), 1.0f));
+    float poly = fmaf(0.5307027145f, t, -0.7265760135f);   // b5, b4
+    poly = fmaf(poly, t, 0.7107068705f);                    // b3
+    poly = fmaf(poly, t, -0.142248368f);                    // b2
+    poly = fmaf(poly, t, 0.127414796f);                     // b1
+    poly *= t;
+    const float q = poly * ex2_approx((kE * v) * v);
+    return v * (v >= 0.f ? 1.0f - q : q);
 }
 
 // ---------------------------------------------------------------------------
@@ -129,21 +143,52 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: while the phase is incomplete the
+// thread may be suspended in hardware for up to about `hint_ns` and resumes
+// as soon as the phase completes, instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Longest single suspension inside mbar_wait: the abort flag and the time
+// limit are checked at least this often.
+constexpr uint32_t kWaitSleepNs = 100000;   // 100 us
+
 // Wait for the phase with the given parity to complete.  Gives up when the
 // CTA-wide abort flag is raised or after kWaitLimitNs (then raises the flag
-// and records MOE_ERR_TIMEOUT).  Returns false when it gave up.
+// and records MOE_ERR_TIMEOUT).  Returns false when it gave up.  Between
+// checks the thread sleeps on the barrier (mbar_try_wait_sleep), so waiting
+// warps take no issue slots from the warps that feed the tensor cores.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             set_error(MOE_ERR_TIMEOUT);
             return false;
         }
+    }
+}
+
+// Teardown wait: until the phase completes or kWaitLimitNs passes (no abort
+// flag, no error: used where a kernel only makes sure its own asynchronous
+// copies or MMAs have finished before it frees or leaves).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs) && globaltimer_ns() - t0 < kWaitLimitNs) {
     }
 }
 

@@ -481,6 +481,8 @@ forward_dispatch_kernel(const int32_t* __restrict__ idx, const float* __restrict
     __shared__ int cnt_s[MOE_MAX_EXPERTS];
     __shared__ float fp_s[MOE_MAX_EXPERTS];
     __shared__ int slot_s[kFwdMaxChunk];
+    __shared__ int red_pre[kFwdThreads], red_tot[kFwdThreads];
+    __shared__ float red_ps[kFwdThreads];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int chunk = blockIdx.x;
     const bool lead = (blockIdx.x == 0 && blockIdx.y == 0);
@@ -488,18 +490,38 @@ forward_dispatch_kernel(const int32_t* __restrict__ idx, const float* __restrict
     const int a0 = chunk * chunk_tokens * k;
     const int na = min(chunk_tokens * k, A - a0);
 
-    if (tid < E) {
-        const int e = tid;
+    // Per-expert totals and this chunk's bases from the router's per-chunk
+    // histograms.  The whole CTA sums: thread (part, e) takes chunks part,
+    // part + parts, ... of expert e (loads coalesced across experts), then
+    // thread e adds the parts' partial sums in part order (a fixed order:
+    // the probability sums are reproducible run to run).
+    const int parts = kFwdThreads / E;   // >= 1
+    if (tid < parts * E) {
+        const int e = tid % E, part = tid / E;
         int pre = 0, tot = 0;
         float ps = 0.f;
-#pragma unroll 8
-        for (int b = 0; b < nchunk; ++b) {
+#pragma unroll 4
+        for (int b = part; b < nchunk; b += parts) {
             const int h = hist[size_t(b) * E + e];
             tot += h;
             pre += (b < chunk) ? h : 0;
         }
         if (lead && st != nullptr && psum_part != nullptr)
-            for (int b = 0; b < nchunk; ++b) ps += psum_part[size_t(b) * E + e];
+            for (int b = part; b < nchunk; b += parts) ps += psum_part[size_t(b) * E + e];
+        red_pre[tid] = pre;
+        red_tot[tid] = tot;
+        red_ps[tid] = ps;
+    }
+    __syncthreads();
+    if (tid < E) {
+        const int e = tid;
+        int pre = 0, tot = 0;
+        float ps = 0.f;
+        for (int p = 0; p < parts; ++p) {
+            pre += red_pre[p * E + e];
+            tot += red_tot[p * E + e];
+            ps += red_ps[p * E + e];
+        }
         base_s[e] = pre;
         cnt_s[e] = tot;
         kept_s[e] = capacity < 0 ? tot : min(tot, capacity);

@@ -36,18 +36,26 @@ struct SharedGroups {
 constexpr int kMaxGroups = MOE_MAX_EXPERTS + MOE_MAX_SHARED;
 
 struct TileTable {
-    int start[kMaxGroups + 1];   // first tile of each group; start[G] = total
+    int start[kMaxGroups + 1];   // first tile of the group at each walk rank; start[G] = total
+    int order[kMaxGroups];       // group at each walk rank
     int mtiles[kMaxGroups];      // M tiles of each group
     int arow[kMaxGroups];        // first A row of each group
     int crow[kMaxGroups];        // first C row (and row_gate / out_rows index)
     int rows[kMaxGroups];        // rows of each group
-    int routed_tiles;            // start[E]: tiles of the routed groups
+    int routed_tiles;            // tiles of the routed groups (ranks 0 .. E-1)
+    int zip;                     // 0: plain walk; > 0: hot/cold interleave, positions per wave
 };
 
 // Must be called by all threads of the CTA; ends with __syncthreads().
 // Routed group e < E covers rows offsets[e] .. offsets[e+1]-1 of A and C.
+//
+// zip > 0 (the number of CTAs, or CTA pairs, walking the tiles together)
+// ranks the routed groups by M tiles, largest first (ties: lower index
+// first), and decode_tile then interleaves the two ends of that list (see
+// there).  zip = 0 keeps the groups in index order.  Shared groups always
+// follow the routed ones.
 __device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ offsets, int E, const SharedGroups& sh,
-                                                 int BM, int ntiles_n, TileTable& tt) {
+                                                 int BM, int ntiles_n, TileTable& tt, int zip = 0) {
     pdl_wait();
     pdl_release();
     const int G = E + sh.S;
@@ -63,6 +71,21 @@ __device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ off
             tt.crow[g] = sh.crow0 + s * sh.rows;
             tt.rows[g] = sh.rows;
         }
+        tt.mtiles[g] = (tt.rows[g] + BM - 1) / BM;
+    }
+    __syncthreads();
+    // walk rank of each group
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+        int r = g;
+        if (zip > 0 && g < E) {
+            const int mg = tt.mtiles[g];
+            r = 0;
+            for (int h = 0; h < E; ++h) {
+                const int mh = tt.mtiles[h];
+                r += (mh > mg || (mh == mg && h < g)) ? 1 : 0;
+            }
+        }
+        tt.order[r] = g;
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -72,13 +95,8 @@ __device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ off
         int sum = 0;
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-            const int g = lane * PER + i;
-            int mt = 0;
-            if (g < G) {
-                mt = (tt.rows[g] + BM - 1) / BM;
-                tt.mtiles[g] = mt;
-            }
-            tl[i] = mt * ntiles_n;
+            const int r = lane * PER + i;
+            tl[i] = (r < G) ? tt.mtiles[tt.order[r]] * ntiles_n : 0;
             sum += tl[i];
         }
         int incl = sum;
@@ -90,14 +108,17 @@ __device__ __forceinline__ void build_tile_table(const int32_t* __restrict__ off
         int run = incl - sum;
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-            const int g = lane * PER + i;
-            if (g < G) tt.start[g] = run;
+            const int r = lane * PER + i;
+            if (r < G) tt.start[r] = run;
             run += tl[i];
         }
         if (lane == 31) tt.start[G] = incl;
     }
     __syncthreads();
-    if (threadIdx.x == 0) tt.routed_tiles = tt.start[E];
+    if (threadIdx.x == 0) {
+        tt.routed_tiles = tt.start[E];
+        tt.zip = zip;
+    }
     __syncthreads();
 }
 
@@ -105,30 +126,63 @@ struct TileCoord {
     int e, mt, nt;   // e: group (routed expert, or E + shared expert)
 };
 
-// Position t of the walk -> tile.  With both routed and shared groups the
-// walk interleaves them in proportion (position t is routed tile
-// floor(t*Rt/N) when that count steps at t, else shared tile t - that
-// count; a bijection since Rt <= N), so the CTAs running at any moment mix
-// routed tiles, which stream their weight panels from HBM, with shared
-// tiles, whose panels stay in L2 across their many M tiles.
+// Position t of the walk -> tile.
+//
+// With both routed and shared groups the walk interleaves them in
+// proportion (position t is routed tile floor(t*Rt/N) when that count steps
+// at t, else shared tile t - that count; a bijection since Rt <= N), so the
+// CTAs running at any moment mix routed tiles, which stream their weight
+// panels from HBM, with shared tiles, whose panels stay in L2 across their
+// many M tiles.
+//
+// With tt.zip > 0 the routed positions alternate between the two ends of
+// the size-ranked tile list: "front" positions take tiles 0, 1, 2, ... (the
+// largest groups, whose weight panels serve many M tiles from L2), "back"
+// positions take tiles Rt-1, Rt-2, ... (the smallest groups, each tile
+// streaming its own panel from HBM).  So at any moment about half the CTAs
+// compute from L2 while the others stream weights, instead of a phase of
+// pure compute followed by a phase bound by HBM.  A position u of wave
+// w = u / zip is a front one when u + w is even (zip even) or u is even
+// (zip odd), so each CTA (position u mod zip) alternates between the two
+// ends from wave to wave.  Front index = front positions before u; back
+// index = the others; the two ranges meet in the middle: a bijection.
 __device__ __forceinline__ TileCoord decode_tile(const TileTable& tt, int G, int t) {
     const int total = tt.start[G], rt = tt.routed_tiles;
+    bool routed = true;
     if (rt > 0 && rt < total) {
         const int r0 = int((long long)t * rt / total);
         const int r1 = int((long long)(t + 1) * rt / total);
-        t = (r1 > r0) ? r0 : rt + (t - r0);
+        routed = r1 > r0;
+        t = routed ? r0 : rt + (t - r0);
+    } else if (rt == 0) {
+        routed = false;
     }
-    int lo = 0, hi = G - 1;   // last g with start[g] <= t (groups with no tiles are skipped)
+    if (routed && tt.zip > 0) {
+        const int Z = tt.zip;
+        const int u = t;
+        int front_before;   // front positions in [0, u)
+        bool front;
+        if (Z & 1) {
+            front = (u & 1) == 0;
+            front_before = (u + 1) >> 1;
+        } else {
+            const int w = u / Z, c = u - w * Z;
+            front = ((c + w) & 1) == 0;
+            front_before = w * (Z >> 1) + ((w & 1) ? (c >> 1) : ((c + 1) >> 1));
+        }
+        t = front ? front_before : rt - 1 - (u - front_before);
+    }
+    int lo = 0, hi = G - 1;   // last rank r with start[r] <= t (groups with no tiles are skipped)
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (tt.start[mid] <= t) lo = mid; else hi = mid - 1;
     }
-    // groups without tiles have start[g] == start[g+1], so the last g with
-    // start[g] <= t is the one whose range [start[g], start[g+1]) holds t
+    // groups without tiles have start[r] == start[r+1], so the last rank with
+    // start[r] <= t is the one whose range [start[r], start[r+1]) holds t
     TileCoord c;
-    c.e = lo;
+    c.e = tt.order[lo];
     const int local = t - tt.start[lo];
-    const int mt = tt.mtiles[lo];
+    const int mt = tt.mtiles[c.e];
     c.nt = local / mt;
     c.mt = local - c.nt * mt;
     return c;
@@ -154,6 +208,8 @@ constexpr int kTcBM = 128;
 constexpr int kTcBK = 64;            // 64 bf16 = 128 B = one swizzle row
 constexpr int kTcEpiWarps = 8;
 constexpr int kTcThreads = 64 + 32 * kTcEpiWarps;
+// threads of the single-CTA kernel with EPIW epilogue warps
+constexpr int tc_threads(int epiw) { return 64 + 32 * epiw; }
 
 template <int BN, int STAGES>
 struct TcCfg {
@@ -165,15 +221,81 @@ struct TcCfg {
     static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;   // + alignment slack
 };
 
-// tmA2 / tmB2 / bias2: the shared experts' A rows and parameters (used when sh.S > 0)
-template <int BN, int STAGES, int MODE>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// One warp's share of a tile's epilogue.  The warp reads TMEM lane quarter
+// q (accumulator rows q*32 .. q*32+31, one per lane) and the 32-column
+// chunks sub, sub + EPIW/4, ... of the BN-column accumulator at `tacc`.  It
+// loads its chunks in groups of at most two (64 registers), waits once per
+// group, and calls release() (the warp's arrival on the accumulator's
+// "empty" barrier) as soon as its last group is in registers, so the MMA
+// can start the next-but-one tile while this one is still being written.
+// Then bias (from global memory: the same 16 bytes for every lane, a
+// broadcast), GELU (fc1) or the row gate (fc2), bf16 rounding and 16-byte
+// stores to row `crow` of C (skipped for rows past the group, `valid`).
+template <int BN, int MODE, int EPIW, typename Release>
+__device__ __forceinline__ void epilogue_tile_warp(uint32_t tacc, int q, int sub, int lane, bool valid, size_t crow,
+                                                   int n0, int N, float g, const __nv_bfloat16* __restrict__ bb,
+                                                   __nv_bfloat16* __restrict__ C, Release release) {
+    constexpr int kSub = EPIW / 4;
+    constexpr int kChunks = (BN / 32 + kSub - 1) / kSub;   // chunks per warp (the last may be past BN)
+    constexpr int kGroup = kChunks < 2 ? kChunks : 2;
+    static_assert(EPIW % 4 == 0 && EPIW >= 4, "whole lane quarters");
+#pragma unroll
+    for (int g0 = 0; g0 < kChunks; g0 += kGroup) {
+        uint32_t r[kGroup][32];
+#pragma unroll
+        for (int j = 0; j < kGroup; ++j) {
+            const int c = sub + (g0 + j) * kSub;
+            if (g0 + j < kChunks && c < BN / 32)   // warp-uniform: the loads are warp-collective
+                tmem_ld_32x32b_x32(tacc + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r[j]);
+        }
+        tmem_ld_wait();
+        if (g0 + kGroup >= kChunks) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) release();
+        }
+#pragma unroll
+        for (int j = 0; j < kGroup; ++j) {
+            const int c = sub + (g0 + j) * kSub;
+            const int nb = n0 + c * 32;
+            if (!(g0 + j < kChunks && c < BN / 32) || !valid || nb >= N) continue;
+            __nv_bfloat16* cp = C + crow * N + nb;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                if (nb + v * 8 >= N) break;
+                // bias[nb + 8v .. +8): one 16-byte load (N % 8 == 0, 16-byte aligned rows)
+                const uint4 bw = __ldg(reinterpret_cast<const uint4*>(bb + nb + v * 8));
+                const uint32_t bwv[4] = {bw.x, bw.y, bw.z, bw.w};
+                float o[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float bi = (i & 1) ? bf16_hi(bwv[i >> 1]) : bf16_lo(bwv[i >> 1]);
+                    const float cval = __uint_as_float(r[j][v * 8 + i]) + bi;
+                    o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
+                }
+                uint4 u;
+                u.x = pack_bf16x2(o[0], o[1]);
+                u.y = pack_bf16x2(o[2], o[3]);
+                u.z = pack_bf16x2(o[4], o[5]);
+                u.w = pack_bf16x2(o[6], o[7]);
+                *reinterpret_cast<uint4*>(cp + v * 8) = u;
+            }
+        }
+    }
+}
+
+// tmA2 / tmB2 / bias2: the shared experts' A rows and parameters (used when sh.S > 0).
+// EPIW epilogue warps (a multiple of 4: EPIW / 4 warps share each TMEM lane
+// quarter and split its 32-column chunks); fc1's GELU epilogue takes 16 so
+// that it keeps up with the main loop at short K.
+template <int BN, int STAGES, int MODE, int EPIW>
+__global__ void __launch_bounds__(tc_threads(EPIW), 1)
 ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const int32_t* __restrict__ offsets, int E, int N, int K,
                    const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
                    const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C, SharedGroups sh,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                   const __nv_bfloat16* __restrict__ bias2) {
+                   const __nv_bfloat16* __restrict__ bias2, int walk_zip) {
     using Cfg = TcCfg<BN, STAGES>;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN: whole 32-column epilogue chunks, MMA N <= 256");
     __shared__ TileTable tt;
@@ -181,7 +303,6 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
-    __shared__ float sbias[BN];
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
 
@@ -193,7 +314,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], kTcEpiWarps);   // one arrival per epilogue warp
+            mbar_init(&tempty_bar[a], EPIW);   // one arrival per epilogue warp
         }
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
@@ -211,7 +332,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         tc_fence_before();
     }
     const int ntn = (N + BN - 1) / BN;
-    build_tile_table(offsets, E, sh, kTcBM, ntn, tt);   // contains __syncthreads()
+    build_tile_table(offsets, E, sh, kTcBM, ntn, tt, walk_zip ? int(gridDim.x) : 0);   // ends with __syncthreads()
     tc_fence_after();
     const uint32_t tmem_base = tmem_slot;
     const int G = E + sh.S;
@@ -250,10 +371,7 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             // (immediate on the normal path, where the MMA consumed them)
             for (int s = 0; s < STAGES; ++s) {
                 if (last_parity[s] < 0) continue;
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(&full_bar[s], uint32_t(last_parity[s])) &&
-                       globaltimer_ns() - t0 < kWaitLimitNs) {
-                }
+                mbar_wait_drain(&full_bar[s], uint32_t(last_parity[s]));
             }
         }
     } else if (warp == 1) {
@@ -289,22 +407,20 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             }
             // every MMA this thread issued completes before TMEM is released
             umma_commit(&drain_bar);
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-            }
+            mbar_wait_drain(&drain_bar, 0);
         }
     } else {
-        // ---------------- epilogue (warps 2..9) ----------------
-        const int etid = threadIdx.x - 64;   // 0..255
-        const int q = warp & 3;              // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;    // which alternate 32-column chunks
+        // ---------------- epilogue (warps 2 .. 1+EPIW) ----------------
+        // Warp w takes TMEM lane quarter w % 4 and every (EPIW/4)-th
+        // 32-column chunk from (w - 2) / 4 (epilogue_tile_warp).  Each warp
+        // leaves the tile loop on its own when a wait gives up or the abort
+        // flag is raised; no named barrier is involved.
+        const int q = warp & 3;
+        const int sub = (warp - 2) >> 2;
         int acc = 0;
         uint32_t acc_phase = 0;
-        bool failed = false;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            // all epilogue warps stop together once any wait has given up, so
-            // none is left behind at a named barrier
-            if (named_bar_red_or(1, 32 * kTcEpiWarps, failed || *abort_p)) break;
+            if (*abort_p) break;
             const TileCoord tc = decode_tile(tt, G, t);
             const bool shared_g = tc.e >= E;
             const int rows = tt.rows[tc.e];
@@ -314,49 +430,15 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             // destination row: the grouped row, or (direct output of a routed
             // group) the row out_rows names
             const size_t crow = (out_rows != nullptr && valid && !shared_g) ? size_t(out_rows[grow]) : grow;
-            const int n0 = tc.nt * BN;
             float g = 1.f;   // shared experts are ungated
             if (MODE == kFc2Gate && row_gate != nullptr && valid && !shared_g) g = row_gate[grow];
             const __nv_bfloat16* bb = shared_g ? bias2 + size_t(tc.e - E) * N : bias + size_t(tc.e) * N;
-            // (the barrier above also ends every read of the previous tile's bias)
-            for (int i = etid; i < BN; i += 32 * kTcEpiWarps)
-                sbias[i] = (n0 + i < N) ? __bfloat162float(bb[n0 + i]) : 0.f;
-            named_bar_sync(1, 32 * kTcEpiWarps);   // this tile's bias is visible
-            // (uniform per warp: the TMEM loads below are warp-collective)
-            if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_p))) {
-                failed = true;
-                continue;
-            }
+            // (uniform per warp: the TMEM loads are warp-collective)
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_p))) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = half; c < BN / 32; c += 2) {
-                uint32_t r[32];
-                __syncwarp();
-                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
-                tmem_ld_wait();
-                const int nb = n0 + c * 32;
-                if (!valid || nb >= N) continue;
-                __nv_bfloat16* cp = C + crow * N + nb;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    if (nb + v * 8 >= N) break;
-                    float o[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float cval = __uint_as_float(r[v * 8 + i]) + sbias[c * 32 + v * 8 + i];
-                        o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
-                    }
-                    uint4 u;
-                    u.x = pack_bf16x2(o[0], o[1]);
-                    u.y = pack_bf16x2(o[2], o[3]);
-                    u.z = pack_bf16x2(o[4], o[5]);
-                    u.w = pack_bf16x2(o[6], o[7]);
-                    *reinterpret_cast<uint4*>(cp + v * 8) = u;
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+            uint64_t* tempty = &tempty_bar[acc];
+            epilogue_tile_warp<BN, MODE, EPIW>(tmem_base + uint32_t(acc * BN), q, sub, lane, valid, crow, tc.nt * BN, N,
+                                               g, bb, C, [tempty]() { mbar_arrive(tempty); });
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
@@ -417,7 +499,7 @@ ffn_tc_f32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const float* __restrict__ bias, const float* __restrict__ row_gate,
                     const int32_t* __restrict__ out_rows, float* __restrict__ C, SharedGroups sh,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                    const float* __restrict__ bias2) {
+                    const float* __restrict__ bias2, int walk_zip) {
     using Cfg = TfCfg<BN, STAGES>;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN: whole 32-column epilogue chunks, MMA N <= 256");
     __shared__ TileTable tt;
@@ -456,7 +538,7 @@ ffn_tc_f32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tc_fence_before();
     }
     const int ntn = (N + BN - 1) / BN;
-    build_tile_table(offsets, E, sh, kTcBM, ntn, tt);   // contains __syncthreads()
+    build_tile_table(offsets, E, sh, kTcBM, ntn, tt, walk_zip ? int(gridDim.x) : 0);   // ends with __syncthreads()
     tc_fence_after();
     const uint32_t tmem_base = tmem_slot;
     const int G = E + sh.S;
@@ -493,10 +575,7 @@ ffn_tc_f32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
             for (int s = 0; s < STAGES; ++s) {
                 if (last_parity[s] < 0) continue;
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(&full_bar[s], uint32_t(last_parity[s])) &&
-                       globaltimer_ns() - t0 < kWaitLimitNs) {
-                }
+                mbar_wait_drain(&full_bar[s], uint32_t(last_parity[s]));
             }
         }
     } else if (warp == 1) {
@@ -536,9 +615,7 @@ ffn_tc_f32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (acc == 0) acc_phase ^= 1u;
             }
             umma_commit(&drain_bar);
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-            }
+            mbar_wait_drain(&drain_bar, 0);
         }
     } else if (warp >= 2 + kTcEpiWarps) {
         // ---------------- converters (warps 10..17) ----------------
@@ -660,14 +737,14 @@ struct Tc2Cfg {
     static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
 };
 
-template <int STAGES, int MODE>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int STAGES, int MODE, int EPIW>
+__global__ void __launch_bounds__(tc_threads(EPIW), 1)
 ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const int32_t* __restrict__ offsets, int E, int N, int K,
                     const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
                     const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C, SharedGroups sh,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                    const __nv_bfloat16* __restrict__ bias2) {
+                    const __nv_bfloat16* __restrict__ bias2, int walk_zip) {
     using Cfg = Tc2Cfg<STAGES>;
     constexpr int BN = kTc2BN;
     __shared__ TileTable tt;
@@ -675,7 +752,6 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     __shared__ __align__(8) uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
-    __shared__ float sbias[BN];
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
 
@@ -689,7 +765,7 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], 2 * kTcEpiWarps);   // CTA 0's copy: every epilogue warp of the pair
+            mbar_init(&tempty_bar[a], 2 * EPIW);   // CTA 0's copy: every epilogue warp of the pair
         }
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
@@ -707,7 +783,7 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tc_fence_before();
     }
     const int ntn = (N + BN - 1) / BN;
-    build_tile_table(offsets, E, sh, kTc2BM, ntn, tt);   // contains __syncthreads()
+    build_tile_table(offsets, E, sh, kTc2BM, ntn, tt, walk_zip ? npairs : 0);   // ends with __syncthreads()
     cluster_sync();   // both CTAs' barriers are initialised before any cross-CTA arrive
     tc_fence_after();
     const uint32_t tmem_base = tmem_slot;
@@ -776,15 +852,16 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             umma_commit_pair(&drain_bar, 0x3);
         }
     } else {
-        // ---------------- epilogue (warps 2..9 of each CTA) ----------------
-        const int etid = threadIdx.x - 64;   // 0..255
-        const int q = warp & 3;              // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;    // which alternate 32-column chunks
+        // ---------------- epilogue (warps 2 .. 1+EPIW of each CTA) ----------------
+        // As in ffn_tc_bf16_kernel: each CTA's warps read their own 128
+        // accumulator rows (the tile's rows 128*rank ..); every warp of the
+        // pair arrives on CTA 0's "empty" barrier (CTA 1 through mapa).
+        const int q = warp & 3;
+        const int sub = (warp - 2) >> 2;
         int acc = 0;
         uint32_t acc_phase = 0;
-        bool failed = false;
         for (int t = pair; t < total; t += npairs) {
-            if (named_bar_red_or(1, 32 * kTcEpiWarps, failed || *abort_p)) break;
+            if (*abort_p) break;
             const TileCoord tc = decode_tile(tt, G, t);
             const bool shared_g = tc.e >= E;
             const int rows = tt.rows[tc.e];
@@ -792,51 +869,18 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const bool valid = r_in < rows;
             const size_t grow = size_t(tt.crow[tc.e]) + r_in;
             const size_t crow = (out_rows != nullptr && valid && !shared_g) ? size_t(out_rows[grow]) : grow;
-            const int n0 = tc.nt * BN;
             float g = 1.f;
             if (MODE == kFc2Gate && row_gate != nullptr && valid && !shared_g) g = row_gate[grow];
             const __nv_bfloat16* bb = shared_g ? bias2 + size_t(tc.e - E) * N : bias + size_t(tc.e) * N;
-            for (int i = etid; i < BN; i += 32 * kTcEpiWarps)
-                sbias[i] = (n0 + i < N) ? __bfloat162float(bb[n0 + i]) : 0.f;
-            named_bar_sync(1, 32 * kTcEpiWarps);
-            // (uniform per warp: the TMEM loads below are warp-collective)
-            if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_p))) {
-                failed = true;
-                continue;
-            }
+            // (uniform per warp: the TMEM loads are warp-collective)
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_p))) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = half; c < BN / 32; c += 2) {
-                uint32_t r[32];
-                __syncwarp();
-                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + c * 32), r);
-                tmem_ld_wait();
-                const int nb = n0 + c * 32;
-                if (!valid || nb >= N) continue;
-                __nv_bfloat16* cp = C + crow * N + nb;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    if (nb + v * 8 >= N) break;
-                    float o[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float cval = __uint_as_float(r[v * 8 + i]) + sbias[c * 32 + v * 8 + i];
-                        o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
-                    }
-                    uint4 u;
-                    u.x = pack_bf16x2(o[0], o[1]);
-                    u.y = pack_bf16x2(o[2], o[3]);
-                    u.z = pack_bf16x2(o[4], o[5]);
-                    u.w = pack_bf16x2(o[6], o[7]);
-                    *reinterpret_cast<uint4*>(cp + v * 8) = u;
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (rank == 0) mbar_arrive(&tempty_bar[acc]);
-                else mbar_arrive_remote(&tempty_bar[acc], 0);
-            }
+            uint64_t* tempty = &tempty_bar[acc];
+            epilogue_tile_warp<BN, MODE, EPIW>(tmem_base + uint32_t(acc * BN), q, sub, lane, valid, crow, tc.nt * BN, N,
+                                               g, bb, C, [tempty, rank]() {
+                                                   if (rank == 0) mbar_arrive(tempty);
+                                                   else mbar_arrive_remote(tempty, 0);
+                                               });
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
@@ -846,9 +890,7 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     // memory and writes both tensor memories) before either CTA frees
     // anything or exits
     if (warp == 1 && lane == 0) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_wait_drain(&drain_bar, 0);
     }
     __syncthreads();
     cluster_sync();

@@ -231,6 +231,28 @@ bool pair_tiles_enabled(bool heuristic) {
     return forced < 0 ? heuristic : forced == 1;
 }
 
+// fc1 on CTA pairs as well: the heuristic's choice unless MOE_FC1_PAIRS is
+// "0" (never) or "1" (always)
+bool fc1_pair_tiles_enabled(bool heuristic) {
+    static const int forced = []() {
+        const char* v = std::getenv("MOE_FC1_PAIRS");
+        if (v == nullptr || *v == 0) return -1;
+        return v[0] == '0' ? 0 : 1;
+    }();
+    return forced < 0 ? heuristic : forced == 1;
+}
+
+// Hot/cold interleaved tile walk in the grouped FFN (decode_tile): the
+// heuristic's choice unless MOE_TILE_ZIP is "0" (never) or "1" (always)
+bool tile_zip_enabled(bool heuristic) {
+    static const int forced = []() {
+        const char* v = std::getenv("MOE_TILE_ZIP");
+        if (v == nullptr || *v == 0) return -1;
+        return v[0] == '0' ? 0 : 1;
+    }();
+    return forced < 0 ? heuristic : forced == 1;
+}
+
 int num_sms() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -267,6 +289,10 @@ int check_reroute(int k, int E, int F) {
 // bf16 tensor-core GEMM tile: 128 x 256 (the widest single-CTA MMA; narrower
 // tiles measured slower on every workload: more A re-reads per FLOP)
 constexpr int kTcBN = 256, kTcStages = 4;
+// fc1's GELU epilogue runs on 16 warps (four per TMEM lane quarter) so that
+// it keeps pace with the main loop at short K; fc2's bias-and-gate epilogue
+// needs only 8
+constexpr int kTcFc1EpiWarps = 16;
 // Scratch of a rerouting dispatch (F rounds, nchunk chunks).
 struct RerouteWs {
     int32_t* srv;     // [T*k]
@@ -626,23 +652,23 @@ long long ffn_tiles_ub(int routed_rows_ub, int E, const SharedArgs& sa, int BM, 
 // Routed groups: E experts over rows offsets[0..E] of `a` (a_rows rows;
 // routed_rows_ub bounds offsets[E]).  E may be 0 when only shared groups run.
 
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, int EPIW = kTcEpiWarps>
 int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
               const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
-              const SharedArgs& sa, int kernel_id, cudaStream_t s) {
+              const SharedArgs& sa, int kernel_id, cudaStream_t s, bool zip = false) {
     FfnMaps mp;
     if (!make_ffn_maps(mp, a, a_cols, a_rows, w, N, E, sa, kTcBM, BN, MOE_BF16)) return MOE_ERR_UNSUPPORTED;
-    auto kern = ffn_tc_bf16_kernel<BN, STAGES, MODE>;
+    auto kern = ffn_tc_bf16_kernel<BN, STAGES, MODE, EPIW>;
     const size_t smem = TcCfg<BN, STAGES>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     const long long tiles_ub = ffn_tiles_ub(routed_rows_ub, E, sa, kTcBM, N, BN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, s, mp.a, mp.b, offsets, E, N, a_cols,
+    launch_err = launch_pdl(kern, dim3(grid), dim3(tc_threads(EPIW)), smem, s, mp.a, mp.b, offsets, E, N, a_cols,
                             static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
                             static_cast<__nv_bfloat16*>(c), sa.g, mp.a2, mp.b2,
-                            static_cast<const __nv_bfloat16*>(sa.bias));
+                            static_cast<const __nv_bfloat16*>(sa.bias), zip ? 1 : 0);
     return L.finish(launch_err);
 }
 
@@ -650,23 +676,23 @@ int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const v
 // rows, weight map boxes of 128 rows (half of the tile's N).
 constexpr int kTc2Stages = 6;
 
-template <int MODE>
+template <int MODE, int EPIW = kTcEpiWarps>
 int launch_tc2(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
                const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
-               const SharedArgs& sa, int kernel_id, cudaStream_t s) {
+               const SharedArgs& sa, int kernel_id, cudaStream_t s, bool zip = false) {
     FfnMaps mp;
     if (!make_ffn_maps(mp, a, a_cols, a_rows, w, N, E, sa, 128, kTc2BN / 2, MOE_BF16)) return MOE_ERR_UNSUPPORTED;
-    auto kern = ffn_tc2_bf16_kernel<kTc2Stages, MODE>;
+    auto kern = ffn_tc2_bf16_kernel<kTc2Stages, MODE, EPIW>;
     const size_t smem = Tc2Cfg<kTc2Stages>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     const long long tiles_ub = ffn_tiles_ub(routed_rows_ub, E, sa, kTc2BM, N, kTc2BN);
     const int pairs = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms() / 2)));
     Launch L(kernel_id, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl_cluster(kern, dim3(2 * pairs), dim3(kTcThreads), smem, 2, s, mp.a, mp.b, offsets, E, N,
+    launch_err = launch_pdl_cluster(kern, dim3(2 * pairs), dim3(tc_threads(EPIW)), smem, 2, s, mp.a, mp.b, offsets, E, N,
                                     a_cols, static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
                                     static_cast<__nv_bfloat16*>(c), sa.g, mp.a2, mp.b2,
-                                    static_cast<const __nv_bfloat16*>(sa.bias));
+                                    static_cast<const __nv_bfloat16*>(sa.bias), zip ? 1 : 0);
     return L.finish(launch_err);
 }
 
@@ -676,7 +702,7 @@ constexpr int kTfBN = 128, kTfStages = 3;
 template <int MODE>
 int launch_tf32x3(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
                   const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
-                  const SharedArgs& sa, int kernel_id, cudaStream_t s) {
+                  const SharedArgs& sa, int kernel_id, cudaStream_t s, bool zip = false) {
     FfnMaps mp;
     if (!make_ffn_maps(mp, a, a_cols, a_rows, w, N, E, sa, kTcBM, kTfBN, MOE_F32)) return MOE_ERR_UNSUPPORTED;
     auto kern = ffn_tc_f32x3_kernel<kTfBN, kTfStages, MODE>;
@@ -688,7 +714,7 @@ int launch_tf32x3(const void* a, int a_cols, int a_rows, int routed_rows_ub, con
     cudaError_t launch_err;
     launch_err = launch_pdl(kern, dim3(grid), dim3(kTfThreads), smem, s, mp.a, mp.b, offsets, E, N, a_cols,
                             static_cast<const float*>(bias), row_gate, out_rows, static_cast<float*>(c), sa.g, mp.a2,
-                            mp.b2, static_cast<const float*>(sa.bias));
+                            mp.b2, static_cast<const float*>(sa.bias), zip ? 1 : 0);
     return L.finish(launch_err);
 }
 
@@ -725,7 +751,8 @@ bool fc2_narrow_tiles(int max_rows, int E, int N, const SharedExperts& se) {
 // average enough rows that the doubled M tile wastes little
 int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, int ff, const void* w1,
             const void* b1, const void* w2, const void* b2, const float* row_gate, void* h, void* yp, int dtype,
-            const int32_t* out_rows, const SharedExperts& se, bool use_pairs, cudaStream_t s) {
+            const int32_t* out_rows, const SharedExperts& se, bool use_pairs, cudaStream_t s,
+            bool fc1_pairs = false) {
     const int h_rows = max_rows + se.S * se.T;
     SharedArgs s1, s2;
     if (se.S > 0) {
@@ -742,31 +769,37 @@ int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, 
         s2.bias = se.b2;
         s2.g = SharedGroups{se.S, se.T, max_rows, se.T, max_rows};
     }
+    const bool zip = tile_zip_enabled(false);
     int rc;
     if (dtype == MOE_BF16) {
         // fc1 stays on single-CTA 128-row tiles: its K (= d) is short, so the
         // pair kernel's doubled M padding costs more than its halved loads
         // save (measured on the skewed and large workloads)
-        rc = launch_tc<kTcBN, kTcStages, kFc1Gelu>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr,
-                                                   nullptr, h, s1, MOE_KERNEL_FFN1, s);
+        if (fc1_pairs)
+            rc = launch_tc2<kFc1Gelu, kTcFc1EpiWarps>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr,
+                                                      nullptr, h, s1, MOE_KERNEL_FFN1, s, zip);
+        else
+            rc = launch_tc<kTcBN, kTcStages, kFc1Gelu, kTcFc1EpiWarps>(xp, d, max_rows, max_rows, w1, ff, E,
+                                                                       offsets, b1, nullptr, nullptr, h, s1,
+                                                                       MOE_KERNEL_FFN1, s, zip);
         if (rc != MOE_OK) return rc;
         if (use_pairs)
             return launch_tc2<kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, s2,
-                                        MOE_KERNEL_FFN2, s);
+                                        MOE_KERNEL_FFN2, s, zip);
         // fc2 of a layer with about one M tile per expert (switch-top1: 96
         // tiles of 256 columns for 148 SMs): 192-column tiles put 4/3 as many
         // SMs on the weight stream
         if (fc2_narrow_tiles(max_rows, E, d, se))
             return launch_tc<kTcBNNarrow, kTcStagesNarrow, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2,
-                                                                     row_gate, out_rows, yp, s2, MOE_KERNEL_FFN2, s);
+                                                                     row_gate, out_rows, yp, s2, MOE_KERNEL_FFN2, s, zip);
         return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate,
-                                                     out_rows, yp, s2, MOE_KERNEL_FFN2, s);
+                                                     out_rows, yp, s2, MOE_KERNEL_FFN2, s, zip);
     }
     rc = launch_tf32x3<kFc1Gelu>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, s1,
-                                 MOE_KERNEL_FFN1, s);
+                                 MOE_KERNEL_FFN1, s, zip);
     if (rc != MOE_OK) return rc;
     return launch_tf32x3<kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, s2,
-                                   MOE_KERNEL_FFN2, s);
+                                   MOE_KERNEL_FFN2, s, zip);
 }
 
 // Dispatch of the fused forward path from the router's per-chunk histograms
@@ -1328,8 +1361,9 @@ int moe_forward_ex(const void* x, const void* w_router, const float* logit_bias,
     // CTA pairs once the routed experts average at least 384 rows (256-row
     // tiles then waste little on padding) or env MOE_PAIR_TILES forces it
     const bool use_pairs = pair_tiles_enabled(static_cast<long long>(A) >= 384ll * E);
+    const bool fc1_pairs = fc1_pair_tiles_enabled(false);
     if ((rc = run_ffn(xp, offsets, A, E, d, ff, w1, b1, w2, b2, row_gate, h, direct ? out : yp, dtype,
-                      direct ? perm : nullptr, se, use_pairs, s)) != MOE_OK)
+                      direct ? perm : nullptr, se, use_pairs, s, fc1_pairs)) != MOE_OK)
         return rc;
     if (!direct) {
         const void* ys = static_cast<const uint8_t*>(yp) + size_t(A) * d * elem_bytes(dtype);

@@ -290,9 +290,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
             for (int i = 0; i < S; ++i) {
                 if (last_parity[i] < 0) continue;
-                const uint64_t w0 = globaltimer_ns();
-                while (!mbar_try_wait(&full_bar[i], uint32_t(last_parity[i])) && globaltimer_ns() - w0 < kWaitLimitNs) {
-                }
+                mbar_wait_drain(&full_bar[i], uint32_t(last_parity[i]));
             }
         }
     } else if (warp == 1) {
@@ -315,9 +313,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
             umma_commit(&done_bar);   // tracks every MMA issued above
             // TMEM is released only after those MMAs complete (bounded wait)
-            const uint64_t w0 = globaltimer_ns();
-            while (!mbar_try_wait(&done_bar, 0) && globaltimer_ns() - w0 < kWaitLimitNs) {
-            }
+            mbar_wait_drain(&done_bar, 0);
         }
     } else {
         const int ew = warp - 2;      // 0..3
