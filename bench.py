@@ -161,14 +161,24 @@ KERNEL_SOURCES = {
     "router": ["router.cuh", "common.cuh"], "combine": ["dispatch.cuh", "common.cuh"],
     "gather": ["dispatch.cuh", "common.cuh"], "permute": ["dispatch.cuh", "common.cuh"],
 }
+# fp32 layers run the grouped FFN in ffn_f32.cuh (which builds on ffn.cuh)
+KERNEL_SOURCES_F32 = {"ffn1": ["ffn_f32.cuh", "ffn.cuh", "common.cuh"],
+                      "ffn2": ["ffn_f32.cuh", "ffn.cuh", "common.cuh"]}
 
 
-def kernel_source_hash(kernel: str) -> str:
+def kernel_source_hash(kernel: str, dtype: str = "bf16") -> str:
+    """Hash of the sources of one kernel of the layer (for dtype's path)."""
+    files = (KERNEL_SOURCES_F32 if dtype == "f32" else {}).get(kernel, KERNEL_SOURCES.get(kernel, []))
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES.get(kernel, []):
+    for f in files:
         with open(os.path.join(ROOT, "mixture_experts_layer_45_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def tag_dtype(workload_tag: str) -> str:
+    """The dtype named in a workload tag (<name>-<dtype>-cf<..>)."""
+    return "f32" if "-f32-" in workload_tag else "bf16"
 
 
 def committed_traffic(kernel: str, workload_tag: str):
@@ -179,7 +189,7 @@ def committed_traffic(kernel: str, workload_tag: str):
     text = open(p).read()
     m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
     s = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    if not m or not s or s.group(1) != kernel_source_hash(kernel):
+    if not m or not s or s.group(1) != kernel_source_hash(kernel, tag_dtype(workload_tag)):
         return None
     return float(m.group(1))
 

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "dispatch.cuh"
 #include "ffn.cuh"
+#include "ffn_f32.cuh"
 #include "router.cuh"
 
 using namespace moe;

@@ -61,16 +61,16 @@ def test_committed_profiles_are_current():
         h = re.search(r"source_hash:\s*([0-9a-f]+)", text)
         if not h:
             continue
-        kernel = name.split("_", 1)[0]
-        assert h.group(1) == bench.kernel_source_hash(kernel), name
+        kernel, tag = name[:-3].split("_", 1)
+        assert h.group(1) == bench.kernel_source_hash(kernel, bench.tag_dtype(tag)), name
         assert re.search(r"dram_bytes_per_launch:\s*[0-9]+", text), name
         checked += 1
     assert checked >= 8
 
 
 def test_traffic_is_read_for_the_bench_workload():
-    w = wl.workload("switch-top1")
-    assert bench.committed_traffic("ffn1", bench.workload_tag(w)) == 164175104.0
+    w = wl.workload("large-top2")                  # the bench's default workload
+    assert bench.committed_traffic("ffn1", bench.workload_tag(w)) == 1538235640.0
     assert bench.committed_traffic("ffn1", "no-such-workload") is None
 
 
