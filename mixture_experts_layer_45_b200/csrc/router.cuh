@@ -202,27 +202,48 @@ router_topk_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr, const 
 }
 
 // ===========================================================================
-// bf16 router on the tensor cores.  One CTA per 128-token tile, 192 threads:
+// bf16 router on the tensor cores.  One CTA per 128-token tile, 320 threads:
 //   warp 0      TMA producer: x tile rows [t0, t0+128) and W_r, 64 columns of
 //               K per stage (128B swizzle; rows past T and experts past E
-//               are zero-filled by the tensor maps)
+//               are zero-filled by the tensor maps); as many stages as fit
 //   warp 1      TMEM allocator and MMA issuer: logits[128 x EP] in fp32
-//   warps 2..5  epilogue, thread = token: +bias, online max/sum over 32-column
-//               TMEM loads, register top-k (ties to the lower index), gates,
-//               then the per-expert probability column sums (shared-memory
-//               transpose, fixed summation order) and the expert histogram
+//   warps 2..9  epilogue, two warps per TMEM lane quarter, thread = token:
+//               for E <= 64 each of the two takes one 32-expert chunk of its
+//               32 tokens' logits (+ bias from shared memory), its local max,
+//               exponentials, sum and top-k; the two exchange those through
+//               shared memory and merge them (softmax of the whole row, top-k
+//               with ties to the lower index); then each warp's share of the
+//               per-expert probability column sums (a shared-memory transpose,
+//               fixed summation order) and the expert histogram.  For E > 64
+//               warps 2..5 make two passes over all the chunks.
+// Once the last MMA has completed the pipeline stages are free, and the
+// epilogue uses them as scratch (the exchange records and the transposes).
 // ===========================================================================
 constexpr int kRtBM = 128;
-constexpr int kRtThreads = 192;
+constexpr int kRtEpiWarps = 8;
+constexpr int kRtThreads = 64 + 32 * kRtEpiWarps;
+// dynamic shared memory the stages may take, leaving room for the static
+// arrays (< 4 KB) below the 227 KB a CTA can have
+constexpr size_t kRtDynBudget = 227u * 1024u - 4096u;
 
 template <int EP>
 struct RtCfg {
     static constexpr uint32_t kABytes = kRtBM * 64 * 2;
     static constexpr uint32_t kBBytes = EP * 64 * 2;
     static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = (EP <= 64) ? 8 : (EP <= 128 ? 6 : 4);
+    static constexpr int kFit = int((kRtDynBudget - 1024) / kStageBytes);
+    static constexpr int kStages = kFit < 12 ? kFit : 12;
     static constexpr uint32_t kTmemCols = EP < 32 ? 32 : EP;
     static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024;
+    static_assert(kStages >= 4, "at least four stages");
+};
+
+// per-row record one epilogue warp hands to its partner (E <= 64)
+template <int KMAX>
+struct RtRec {
+    float m, s;          // chunk max logit, sum of exp(logit - m)
+    float v[KMAX];       // chunk top-KMAX logits, largest first
+    int ix[KMAX];        // their expert indices (ties: lower index first)
 };
 
 // KMAX >= k + F: the selection also yields the F fallback experts (fb_idx /
@@ -240,8 +261,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
     __shared__ int s_hist[EP];
-    __shared__ float s_col[4][NCH * 32];     // per-warp column sums of the probabilities
-    __shared__ float s_tr[4][32][33];        // per-warp 32 x 32 transpose
+    __shared__ float s_bias[EP];
+    __shared__ float s_col[4][NCH * 32];     // per lane quarter: column sums of the probabilities
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
 
@@ -288,10 +309,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 last_parity[stage] = int(phase);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
-            for (int i = 0; i < S; ++i) {
-                if (last_parity[i] < 0) continue;
-                mbar_wait_drain(&full_bar[i], uint32_t(last_parity[i]));
-            }
+            for (int i = 0; i < S; ++i)
+                if (last_parity[i] >= 0) mbar_wait_drain(&full_bar[i], uint32_t(last_parity[i]));
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -316,21 +335,25 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             mbar_wait_drain(&done_bar, 0);
         }
     } else {
-        const int ew = warp - 2;      // 0..3
-        const int q = warp & 3;       // TMEM lane quarter
+        const int etid = threadIdx.x - 64;    // 0..255
+        const int q = warp & 3;               // TMEM lane quarter
+        const int c = (warp - 2) >> 2;        // 0: warps 2..5, 1: warps 6..9
         const int row = q * 32 + lane;
         const int t = t0 + row;
         const bool valid = t < T;
+        for (int e = etid; e < EP; e += 32 * kRtEpiWarps) s_bias[e] = (bias != nullptr && e < E) ? bias[e] : 0.f;
+        named_bar_sync(1, 32 * kRtEpiWarps);   // the bias is visible
         const bool ok = mbar_wait(&done_bar, 0, abort_p);
         tc_fence_after();
+        // scratch in the (now idle) pipeline stages: per warp a 32 x 33
+        // transpose tile, then the exchange records [2][128]
+        float* tr = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33);
+        RtRec<KMAX>* rec = reinterpret_cast<RtRec<KMAX>*>(smem + size_t(kRtEpiWarps) * 32 * 33 * sizeof(float));
         if constexpr (NCH <= 2) {
-            // E <= 64: the whole logits row stays in registers, so one
-            // tensor-memory read serves the max, the exponentials (computed
-            // once), the top-k and the probability column sums
-            float l[NCH][32];
+            // ---- one 32-expert chunk per warp ----
+            float l[32];
             float m = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < NCH; ++c) {
+            if (c < NCH) {
                 uint32_t r[32];
                 __syncwarp();
                 tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
@@ -338,58 +361,102 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int e = c * 32 + i;
-                    float v = (e < E && ok) ? __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f) : -INFINITY;
+                    float v = (e < E && ok) ? __uint_as_float(r[i]) + s_bias[e] : -INFINITY;
                     if (v != v) v = -INFINITY;
-                    l[c][i] = v;
+                    l[i] = v;
                     m = fmaxf(m, v);
                 }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) l[i] = -INFINITY;
             }
-            // exponentials and their sum (four partial sums for shorter chains)
+            // exponentials relative to the chunk max and their sum
+            float ex[32];
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float ex = (l[c][i] == -INFINITY) ? 0.f : __expf(l[c][i] - m);
-                    ps[i & 3] += ex;
-                    l[c][i] = ex;   // l now holds the exponentials; the logits order is kept in tv/ti below
-                }
-            const float inv = 1.0f / ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-            // top-k by exponential (monotone in the logit; exact ties keep
-            // the lower index since later equal values do not displace)
+            for (int i = 0; i < 32; ++i) {
+                ex[i] = (l[i] == -INFINITY) ? 0.f : __expf(l[i] - m);
+                ps[i & 3] += ex[i];
+            }
+            const float sc = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            // chunk top-KMAX by logit (largest first; a later equal value does
+            // not displace an earlier one, so ties keep the lower index)
             float tv[KMAX];
             int ti[KMAX];
 #pragma unroll
             for (int j = 0; j < KMAX; ++j) {
-                tv[j] = -1.f;
+                tv[j] = -INFINITY;
                 ti[j] = 0x7fffffff;
             }
 #pragma unroll
-            for (int c = 0; c < NCH; ++c)
+            for (int i = 0; i < 32; ++i) {
+                float v = l[i];
+                int ix = c * 32 + i;
+                if (v == -INFINITY || !(v > tv[KMAX - 1])) continue;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    float v = (c * 32 + i < E) ? l[c][i] : -1.f;
-                    int ix = c * 32 + i;
-                    if (!(v > tv[KMAX - 1])) continue;
-#pragma unroll
-                    for (int j = 0; j < KMAX; ++j) {
-                        if (v > tv[j]) {
-                            const float tf = tv[j];
-                            tv[j] = v;
-                            v = tf;
-                            const int tix = ti[j];
-                            ti[j] = ix;
-                            ix = tix;
-                        }
+                for (int j = 0; j < KMAX; ++j) {
+                    if (v > tv[j]) {
+                        const float tf = tv[j];
+                        tv[j] = v;
+                        v = tf;
+                        const int tix = ti[j];
+                        ti[j] = ix;
+                        ix = tix;
                     }
                 }
-            if (valid && ok) {
+            }
+            // exchange with the partner warp (same lane quarter, other chunk)
+            {
+                RtRec<KMAX>& mine = rec[c * kRtBM + row];
+                mine.m = m;
+                mine.s = sc;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    mine.v[j] = tv[j];
+                    mine.ix[j] = ti[j];
+                }
+            }
+            named_bar_sync(1, 32 * kRtEpiWarps);
+            const RtRec<KMAX>& other = rec[(1 - c) * kRtBM + row];
+            const float mo = other.m;
+            const float M = fmaxf(m, mo);
+            const float f_mine = (m == -INFINITY) ? 0.f : __expf(m - M);
+            const float f_other = (mo == -INFINITY) ? 0.f : __expf(mo - M);
+            const float Ssum = sc * f_mine + other.s * f_other;
+            const float inv = Ssum > 0.f ? 1.0f / Ssum : 0.f;
+            if (c == 0 && valid && ok) {
+                // merge the two sorted lists: chunk 0 holds the lower indices,
+                // so on equal logits it goes first (the heads are compared and
+                // the taken list shifted, keeping every index static)
+                float ov[KMAX];
+                int oi[KMAX];
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    ov[j] = other.v[j];
+                    oi[j] = other.ix[j];
+                }
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j) {
                     if (j < k + F) {
-                        int e = ti[j];
-                        if (e >= E) e = j;
-                        const float g = (tv[j] < 0.f) ? 0.f : tv[j] * inv;
+                        const bool take_a = tv[0] >= ov[0];
+                        const float v = take_a ? tv[0] : ov[0];
+                        int e = take_a ? ti[0] : oi[0];
+#pragma unroll
+                        for (int i = 0; i + 1 < KMAX; ++i) {
+                            tv[i] = take_a ? tv[i + 1] : tv[i];
+                            ti[i] = take_a ? ti[i + 1] : ti[i];
+                            ov[i] = take_a ? ov[i] : ov[i + 1];
+                            oi[i] = take_a ? oi[i] : oi[i + 1];
+                        }
+                        if (take_a) {
+                            tv[KMAX - 1] = -INFINITY;
+                            ti[KMAX - 1] = 0x7fffffff;
+                        } else {
+                            ov[KMAX - 1] = -INFINITY;
+                            oi[KMAX - 1] = 0x7fffffff;
+                        }
+                        if (e >= E) e = j;   // fewer finite logits than k + F (a NaN row): valid indices
+                        const float g = (v == -INFINITY) ? 0.f : __expf(v - M) * inv;
                         if (j < k) {
                             topk_idx[size_t(t) * k + j] = e;
                             topk_gate[size_t(t) * k + j] = g;
@@ -401,42 +468,40 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     }
                 }
             }
-            if (prob_sum != nullptr || psum_part != nullptr) {
+            if ((prob_sum != nullptr || psum_part != nullptr) && c < NCH) {
+                const float scale = f_mine * inv;
 #pragma unroll
-                for (int c = 0; c < NCH; ++c) {
+                for (int i = 0; i < 32; ++i)
+                    tr[lane * 33 + i] = (valid && ok && c * 32 + i < E) ? ex[i] * scale : 0.f;
+                __syncwarp();
+                float cs = 0.f;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        s_tr[ew][lane][i] = (valid && ok && c * 32 + i < E) ? l[c][i] * inv : 0.f;
-                    __syncwarp();
-                    float cs = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) cs += s_tr[ew][i][lane];
-                    s_col[q][c * 32 + lane] = cs;
-                    __syncwarp();
-                }
+                for (int i = 0; i < 32; ++i) cs += tr[i * 33 + lane];
+                s_col[q][c * 32 + lane] = cs;
             }
-        } else {
+        } else if (c == 0) {
+            // ---- E > 64: warps 2..5, two passes over all the chunks ----
             float m = -INFINITY, ssum = 0.f;
             float tv[KMAX];
             int ti[KMAX];
-    #pragma unroll
+#pragma unroll
             for (int j = 0; j < KMAX; ++j) {
                 tv[j] = -INFINITY;
                 ti[j] = 0x7fffffff;
             }
             // pass 1: online softmax statistics and top-k over the logits row
-    #pragma unroll 1
-            for (int c = 0; c < NCH; ++c) {
+#pragma unroll 1
+            for (int ch = 0; ch < NCH; ++ch) {
                 uint32_t r[32];
                 __syncwarp();
-                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(ch * 32), r);
                 tmem_ld_wait();
                 float l[32];
                 float cm = -INFINITY;
-    #pragma unroll
+#pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int e = c * 32 + i;
-                    float v = (e < E && ok) ? __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f) : -INFINITY;
+                    const int e = ch * 32 + i;
+                    float v = (e < E && ok) ? __uint_as_float(r[i]) + s_bias[e] : -INFINITY;
                     if (v != v) v = -INFINITY;
                     l[i] = v;
                     cm = fmaxf(cm, v);
@@ -444,17 +509,17 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 const float mn = fmaxf(m, cm);
                 if (mn != -INFINITY) {
                     float acc = (m == -INFINITY) ? 0.f : ssum * expf(m - mn);
-    #pragma unroll
+#pragma unroll
                     for (int i = 0; i < 32; ++i) acc += (l[i] == -INFINITY) ? 0.f : expf(l[i] - mn);
                     ssum = acc;
                     m = mn;
                 }
-    #pragma unroll
+#pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     float v = l[i];
-                    int ix = c * 32 + i;
+                    int ix = ch * 32 + i;
                     if (v == -INFINITY || !(v > tv[KMAX - 1])) continue;
-    #pragma unroll
+#pragma unroll
                     for (int j = 0; j < KMAX; ++j) {
                         if (v > tv[j]) {
                             const float tf = tv[j];
@@ -469,7 +534,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
             const float inv = 1.0f / ssum;
             if (valid && ok) {
-    #pragma unroll
+#pragma unroll
                 for (int j = 0; j < KMAX; ++j) {
                     if (j < k + F) {
                         // fewer than k + F finite logits cannot happen for k + F <= E with finite inputs;
@@ -490,27 +555,27 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
             // pass 2: per-expert sums of this tile's probabilities (fixed order)
             if (prob_sum != nullptr || psum_part != nullptr) {
-    #pragma unroll 1
-                for (int c = 0; c < NCH; ++c) {
+#pragma unroll 1
+                for (int ch = 0; ch < NCH; ++ch) {
                     uint32_t r[32];
                     __syncwarp();
-                    tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
+                    tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(ch * 32), r);
                     tmem_ld_wait();
-    #pragma unroll
+#pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const int e = c * 32 + i;
+                        const int e = ch * 32 + i;
                         float p = 0.f;
                         if (valid && ok && e < E) {
-                            float v = __uint_as_float(r[i]) + (bias != nullptr ? bias[e] : 0.f);
+                            float v = __uint_as_float(r[i]) + s_bias[e];
                             p = (v != v) ? 0.f : expf(v - m) * inv;
                         }
-                        s_tr[ew][lane][i] = p;
+                        tr[lane * 33 + i] = p;
                     }
                     __syncwarp();
                     float cs = 0.f;
-    #pragma unroll
-                    for (int i = 0; i < 32; ++i) cs += s_tr[ew][i][lane];
-                    s_col[q][c * 32 + lane] = cs;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) cs += tr[i * 33 + lane];
+                    s_col[q][ch * 32 + lane] = cs;
                     __syncwarp();
                 }
             }
