@@ -410,6 +410,109 @@ __device__ __forceinline__ void gather_chunk_rows(const int* slot_s, int a0, int
     }
 }
 
+// ---------------------------------------------------------------------------
+// Row gather by bulk copies (TMA, untiled cp.async.bulk; no multicast): one
+// thread streams the CTA's token rows of x through a ring of shared-memory
+// row buffers and stores each row to its kept slots of xp.  Addresses are
+// 16-byte aligned and sizes multiples of 16 bytes (the host checks both).
+// ---------------------------------------------------------------------------
+constexpr int kGatherRing = 32;                  // at most this many row buffers
+constexpr uint32_t kGatherSmem = 48u * 1024u;    // shared memory for the ring (and a zero row)
+constexpr int kGatherLag = 2;                    // store groups in flight before a buffer is refilled
+// Rows of fewer bytes use the thread-wide gather (ncu: bulk rows of 8 KB,
+// large-top2: 50.0 -> 41.2 us; rows of 1.5-2 KB: 23 -> 31 us, 31 -> 34 us)
+constexpr int kGatherBulkMinRow = 4096;
+
+// global -> shared (this CTA), completion counted on `bar`
+__device__ __forceinline__ void bulk_load_row(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(sdst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// shared -> global, in the thread's current bulk group
+__device__ __forceinline__ void bulk_store_row(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_u32(ssrc)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the source shared memory of all but the newest kGatherLag groups has been read
+__device__ __forceinline__ void bulk_wait_read_lag() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kGatherLag) : "memory");
+}
+// every bulk group of this thread has completed (its global writes done)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Tokens of this CTA in a chunk: y, y + Y, ... below nt (Y = gridDim.y).
+__device__ __forceinline__ int gather_my_tokens(int nt) {
+    const int Y = int(gridDim.y), y = int(blockIdx.y);
+    return (nt - y + Y - 1) / Y;
+}
+
+// Issued by one thread at the start: the first loads of the ring.
+__device__ __forceinline__ void gather_tma_start(uint8_t* ring, int ring_rows, uint64_t* bars, int t0, int nt,
+                                                 const uint8_t* __restrict__ x, int row_bytes) {
+    const int Y = int(gridDim.y), y = int(blockIdx.y);
+    const int my = gather_my_tokens(nt);
+    for (int i = 0; i < ring_rows; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+    for (int il = 0; il < min(ring_rows, my); ++il) {
+        mbar_arrive_expect_tx(&bars[il], uint32_t(row_bytes));
+        bulk_load_row(ring + size_t(il) * row_bytes, x + size_t(t0 + y + Y * il) * row_bytes, uint32_t(row_bytes),
+                      &bars[il]);
+    }
+}
+
+// Issued by the same thread once slot_s holds the chunk's slots: for each
+// token, wait for its row, store it to each kept slot (or the zero row to
+// its output row when every slot was dropped and out_zero_dropped is set),
+// then refill the buffer of the token kGatherLag back with the row
+// ring_rows ahead.  Ends when every store has completed.  A wait that gives
+// up (2 s) records MOE_ERR_TIMEOUT; the loads already issued are still
+// waited for before returning.
+__device__ __forceinline__ void gather_tma_run(uint8_t* ring, int ring_rows, uint64_t* bars, const uint8_t* zero_row,
+                                               const int* slot_s, int t0, int nt, int k,
+                                               const uint8_t* __restrict__ x, int row_bytes,
+                                               uint8_t* __restrict__ xp, uint8_t* __restrict__ out_zero_dropped,
+                                               volatile int* abort_p) {
+    const int Y = int(gridDim.y), y = int(blockIdx.y);
+    const int my = gather_my_tokens(nt);
+    int il = 0;
+    for (; il < my; ++il) {
+        const int b = il % ring_rows;
+        if (!mbar_wait(&bars[b], uint32_t((il / ring_rows) & 1), abort_p)) break;
+        const int tl = y + Y * il;
+        const uint8_t* buf = ring + size_t(b) * row_bytes;
+        bool any = false;
+        for (int c = 0; c < k; ++c) {
+            const int slot = slot_s[tl * k + c];
+            if (slot >= 0) {
+                bulk_store_row(xp + size_t(slot) * row_bytes, buf, uint32_t(row_bytes));
+                any = true;
+            }
+        }
+        if (!any && out_zero_dropped != nullptr)
+            bulk_store_row(out_zero_dropped + size_t(t0 + tl) * row_bytes, zero_row, uint32_t(row_bytes));
+        bulk_commit_group();
+        const int nxt = il + ring_rows - kGatherLag;   // reuses the buffer of token il - kGatherLag
+        if (il >= kGatherLag && nxt < my) {
+            bulk_wait_read_lag();
+            const int nb = nxt % ring_rows;
+            mbar_arrive_expect_tx(&bars[nb], uint32_t(row_bytes));
+            bulk_load_row(ring + size_t(nb) * row_bytes, x + size_t(t0 + y + Y * nxt) * row_bytes,
+                          uint32_t(row_bytes), &bars[nb]);
+        }
+    }
+    if (il < my) {
+        // gave up: every load issued so far lands before the CTA may exit
+        // loads went out for tokens [0, issued): the first ring_rows, then
+        // one refill per iteration kGatherLag .. il-1
+        const int issued = min(my, max(ring_rows, il + ring_rows - kGatherLag));
+        for (int j = il; j < issued; ++j) mbar_wait_drain(&bars[j % ring_rows], uint32_t((j / ring_rows) & 1));
+    }
+    bulk_wait_all();
+}
+
 // drop_mask (nullable): 1 for dropped assignments, 0 for kept ones
 __global__ void __launch_bounds__(kFwdThreads)
 forward_permute_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, int T, int k, int E,
@@ -471,9 +574,27 @@ forward_dispatch_kernel(const int32_t* __restrict__ idx, const float* __restrict
                         int nchunk, int capacity, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                         moe_stats* __restrict__ st, int32_t* __restrict__ perm, int32_t* __restrict__ slot_of,
                         float* __restrict__ row_gate, const uint8_t* __restrict__ x, int row_bytes,
-                        uint8_t* __restrict__ xp, uint8_t* __restrict__ out_zero_dropped) {
+                        uint8_t* __restrict__ xp, uint8_t* __restrict__ out_zero_dropped, int ring_rows) {
     pdl_wait();
     pdl_release();
+    // ring_rows > 0: the row gather runs on bulk copies through ring_rows
+    // row buffers in dynamic shared memory (then a zero row, for
+    // out_zero_dropped); its first loads go out now, under the scan
+    extern __shared__ __align__(128) uint8_t g_ring[];
+    __shared__ __align__(8) uint64_t g_bar[kGatherRing];
+    __shared__ int g_abort;
+    if (ring_rows > 0) {
+        if (threadIdx.x == 0) {
+            g_abort = 0;
+            gather_tma_start(g_ring, ring_rows, g_bar, blockIdx.x * chunk_tokens,
+                             min(chunk_tokens, T - int(blockIdx.x) * chunk_tokens), x, row_bytes);
+        }
+        if (out_zero_dropped != nullptr) {
+            uint4* z = reinterpret_cast<uint4*>(g_ring + size_t(ring_rows) * row_bytes);
+            for (int i = threadIdx.x; i < (row_bytes >> 4); i += kFwdThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
+            fence_proxy_async_smem();   // the bulk stores (async proxy) read these zeros
+        }
+    }
     __shared__ int wcnt[kDispWarps][MOE_MAX_EXPERTS];
     __shared__ int off_s[MOE_MAX_EXPERTS + 1];
     __shared__ int base_s[MOE_MAX_EXPERTS];
@@ -610,7 +731,13 @@ forward_dispatch_kernel(const int32_t* __restrict__ idx, const float* __restrict
         }
     }
     __syncthreads();
-    gather_chunk_rows(slot_s, a0, na, k, x, row_bytes, xp, out_zero_dropped);
+    if (ring_rows > 0) {
+        if (threadIdx.x == 0)
+            gather_tma_run(g_ring, ring_rows, g_bar, g_ring + size_t(ring_rows) * row_bytes, slot_s,
+                           int(blockIdx.x) * chunk_tokens, na / k, k, x, row_bytes, xp, out_zero_dropped, &g_abort);
+    } else {
+        gather_chunk_rows(slot_s, a0, na, k, x, row_bytes, xp, out_zero_dropped);
+    }
 }
 
 // ---------------------------------------------------------------------------

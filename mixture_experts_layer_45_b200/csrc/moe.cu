@@ -820,12 +820,27 @@ int run_forward_dispatch(const int32_t* idx, const float* gate, int T, int k, in
     int rc;
     if (drop_mask == nullptr && static_cast<long long>(nchunk) * E <= kFusedScanMaxEntries) {
         const int row_bytes = int(size_t(d) * elem_bytes(dtype));
+        // the row gather on bulk copies through a ring of row buffers, for
+        // rows of at least kGatherBulkMinRow bytes (below that one issuing
+        // thread's per-row overhead outweighs the copies: the thread-wide
+        // 16-byte gather is faster), when every address is 16-byte aligned
+        // and the ring holds enough rows
+        const int zero_bytes = out_zero_dropped != nullptr ? row_bytes : 0;
+        int ring_rows = 0;
+        if (x != nullptr && xp != nullptr && row_bytes >= kGatherBulkMinRow && row_bytes % 16 == 0 &&
+            aligned16(x) && aligned16(xp) &&
+            (out_zero_dropped == nullptr || aligned16(out_zero_dropped)) && row_bytes <= int(kGatherSmem)) {
+            ring_rows = std::min(kGatherRing, int((kGatherSmem - uint32_t(zero_bytes)) / uint32_t(row_bytes)));
+            if (ring_rows < kGatherLag + 1) ring_rows = 0;
+        }
+        const size_t dyn = ring_rows > 0 ? size_t(ring_rows) * row_bytes + zero_bytes : 0;
+        if (dyn > 0 && !set_smem_attr(forward_dispatch_kernel, size_t(kGatherSmem))) return MOE_ERR_CUDA;
         Launch L(MOE_KERNEL_PERMUTE, s);
         cudaError_t launch_err;
-        launch_err = launch_pdl(forward_dispatch_kernel, dim3(nchunk, permute_split(nchunk)), dim3(kFwdThreads), 0,
+        launch_err = launch_pdl(forward_dispatch_kernel, dim3(nchunk, permute_split(nchunk)), dim3(kFwdThreads), dyn,
                                 s, idx, gate, T, k, E, chunk_tokens, fhist, fpsum, nchunk, capacity, counts, offsets,
                                 st, perm, slot_of, row_gate, static_cast<const uint8_t*>(x), row_bytes,
-                                static_cast<uint8_t*>(xp), static_cast<uint8_t*>(out_zero_dropped));
+                                static_cast<uint8_t*>(xp), static_cast<uint8_t*>(out_zero_dropped), ring_rows);
         return L.finish(launch_err);
     }
     {
