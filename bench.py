@@ -394,7 +394,9 @@ def run_e2e(args, layer, x, w, world, dev):
     import torch
     import torch.distributed as dist
     from mixture_experts_layer_45_b200.layer import HostPipeline
-    e2e_steps = args.e2e_steps or max(3, min(args.steps, 100))
+    # at least 50 steps: the pipeline's first input copy and last output
+    # copy (no layer beside them) are then a small part of the timed region
+    e2e_steps = args.e2e_steps or max(50, min(args.steps, 200))
     nbuf = 4
     x_hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for _ in range(nbuf)]
     for xh in x_hosts:
