@@ -511,30 +511,46 @@ int launch_router_ep(const void* x, const void* wr, const float* bias, int T, in
     return L.finish(launch_err);
 }
 
-template <int EP, int KMAX>
+// SPLIT = 2: clusters of two CTAs share each 128-token tile's K stages
+template <int EP, int KMAX, int SPLIT>
 int launch_router_tc(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
                      const RouterOut& o, cudaStream_t s) {
     CUtensorMap tmX, tmW;
     if (!make_map_2d(&tmX, x, uint64_t(d), uint64_t(T), kRtBM)) return MOE_ERR_UNSUPPORTED;
     if (!make_map_2d(&tmW, wr, uint64_t(d), uint64_t(E), EP)) return MOE_ERR_UNSUPPORTED;
-    auto kern = router_tc_kernel<EP, KMAX>;
-    const size_t smem = RtCfg<EP>::kSmemBytes;
+    auto kern = router_tc_kernel<EP, KMAX, SPLIT>;
+    const size_t smem = RtCfg<EP, SPLIT>::kSmemBytes;
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
+    const int tiles = ceil_div(T, kRtBM);
     Launch L(MOE_KERNEL_ROUTER, s);
     cudaError_t launch_err;
-    launch_err = launch_pdl(kern, dim3(ceil_div(T, kRtBM)), dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k,
-                            o.idx, o.gate, o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate);
+    if (SPLIT == 2)
+        launch_err = launch_pdl_cluster(kern, dim3(2 * tiles), dim3(kRtThreads), smem, 2, s, tmX, tmW, bias, T, d, E,
+                                        k, o.idx, o.gate, o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate);
+    else
+        launch_err = launch_pdl(kern, dim3(tiles), dim3(kRtThreads), smem, s, tmX, tmW, bias, T, d, E, k, o.idx,
+                                o.gate, o.psum, o.psum_part, o.hist, o.F, o.fb_idx, o.fb_gate);
     return L.finish(launch_err);
 }
 
+// The K split over two CTAs per tile when the tiles leave half the SMs idle
+// and each CTA still gets eight or more K stages (large d, few tokens:
+// large-top2 runs 64 tiles of 64 stages), for up to 64 experts.
 template <int KMAX>
 int launch_router_tc_k(const void* x, const void* wr, const float* bias, int T, int d, int E, int k,
                        const RouterOut& o, cudaStream_t s) {
-    if (E <= 16) return launch_router_tc<16, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 32) return launch_router_tc<32, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 64) return launch_router_tc<64, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    if (E <= 128) return launch_router_tc<128, KMAX>(x, wr, bias, T, d, E, k, o, s);
-    return launch_router_tc<256, KMAX>(x, wr, bias, T, d, E, k, o, s);
+    const bool split = 2 * ceil_div(T, kRtBM) <= num_sms() && ceil_div(d, 64) >= 16;
+    if (E <= 16)
+        return split ? launch_router_tc<16, KMAX, 2>(x, wr, bias, T, d, E, k, o, s)
+                     : launch_router_tc<16, KMAX, 1>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 32)
+        return split ? launch_router_tc<32, KMAX, 2>(x, wr, bias, T, d, E, k, o, s)
+                     : launch_router_tc<32, KMAX, 1>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 64)
+        return split ? launch_router_tc<64, KMAX, 2>(x, wr, bias, T, d, E, k, o, s)
+                     : launch_router_tc<64, KMAX, 1>(x, wr, bias, T, d, E, k, o, s);
+    if (E <= 128) return launch_router_tc<128, KMAX, 1>(x, wr, bias, T, d, E, k, o, s);
+    return launch_router_tc<256, KMAX, 1>(x, wr, bias, T, d, E, k, o, s);
 }
 
 template <typename Tin>

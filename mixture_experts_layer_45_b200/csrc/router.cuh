@@ -226,17 +226,35 @@ constexpr int kRtThreads = 64 + 32 * kRtEpiWarps;
 // arrays (< 4 KB) below the 227 KB a CTA can have
 constexpr size_t kRtDynBudget = 227u * 1024u - 4096u;
 
-template <int EP>
+// SPLIT = 2: the two CTAs of a cluster split a tile's K stages; the
+// second sends its partial logits [128 x EP] (fp32) into the first's
+// shared memory, past the stages
+template <int EP, int SPLIT = 1>
 struct RtCfg {
     static constexpr uint32_t kABytes = kRtBM * 64 * 2;
     static constexpr uint32_t kBBytes = EP * 64 * 2;
     static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-    static constexpr int kFit = int((kRtDynBudget - 1024) / kStageBytes);
+    static constexpr uint32_t kPartBytes = SPLIT == 2 ? kRtBM * EP * 4 : 0;
+    static constexpr int kFit = int((kRtDynBudget - 1024 - kPartBytes) / kStageBytes);
     static constexpr int kStages = kFit < 12 ? kFit : 12;
     static constexpr uint32_t kTmemCols = EP < 32 ? 32 : EP;
-    static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024;
+    static constexpr size_t kPartOffset = size_t(kStages) * kStageBytes;
+    static constexpr size_t kSmemBytes = kPartOffset + kPartBytes + 1024;
     static_assert(kStages >= 4, "at least four stages");
+    static_assert(SPLIT == 1 || EP <= 64, "K split only with one or two logit chunks");
 };
+
+// shared::cluster address of the same shared-memory location in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+// 16-byte store to a shared::cluster address (another CTA's shared memory)
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
 
 // per-row record one epilogue warp hands to its partner (E <= 64)
 template <int KMAX>
@@ -248,13 +266,19 @@ struct RtRec {
 
 // KMAX >= k + F: the selection also yields the F fallback experts (fb_idx /
 // fb_gate [T, F]), as in router_topk_kernel.
-template <int EP, int KMAX>
+// SPLIT = 2 (clusters of two CTAs, grid = 2 x tiles): CTA rank r of tile
+// blockIdx.x / 2 takes K stages [r * KB/2, (r+1) * KB/2) (the second half
+// also the remainder); rank 1's epilogue warps store their partial logits
+// into rank 0's shared memory (distributed shared memory), one cluster
+// barrier that every thread of both CTAs reaches, then rank 0 adds them
+// and runs the epilogue below on the whole tile; rank 1 writes nothing else.
+template <int EP, int KMAX, int SPLIT>
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ bias, int T, int d, int E, int k, int32_t* __restrict__ topk_idx,
                  float* __restrict__ topk_gate, float* __restrict__ prob_sum, float* __restrict__ psum_part,
                  int32_t* __restrict__ hist, int F, int32_t* __restrict__ fb_idx, float* __restrict__ fb_gate) {
-    using Cfg = RtCfg<EP>;
+    using Cfg = RtCfg<EP, SPLIT>;
     constexpr int S = Cfg::kStages;
     constexpr int NCH = (EP + 31) / 32;   // 32-column TMEM chunks
     __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], done_bar;
@@ -291,7 +315,11 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     pdl_release();
     const uint32_t tmem_base = tmem_slot;
     const int KB = (d + 63) / 64;
-    const int t0 = blockIdx.x * kRtBM;
+    const uint32_t rank = SPLIT == 2 ? cluster_ctarank() : 0u;
+    const int tile = SPLIT == 2 ? int(blockIdx.x >> 1) : int(blockIdx.x);
+    const int kb_lo = SPLIT == 2 ? int(rank) * (KB / 2) : 0;
+    const int kb_hi = (SPLIT == 2 && rank == 0) ? KB / 2 : KB;
+    const int t0 = tile * kRtBM;
     volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
@@ -300,7 +328,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             uint32_t phase = 0;
             int last_parity[S];
             for (int i = 0; i < S; ++i) last_parity[i] = -1;
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = kb_lo; kb < kb_hi; ++kb) {
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_p)) break;
                 uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
                 mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
@@ -312,12 +340,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             for (int i = 0; i < S; ++i)
                 if (last_parity[i] >= 0) mbar_wait_drain(&full_bar[i], uint32_t(last_parity[i]));
         }
+        if constexpr (SPLIT == 2) cluster_sync();
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kRtBM, EP);
             int stage = 0;
             uint32_t phase = 0;
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = kb_lo; kb < kb_hi; ++kb) {
                 if (!mbar_wait(&full_bar[stage], phase, abort_p)) break;
                 tc_fence_after();
                 const uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
@@ -326,7 +355,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16(tmem_base, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc,
-                             (kb > 0 || kk > 0) ? 1u : 0u);
+                             (kb > kb_lo || kk > 0) ? 1u : 0u);
                 umma_commit(&empty_bar[stage]);
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
@@ -334,6 +363,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             // TMEM is released only after those MMAs complete (bounded wait)
             mbar_wait_drain(&done_bar, 0);
         }
+        if constexpr (SPLIT == 2) cluster_sync();
     } else {
         const int etid = threadIdx.x - 64;    // 0..255
         const int q = warp & 3;               // TMEM lane quarter
@@ -351,13 +381,32 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         RtRec<KMAX>* rec = reinterpret_cast<RtRec<KMAX>*>(smem + size_t(kRtEpiWarps) * 32 * 33 * sizeof(float));
         if constexpr (NCH <= 2) {
             // ---- one 32-expert chunk per warp ----
-            float l[32];
-            float m = -INFINITY;
+            uint32_t r[32];
             if (c < NCH) {
-                uint32_t r[32];
                 __syncwarp();
                 tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(c * 32), r);
                 tmem_ld_wait();
+            }
+            if constexpr (SPLIT == 2) {
+                // the K split: rank 1 hands its partial logits to rank 0
+                constexpr int kCols = EP < 32 ? EP : 32;   // valid columns of a chunk
+                float* part = reinterpret_cast<float*>(smem + Cfg::kPartOffset) + size_t(row) * EP + c * 32;
+                if (rank == 1 && c < NCH) {
+                    const uint32_t remote = mapa_rank(smem_u32(part), 0);
+#pragma unroll
+                    for (int i = 0; i < kCols; i += 4)
+                        st_cluster_v4(remote + uint32_t(i) * 4u, r[i], r[i + 1], r[i + 2], r[i + 3]);
+                }
+                cluster_sync();   // every thread of both CTAs passes here once
+                if (rank == 0 && c < NCH) {
+#pragma unroll
+                    for (int i = 0; i < kCols; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + part[i]);
+                }
+            }
+          if (SPLIT == 1 || rank == 0) {
+            float l[32];
+            float m = -INFINITY;
+            if (c < NCH) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int e = c * 32 + i;
@@ -479,6 +528,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 for (int i = 0; i < 32; ++i) cs += tr[i * 33 + lane];
                 s_col[q][c * 32 + lane] = cs;
             }
+          }
         } else if (c == 0) {
             // ---- E > 64: warps 2..5, two passes over all the chunks ----
             float m = -INFINITY, ssum = 0.f;
@@ -583,11 +633,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         tc_fence_before();
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kRtThreads) {
-        const float tot = ((s_col[0][e] + s_col[1][e]) + s_col[2][e]) + s_col[3][e];
-        if (psum_part != nullptr) psum_part[size_t(blockIdx.x) * E + e] = tot;
-        else if (prob_sum != nullptr) atomicAdd(prob_sum + e, tot);
-        if (hist != nullptr) hist[size_t(blockIdx.x) * E + e] = s_hist[e];
+    if (SPLIT == 1 || rank == 0) {
+        for (int e = threadIdx.x; e < E; e += kRtThreads) {
+            const float tot = ((s_col[0][e] + s_col[1][e]) + s_col[2][e]) + s_col[3][e];
+            if (psum_part != nullptr) psum_part[size_t(tile) * E + e] = tot;
+            else if (prob_sum != nullptr) atomicAdd(prob_sum + e, tot);
+            if (hist != nullptr) hist[size_t(tile) * E + e] = s_hist[e];
+        }
     }
     if (warp == 1) {
         tc_fence_after();

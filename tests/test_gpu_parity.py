@@ -143,6 +143,29 @@ def test_router_expert_count_edges(E, k):
     assert pu.max_rel_err(gate, np.take_along_axis(r["gates"], idx.astype(np.int64), 1)) <= 1e-5
 
 
+@pytest.mark.parametrize("T,d,E,k,bias", [
+    (1000, 1024, 8, 2, False),     # 16 K stages, 8 tiles: the K split over CTA pairs, ragged last tile
+    (300, 1096, 40, 3, True),      # split with a K tail (1096 = 17 * 64 + 8) and a logit bias
+    (4000, 2048, 64, 2, False),    # split at 64 experts (two logit chunks), 32 tiles
+    (64, 4096, 16, 1, True),       # one tile, 64 K stages: the pair's halves of 32 stages each
+])
+def test_router_k_split_matches_oracle(T, d, E, k, bias):
+    """Tiles of large d on few tokens split their K stages over the two CTAs
+    of a cluster (the second's partial logits added in the first's shared
+    memory); indices, gates, probability sums and the per-tile histograms
+    must be those of the one-CTA form's definition."""
+    inp = wl.draw_custom(13, T=T, d=d, ff=8, E=E, dtype="bf16", router_std=0.05)
+    if bias:
+        inp["logit_bias"] = np.linspace(-1.0, 1.0, E).astype(np.float32)
+    idx, gate, psum = run_router(inp, k, _lib.MOE_BF16)
+    r = moe_ref.route(inp["x"], inp["w_router"], k, inp.get("logit_bias"))
+    delta = pu.logit_error_bound(inp["x"], inp["w_router"], inp.get("logit_bias"))
+    n_diff, _ = pu.check_routing(idx, r["logits"], k, delta)
+    assert n_diff <= 2
+    assert pu.max_rel_err(gate, np.take_along_axis(r["gates"], idx.astype(np.int64), 1)) <= 1e-5
+    assert pu.max_rel_err(psum, r["gates"].sum(0)) <= 1e-4
+
+
 # ---------------------------------------------------------------------------
 # step 2: dispatch (bit-exact)
 # ---------------------------------------------------------------------------
