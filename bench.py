@@ -41,6 +41,10 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE layer tokens/s on 1 B200; expert-FFN TFLOP/s as % of bf16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+# dense bf16 tensor-core rate of one SM per cycle (tcgen05.mma kind::f16: a
+# 128 x 256 x 16 MMA every 128 cycles; NVIDIA's nominal 2.25 PFLOP/s dense
+# bf16 over 148 SMs at about 1.86 GHz)
+TC_FLOP_PER_SM_CYCLE = 8192
 
 
 def parse_args(argv=None):
@@ -483,6 +487,9 @@ def run_ours(args):
     offs = layer.workspace_view(w.T, "offsets", torch.int32, w.E + 1).cpu().numpy()
     E_active = int((offs[1:] > offs[:-1]).sum())
 
+    # the grouped FFN's own record of the SM clock it runs at (one load and
+    # four stores per CTA; read after the timed region: the last step's launches)
+    _lib.moe_ffn_clock_enable(True)
     sampler = ClockSampler(local_rank).start() if rank == 0 else None
     time.sleep(0.05)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -503,6 +510,8 @@ def run_ours(args):
     launches = _lib.moe_launch_count() - n0
     if sampler:
         sampler.stop()
+    ffn_clock = _lib.moe_ffn_clock_read()
+    _lib.moe_ffn_clock_enable(False)
     err = _lib.moe_get_error()
     if err != 0:
         raise RuntimeError(f"device error in the timed region: {_lib.status_string(err)}")
@@ -570,6 +579,21 @@ def run_ours(args):
                 "frac": achieved / peaks["hbm_gbs"]}
     roof.update({"kernel": dom, "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes,
                  "traffic": committed_traffic(dom, workload_tag(w))})
+    # the FFN launches at the clock they ran at: tcgen05 kind::f16 retires
+    # TC_FLOP_PER_SM_CYCLE dense bf16 flop per SM per cycle
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ffn_clock_rec = {}
+    for k in ("ffn1", "ffn2"):
+        mhz, span_us = ffn_clock[k]
+        if mhz > 0 and span_us > 0:
+            rec = {"sm_mhz": mhz, "span_us": span_us}
+            if w.dtype == "bf16":
+                rec["tensor_frac_at_clock"] = flops_dom / (sms * TC_FLOP_PER_SM_CYCLE * mhz * 1e6 * span_us * 1e-6)
+            ffn_clock_rec[k] = rec
+    if dom in ffn_clock_rec:
+        roof["sm_mhz_in_kernel"] = ffn_clock_rec[dom]["sm_mhz"]
+        if "tensor_frac_at_clock" in ffn_clock_rec[dom]:
+            roof["tensor_frac_at_clock"] = ffn_clock_rec[dom]["tensor_frac_at_clock"]
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -586,6 +610,8 @@ def run_ours(args):
                 "frac_of_burst": (ffn_tflops / peaks["bf16_tflops"]) if ffn_tflops else None,
                 "flops_per_step": ffn_flops, "ms_per_step": ffn_ms},
         "kernels": kernels,
+        "ffn_clock": dict(ffn_clock_rec, note="SM cycles / ns inside the last timed step's fc1 and fc2 launches "
+                          "(median over CTAs); tensor_frac_at_clock = FLOPs / (SMs x 8192 x cycles)"),
         "e2e": e2e,
         "clocks": clocks,
         "gpu_launches": launches,

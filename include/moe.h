@@ -445,6 +445,23 @@ MOE_API int moe_timing_enable(int enable);
  * entries; either may be NULL. */
 MOE_API int moe_timing_read(double* ms_per_kernel, int64_t* launches_per_kernel);
 
+/* SM clock of the grouped-FFN launches.  The power cap can hold the SM
+ * clock well below its maximum within a millisecond, faster than an
+ * outside clock sampler (nvidia-smi) follows it, so a tensor-bound launch
+ * is judged by the clock it actually ran at.  moe_ffn_clock_enable(1)
+ * clears the record and makes every later fc1 / fc2 launch of the grouped
+ * FFN note, in thread 0 of each CTA, the SM cycle counter and the global
+ * nanosecond timer when the CTA starts its tiles and when it is done;
+ * moe_ffn_clock_enable(0) stops that.  Both synchronise the device.
+ * moe_ffn_clock_read synchronises and writes, for the most recent fc1 (index
+ * 0) and fc2 (index 1) launch, the median over its CTAs of cycles per
+ * microsecond (sm_mhz[2], MHz) and the time from the first CTA's start to
+ * the last one's end (span_us[2]); 0 where no launch was recorded.  Either
+ * array may be NULL.  Device-side cost while on: one load and four stores
+ * per CTA. */
+MOE_API int moe_ffn_clock_enable(int enable);
+MOE_API int moe_ffn_clock_read(double* sm_mhz, double* span_us);
+
 /* Profiler annotations (the blog "MoE Parallelism for Inference", section
  * on profiling: look at the router step and the expert passes separately).
  * When on, every entry point that enqueues GPU work opens an NVTX range

@@ -85,6 +85,8 @@ _SIGS = {
     "moe_timing_enable": (_I, [_I]),
     "moe_timing_read": (_I, [_P, _P]),
     "moe_trace_enable": (_I, [_I]),
+    "moe_ffn_clock_enable": (_I, [_I]),
+    "moe_ffn_clock_read": (_I, [_P, _P]),
     "moe_trace_enabled": (_I, []),
 }
 EXPORTED = sorted(_SIGS)
@@ -324,6 +326,18 @@ def moe_timing_read():
     n = (ctypes.c_int64 * MOE_NUM_KERNELS)()
     _check(load().moe_timing_read(ctypes.cast(ms, _P), ctypes.cast(n, _P)), "moe_timing_read")
     return {name: (ms[i], int(n[i])) for i, name in enumerate(KERNEL_NAMES)}
+
+
+def moe_ffn_clock_enable(enable: bool):
+    _check(load().moe_ffn_clock_enable(1 if enable else 0), "moe_ffn_clock_enable")
+
+
+def moe_ffn_clock_read():
+    """{"ffn1": (SM MHz, span us), "ffn2": (...)} of the most recent launches."""
+    mhz = (ctypes.c_double * 2)()
+    us = (ctypes.c_double * 2)()
+    _check(load().moe_ffn_clock_read(ctypes.cast(mhz, _P), ctypes.cast(us, _P)), "moe_ffn_clock_read")
+    return {"ffn1": (mhz[0], us[0]), "ffn2": (mhz[1], us[1])}
 
 
 def moe_debug_wait_timeout(limit_ns: int, stream=None):

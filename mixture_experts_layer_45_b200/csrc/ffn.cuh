@@ -20,6 +20,27 @@ namespace moe {
 
 enum FfnMode { kFc1Gelu = 0, kFc2Gate = 1 };
 
+// SM clock of the grouped-FFN launches (moe_ffn_clock_enable / _read):
+// while g_ffn_clock_on is set, thread 0 of every CTA records %clock64 and
+// %globaltimer when it starts its tiles and when it is done (slots
+// [mode][cta][0..3]), so that the host can divide cycles by nanoseconds:
+// under the power cap the clock drops within a millisecond, faster than an
+// outside sampler follows it.
+constexpr int kClockCtas = 256;
+__device__ int g_ffn_clock_on;
+__device__ unsigned long long g_ffn_clock[2][kClockCtas][4];
+
+__device__ __forceinline__ bool ffn_clock_on() { return *reinterpret_cast<volatile int*>(&g_ffn_clock_on) != 0; }
+
+__device__ __forceinline__ void ffn_clock_mark(bool on, int mode, int slot) {
+    if (on && threadIdx.x == 0 && blockIdx.x < kClockCtas) {
+        unsigned long long c;
+        asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+        g_ffn_clock[mode][blockIdx.x][slot] = c;
+        g_ffn_clock[mode][blockIdx.x][slot + 1] = globaltimer_ns();
+    }
+}
+
 // Shared always-on experts (notebook section "Exercises", item 3: every
 // token also passes through a few experts outside the router) run as S
 // extra row groups after the E routed ones, in the same launch: group E + s
@@ -211,6 +232,16 @@ constexpr int kTcThreads = 64 + 32 * kTcEpiWarps;
 // threads of the single-CTA kernel with EPIW epilogue warps
 constexpr int tc_threads(int epiw) { return 64 + 32 * epiw; }
 
+// Per-warp shared-memory staging of the epilogue's output: the warp turns
+// its lane-per-row values into row segments so that each global store
+// instruction writes whole 32-byte sectors of a few rows instead of 16
+// bytes of each of 32 rows.  kEpiSegB bytes (columns x 2) per row and
+// round: 64 with up to eight epilogue warps, 32 with more (the staging of
+// all epilogue warps then still fits beside the pipeline stages).
+__host__ __device__ constexpr uint32_t epi_seg_bytes(int epiw) { return epiw <= 8 ? 64u : 32u; }
+__host__ __device__ constexpr uint32_t epi_stage_bytes(int epiw) { return uint32_t(epiw) * 32u * epi_seg_bytes(epiw); }
+
+
 template <int BN, int STAGES>
 struct TcCfg {
     static constexpr uint32_t kABytes = kTcBM * kTcBK * 2;
@@ -218,8 +249,37 @@ struct TcCfg {
     static constexpr uint32_t kStageBytes = kABytes + kBBytes;
     static constexpr uint32_t kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                          : (2 * BN <= 256) ? 256 : 512;
-    static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;   // + alignment slack
+    // stages, then the epilogue warps' staging buffers (+ alignment slack)
+    static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
+    static constexpr size_t smem_bytes(int epiw) { return kSmemBytes + epi_stage_bytes(epiw); }
 };
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// TMA tile store (no multicast) of one staged box from shared memory, and
+// the issuing thread's bulk-group bookkeeping
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void epi_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the staged box has been read out of shared memory
+__device__ __forceinline__ void epi_bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the stores are complete
+__device__ __forceinline__ void epi_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // One warp's share of a tile's epilogue.  The warp reads TMEM lane quarter
 // q (accumulator rows q*32 .. q*32+31, one per lane) and the 32-column
@@ -229,16 +289,42 @@ struct TcCfg {
 // "empty" barrier) as soon as its last group is in registers, so the MMA
 // can start the next-but-one tile while this one is still being written.
 // Then bias (from global memory: the same 16 bytes for every lane, a
-// broadcast), GELU (fc1) or the row gate (fc2), bf16 rounding and 16-byte
-// stores to row `crow` of C (skipped for rows past the group, `valid`).
+// broadcast), GELU (fc1) or the row gate (fc2) and bf16 rounding, row by
+// row (lane = row) into the warp's staging buffer `stg` (32 rows x SEG
+// bytes; 16-byte unit u of row r at unit u ^ swz(r): the layout of the
+// TMA 64-byte / 32-byte swizzle, free of bank conflicts both row-wise and
+// column-wise).  When all 32 rows are inside the group and C's rows are
+// contiguous (`tma`), one lane stores the box with a TMA tile store
+// through tmC (box {SEG / 2 columns, 32 rows}), so the output leaves
+// through the copy engine rather than the load/store pipeline that the
+// operand stream shares; otherwise each store instruction covers
+// 32 / (SEG / 16) rows x SEG bytes, to row `crow` of C for rows inside the
+// group (`valid`).  The warp's lane 0 waits for its boxes to be read out of
+// the buffer before the buffer is rewritten; the caller waits for them to
+// complete before the CTA exits.
 template <int BN, int MODE, int EPIW, typename Release>
 __device__ __forceinline__ void epilogue_tile_warp(uint32_t tacc, int q, int sub, int lane, bool valid, size_t crow,
                                                    int n0, int N, float g, const __nv_bfloat16* __restrict__ bb,
-                                                   __nv_bfloat16* __restrict__ C, Release release) {
+                                                   __nv_bfloat16* __restrict__ C, uint32_t stg, const CUtensorMap* tmC,
+                                                   bool tma_rows, Release release) {
     constexpr int kSub = EPIW / 4;
     constexpr int kChunks = (BN / 32 + kSub - 1) / kSub;   // chunks per warp (the last may be past BN)
     constexpr int kGroup = kChunks < 2 ? kChunks : 2;
+    constexpr int kSegB = int(epi_seg_bytes(EPIW));
+    constexpr int kUnits = kSegB / 16;                     // 16-byte units per row and round
+    constexpr int kRounds = 64 / kSegB;                    // rounds per 32-column chunk
+    constexpr int kRowsPer = 32 / kUnits;                  // rows per store instruction
     static_assert(EPIW % 4 == 0 && EPIW >= 4, "whole lane quarters");
+    // unit swizzle of row r: 4 units (64-byte rows) or 2 (32-byte rows)
+    auto swz = [](int r) { return kUnits == 4 ? ((r >> 1) & 3) : ((r >> 2) & 1); };
+    // the rows this lane stores (one per store instruction i) and their masks
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    const bool tma = tma_rows && vmask == 0xffffffffu;   // warp-uniform
+    size_t drow[kUnits];
+#pragma unroll
+    for (int i = 0; i < kUnits; ++i)
+        drow[i] = size_t(__shfl_sync(0xffffffffu, static_cast<unsigned long long>(crow), i * kRowsPer + lane / kUnits));
+    const int uu = lane % kUnits;
 #pragma unroll
     for (int g0 = 0; g0 < kChunks; g0 += kGroup) {
         uint32_t r[kGroup][32];
@@ -258,27 +344,53 @@ __device__ __forceinline__ void epilogue_tile_warp(uint32_t tacc, int q, int sub
         for (int j = 0; j < kGroup; ++j) {
             const int c = sub + (g0 + j) * kSub;
             const int nb = n0 + c * 32;
-            if (!(g0 + j < kChunks && c < BN / 32) || !valid || nb >= N) continue;
-            __nv_bfloat16* cp = C + crow * N + nb;
+            if (!(g0 + j < kChunks && c < BN / 32) || nb >= N) continue;   // warp-uniform
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                if (nb + v * 8 >= N) break;
-                // bias[nb + 8v .. +8): one 16-byte load (N % 8 == 0, 16-byte aligned rows)
-                const uint4 bw = __ldg(reinterpret_cast<const uint4*>(bb + nb + v * 8));
-                const uint32_t bwv[4] = {bw.x, bw.y, bw.z, bw.w};
-                float o[8];
+            for (int h = 0; h < kRounds; ++h) {
+                if (lane == 0) epi_bulk_wait_read();   // the buffer's previous box is out
+                __syncwarp();
+                // this lane's row: kUnits units of 8 columns each
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float bi = (i & 1) ? bf16_hi(bwv[i >> 1]) : bf16_lo(bwv[i >> 1]);
-                    const float cval = __uint_as_float(r[j][v * 8 + i]) + bi;
-                    o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
+                for (int v = 0; v < kUnits; ++v) {
+                    const int col = h * (kSegB / 2) + v * 8;   // within the chunk
+                    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                    if (nb + col < N) {
+                        // bias[nb + col .. +8): one 16-byte load (N % 8 == 0, 16-byte aligned rows)
+                        const uint4 bw = __ldg(reinterpret_cast<const uint4*>(bb + nb + col));
+                        const uint32_t bwv[4] = {bw.x, bw.y, bw.z, bw.w};
+                        float o[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float bi = (i & 1) ? bf16_hi(bwv[i >> 1]) : bf16_lo(bwv[i >> 1]);
+                            const float cval = __uint_as_float(r[j][col + i]) + bi;
+                            o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
+                        }
+                        u.x = pack_bf16x2(o[0], o[1]);
+                        u.y = pack_bf16x2(o[2], o[3]);
+                        u.z = pack_bf16x2(o[4], o[5]);
+                        u.w = pack_bf16x2(o[6], o[7]);
+                    }
+                    st_shared_v4(stg + uint32_t(lane * kSegB + ((v ^ swz(lane)) << 4)), u);
                 }
-                uint4 u;
-                u.x = pack_bf16x2(o[0], o[1]);
-                u.y = pack_bf16x2(o[2], o[3]);
-                u.z = pack_bf16x2(o[4], o[5]);
-                u.w = pack_bf16x2(o[6], o[7]);
-                *reinterpret_cast<uint4*>(cp + v * 8) = u;
+                if (tma) {
+                    fence_proxy_async_smem();   // the TMA store (async proxy) reads these writes
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(tmC, stg, nb + h * (kSegB / 2), int(drow[0]));
+                        epi_bulk_commit();
+                    }
+                } else {
+                    __syncwarp();
+                    // row segments out: instruction i covers rows i*kRowsPer ..
+#pragma unroll
+                    for (int i = 0; i < kUnits; ++i) {
+                        const int rr = i * kRowsPer + lane / kUnits;
+                        const uint4 u = ld_shared_v4(stg + uint32_t(rr * kSegB + ((uu ^ swz(rr)) << 4)));
+                        const int col = nb + h * (kSegB / 2) + uu * 8;
+                        if (((vmask >> rr) & 1u) && col < N) *reinterpret_cast<uint4*>(C + drow[i] * N + col) = u;
+                    }
+                    __syncwarp();
+                }
             }
         }
     }
@@ -295,7 +407,8 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                    const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
                    const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C, SharedGroups sh,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                   const __nv_bfloat16* __restrict__ bias2, int walk_zip) {
+                   const __nv_bfloat16* __restrict__ bias2, int walk_zip, const __grid_constant__ CUtensorMap tmC,
+                   int c_tma) {
     using Cfg = TcCfg<BN, STAGES>;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN: whole 32-column epilogue chunks, MMA N <= 256");
     __shared__ TileTable tt;
@@ -339,6 +452,8 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     const int total = tt.start[G];
     const int KB = (K + kTcBK - 1) / kTcBK;
     volatile int* abort_p = &abort_flag;
+    const bool clock_on = ffn_clock_on();
+    ffn_clock_mark(clock_on, MODE, 0);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -417,6 +532,8 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         // flag is raised; no named barrier is involved.
         const int q = warp & 3;
         const int sub = (warp - 2) >> 2;
+        const uint32_t stg = smem_u32(smem + size_t(STAGES) * Cfg::kStageBytes) +
+                             uint32_t(warp - 2) * 32u * epi_seg_bytes(EPIW);
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -438,13 +555,16 @@ ffn_tc_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             tc_fence_after();
             uint64_t* tempty = &tempty_bar[acc];
             epilogue_tile_warp<BN, MODE, EPIW>(tmem_base + uint32_t(acc * BN), q, sub, lane, valid, crow, tc.nt * BN, N,
-                                               g, bb, C, [tempty]() { mbar_arrive(tempty); });
+                                               g, bb, C, stg, &tmC, c_tma != 0,
+                                               [tempty]() { mbar_arrive(tempty); });
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        if (lane == 0) epi_bulk_wait_all();   // this warp's tile stores are complete
     }
 
     __syncthreads();
+    ffn_clock_mark(clock_on, MODE, 2);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);
@@ -475,7 +595,9 @@ struct Tc2Cfg {
     static constexpr uint32_t kBBytes = (kTc2BN / 2) * kTcBK * 2;
     static constexpr uint32_t kStageBytes = kABytes + kBBytes;
     static constexpr uint32_t kTmemCols = 2 * kTc2BN;   // two accumulators
+    // stages, then the epilogue warps' staging buffers (+ alignment slack)
     static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
+    static constexpr size_t smem_bytes(int epiw) { return kSmemBytes + epi_stage_bytes(epiw); }
 };
 
 template <int STAGES, int MODE, int EPIW>
@@ -485,7 +607,8 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const __nv_bfloat16* __restrict__ bias, const float* __restrict__ row_gate,
                     const int32_t* __restrict__ out_rows, __nv_bfloat16* __restrict__ C, SharedGroups sh,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                    const __nv_bfloat16* __restrict__ bias2, int walk_zip) {
+                    const __nv_bfloat16* __restrict__ bias2, int walk_zip, const __grid_constant__ CUtensorMap tmC,
+                    int c_tma) {
     using Cfg = Tc2Cfg<STAGES>;
     constexpr int BN = kTc2BN;
     __shared__ TileTable tt;
@@ -532,6 +655,8 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int total = tt.start[G];
     const int KB = (K + kTcBK - 1) / kTcBK;
     volatile int* abort_p = &abort_flag;
+    const bool clock_on = ffn_clock_on();
+    ffn_clock_mark(clock_on, MODE, 0);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -599,6 +724,8 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // pair arrives on CTA 0's "empty" barrier (CTA 1 through mapa).
         const int q = warp & 3;
         const int sub = (warp - 2) >> 2;
+        const uint32_t stg = smem_u32(smem + size_t(STAGES) * Cfg::kStageBytes) +
+                             uint32_t(warp - 2) * 32u * epi_seg_bytes(EPIW);
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = pair; t < total; t += npairs) {
@@ -618,13 +745,15 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tc_fence_after();
             uint64_t* tempty = &tempty_bar[acc];
             epilogue_tile_warp<BN, MODE, EPIW>(tmem_base + uint32_t(acc * BN), q, sub, lane, valid, crow, tc.nt * BN, N,
-                                               g, bb, C, [tempty, rank]() {
+                                               g, bb, C, stg, &tmC, c_tma != 0,
+                                               [tempty, rank]() {
                                                    if (rank == 0) mbar_arrive(tempty);
                                                    else mbar_arrive_remote(tempty, 0);
                                                });
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        if (lane == 0) epi_bulk_wait_all();   // this warp's tile stores are complete
     }
 
     // teardown: every pair MMA has completed (it reads both CTAs' shared
@@ -635,6 +764,7 @@ ffn_tc2_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     __syncthreads();
     cluster_sync();
+    ffn_clock_mark(clock_on, MODE, 2);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);

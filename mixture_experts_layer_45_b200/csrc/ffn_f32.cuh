@@ -102,6 +102,8 @@ ffn_tc_f32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int total = tt.start[G];
     const int KB = (K + kTfBK - 1) / kTfBK;
     volatile int* abort_p = &abort_flag;
+    const bool clock_on = ffn_clock_on();
+    ffn_clock_mark(clock_on, MODE, 0);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -261,6 +263,7 @@ ffn_tc_f32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
 
     __syncthreads();
+    ffn_clock_mark(clock_on, MODE, 2);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);

@@ -439,6 +439,21 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The grouped FFN's output C [rows, cols] bf16 for the epilogue's TMA
+// tile stores: box {seg_bytes / 2 columns, 32 rows}, the swizzle whose
+// span equals the box's row (64 or 32 bytes)
+bool make_store_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t seg_bytes) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {seg_bytes / 2, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, seg_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Raises a kernel's dynamic shared memory limit once per device (later
 // calls, e.g. while a CUDA graph is being captured, only look it up).
 std::mutex g_attr_mu;
@@ -672,11 +687,13 @@ long long ffn_tiles_ub(int routed_rows_ub, int E, const SharedArgs& sa, int BM, 
 template <int BN, int STAGES, int MODE, int EPIW = kTcEpiWarps>
 int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
               const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
-              const SharedArgs& sa, int kernel_id, cudaStream_t s, bool zip = false) {
+              int c_rows, const SharedArgs& sa, int kernel_id, cudaStream_t s, bool zip = false) {
     FfnMaps mp;
     if (!make_ffn_maps(mp, a, a_cols, a_rows, w, N, E, sa, kTcBM, BN, MOE_BF16)) return MOE_ERR_UNSUPPORTED;
+    CUtensorMap tmC;
+    if (!make_store_map(&tmC, c, uint64_t(N), uint64_t(c_rows), epi_seg_bytes(EPIW))) return MOE_ERR_UNSUPPORTED;
     auto kern = ffn_tc_bf16_kernel<BN, STAGES, MODE, EPIW>;
-    const size_t smem = TcCfg<BN, STAGES>::kSmemBytes;
+    const size_t smem = TcCfg<BN, STAGES>::smem_bytes(EPIW);
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     const long long tiles_ub = ffn_tiles_ub(routed_rows_ub, E, sa, kTcBM, N, BN);
     const int grid = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms())));
@@ -685,7 +702,7 @@ int launch_tc(const void* a, int a_cols, int a_rows, int routed_rows_ub, const v
     launch_err = launch_pdl(kern, dim3(grid), dim3(tc_threads(EPIW)), smem, s, mp.a, mp.b, offsets, E, N, a_cols,
                             static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
                             static_cast<__nv_bfloat16*>(c), sa.g, mp.a2, mp.b2,
-                            static_cast<const __nv_bfloat16*>(sa.bias), zip ? 1 : 0);
+                            static_cast<const __nv_bfloat16*>(sa.bias), zip ? 1 : 0, tmC, out_rows == nullptr ? 1 : 0);
     return L.finish(launch_err);
 }
 
@@ -696,11 +713,13 @@ constexpr int kTc2Stages = 6;
 template <int MODE, int EPIW = kTcEpiWarps>
 int launch_tc2(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
                const int32_t* offsets, const void* bias, const float* row_gate, const int32_t* out_rows, void* c,
-               const SharedArgs& sa, int kernel_id, cudaStream_t s, bool zip = false) {
+               int c_rows, const SharedArgs& sa, int kernel_id, cudaStream_t s, bool zip = false) {
     FfnMaps mp;
     if (!make_ffn_maps(mp, a, a_cols, a_rows, w, N, E, sa, 128, kTc2BN / 2, MOE_BF16)) return MOE_ERR_UNSUPPORTED;
+    CUtensorMap tmC;
+    if (!make_store_map(&tmC, c, uint64_t(N), uint64_t(c_rows), epi_seg_bytes(EPIW))) return MOE_ERR_UNSUPPORTED;
     auto kern = ffn_tc2_bf16_kernel<kTc2Stages, MODE, EPIW>;
-    const size_t smem = Tc2Cfg<kTc2Stages>::kSmemBytes;
+    const size_t smem = Tc2Cfg<kTc2Stages>::smem_bytes(EPIW);
     if (!set_smem_attr(kern, smem)) return MOE_ERR_CUDA;
     const long long tiles_ub = ffn_tiles_ub(routed_rows_ub, E, sa, kTc2BM, N, kTc2BN);
     const int pairs = int(std::max(1ll, std::min<long long>(tiles_ub, num_sms() / 2)));
@@ -709,7 +728,8 @@ int launch_tc2(const void* a, int a_cols, int a_rows, int routed_rows_ub, const 
     launch_err = launch_pdl_cluster(kern, dim3(2 * pairs), dim3(tc_threads(EPIW)), smem, 2, s, mp.a, mp.b, offsets, E, N,
                                     a_cols, static_cast<const __nv_bfloat16*>(bias), row_gate, out_rows,
                                     static_cast<__nv_bfloat16*>(c), sa.g, mp.a2, mp.b2,
-                                    static_cast<const __nv_bfloat16*>(sa.bias), zip ? 1 : 0);
+                                    static_cast<const __nv_bfloat16*>(sa.bias), zip ? 1 : 0, tmC,
+                                    out_rows == nullptr ? 1 : 0);
     return L.finish(launch_err);
 }
 
@@ -794,23 +814,26 @@ int run_ffn(const void* xp, const int32_t* offsets, int max_rows, int E, int d, 
         // save (measured on the skewed and large workloads)
         if (fc1_pairs)
             rc = launch_tc2<kFc1Gelu, kTcFc1EpiWarps>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr,
-                                                      nullptr, h, s1, MOE_KERNEL_FFN1, s, zip);
+                                                      nullptr, h, h_rows, s1, MOE_KERNEL_FFN1, s, zip);
         else
             rc = launch_tc<kTcBN, kTcStages, kFc1Gelu, kTcFc1EpiWarps>(xp, d, max_rows, max_rows, w1, ff, E,
-                                                                       offsets, b1, nullptr, nullptr, h, s1,
-                                                                       MOE_KERNEL_FFN1, s, zip);
+                                                                       offsets, b1, nullptr, nullptr, h, h_rows,
+                                                                       s1, MOE_KERNEL_FFN1, s, zip);
         if (rc != MOE_OK) return rc;
+        // yp's rows for the epilogue's TMA stores (h_rows; with out_rows the
+        // kernels store row by row and never use that map)
         if (use_pairs)
-            return launch_tc2<kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp, s2,
-                                        MOE_KERNEL_FFN2, s, zip);
+            return launch_tc2<kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate, out_rows, yp,
+                                        h_rows, s2, MOE_KERNEL_FFN2, s, zip);
         // fc2 of a layer with about one M tile per expert (switch-top1: 96
         // tiles of 256 columns for 148 SMs): 192-column tiles put 4/3 as many
         // SMs on the weight stream
         if (fc2_narrow_tiles(max_rows, E, d, se))
             return launch_tc<kTcBNNarrow, kTcStagesNarrow, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2,
-                                                                     row_gate, out_rows, yp, s2, MOE_KERNEL_FFN2, s, zip);
+                                                                     row_gate, out_rows, yp, h_rows, s2, MOE_KERNEL_FFN2, s,
+                                                                     zip);
         return launch_tc<kTcBN, kTcStages, kFc2Gate>(h, ff, h_rows, max_rows, w2, d, E, offsets, b2, row_gate,
-                                                     out_rows, yp, s2, MOE_KERNEL_FFN2, s, zip);
+                                                     out_rows, yp, h_rows, s2, MOE_KERNEL_FFN2, s, zip);
     }
     rc = launch_tf32x3<kFc1Gelu>(xp, d, max_rows, max_rows, w1, ff, E, offsets, b1, nullptr, nullptr, h, s1,
                                  MOE_KERNEL_FFN1, s, zip);
@@ -1440,6 +1463,44 @@ int moe_timing_enable(int enable) {
         }
     }
     g_timing.enabled = enable != 0;
+    return MOE_OK;
+}
+
+int moe_ffn_clock_enable(int enable) {
+    const int on = enable ? 1 : 0;
+    if (on) {
+        // a fresh record: launches that ran before this call leave no trace
+        void* rec = nullptr;
+        if (cudaGetSymbolAddress(&rec, g_ffn_clock) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemset(rec, 0, sizeof(g_ffn_clock)) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (cudaMemcpyToSymbol(g_ffn_clock_on, &on, sizeof(on)) != cudaSuccess) return MOE_ERR_CUDA;
+    return cudaDeviceSynchronize() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_ffn_clock_read(double* sm_mhz, double* span_us) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    static unsigned long long rec[2][kClockCtas][4];
+    if (cudaMemcpyFromSymbol(rec, g_ffn_clock, sizeof(rec)) != cudaSuccess) return MOE_ERR_CUDA;
+    for (int m = 0; m < 2; ++m) {
+        std::vector<double> mhz;
+        unsigned long long t_lo = ~0ull, t_hi = 0;
+        for (int c = 0; c < kClockCtas; ++c) {
+            const unsigned long long* r = rec[m][c];
+            if (r[1] == 0 || r[3] <= r[1]) continue;   // no launch, or one still running
+            mhz.push_back(double(r[2] - r[0]) / double(r[3] - r[1]) * 1e3);
+            t_lo = std::min(t_lo, r[1]);
+            t_hi = std::max(t_hi, r[3]);
+        }
+        double med = 0.0;
+        if (!mhz.empty()) {
+            std::sort(mhz.begin(), mhz.end());
+            const size_t n = mhz.size();
+            med = (n & 1) ? mhz[n / 2] : 0.5 * (mhz[n / 2 - 1] + mhz[n / 2]);
+        }
+        if (sm_mhz) sm_mhz[m] = med;
+        if (span_us) span_us[m] = mhz.empty() ? 0.0 : double(t_hi - t_lo) * 1e-3;
+    }
     return MOE_OK;
 }
 
