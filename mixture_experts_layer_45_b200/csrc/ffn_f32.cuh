@@ -11,22 +11,43 @@ namespace moe {
 // ===========================================================================
 // fp32 path: three-pass TF32 on the tensor cores (error-compensated).
 //
-// Each fp32 operand v is split into hi = v rounded to TF32 (low 13 mantissa
-// bits cleared, round to nearest) and lo = v - hi (exact in fp32, |lo| <=
-// 2^-11 |hi|); then A B^T = hi_A hi_B^T + hi_A lo_B^T + lo_A hi_B^T + lo_A lo_B^T
-// and the last product, about 2^-22 of the result, is dropped.  Each kept
+// Each fp32 operand v is split into a TF32 part hi and lo = v - hi (exact in
+// fp32): for the activations A hi = v rounded to nearest on the 13 low
+// mantissa bits (|lo| <= 2^-11 |hi|); for the weights hi = v truncated to
+// its top 19 bits, which is what the tensor cores read of the raw fp32
+// value, so the weight tile is used as loaded (|lo| < 2^-10 |hi|).  Then
+// A B^T = hi_A hi_B^T + hi_A lo_B^T + lo_A hi_B^T + lo_A lo_B^T and the last
+// product, at most about 2^-21 of the result, is dropped.  Each kept
 // product is a tcgen05.mma kind::tf32 with fp32 accumulation in tensor
 // memory, so the result carries fp32-level error (the split-precision
 // scheme of Ootomo & Yokota 2022) at the tensor cores' TF32 rate.
 //
+// The A operand (the 128 activation rows) goes to the tensor cores from
+// tensor memory, the weight operand from shared memory: per K step the
+// converters read the landed A tile once and write its hi and lo parts
+// straight into the stage's two TMEM operand regions (tcgen05.st), and
+// the weight tile gets only a lo tile beside it.  Per stage that moves 128
+// KB through shared memory (TMA 32, converter reads 32, weight lo writes
+// 16, MMA operand reads 48) for 768 tensor cycles, where staging A's parts
+// in shared memory too (and rewriting both hi parts) moved 224 KB.
+//
 // Warp roles (576 threads):
 //   warp 0        TMA producer: raw fp32 A and W tiles, 32 columns (128 B)
 //                 of K per stage, 128B swizzle
-//   warp 1        TMEM allocator and MMA issuer: 3 MMAs per K step of 8
+//   warp 1        TMEM allocator and MMA issuer: 3 MMAs per K step of 8,
+//                 A from tensor memory
 //   warps 2..9    epilogue, as the bf16 kernel, fp32 stores
-//   warps 10..17  converters: for each landed stage, hi in place and lo
-//                 into the stage's lo tiles (same swizzled positions), then a
-//                 proxy fence so the tensor cores see the generic writes
+//   warps 10..17  converters: for each landed stage, warp w takes TMEM lane
+//                 quarter w % 4 and half (w - 10) / 4 of the 32 K columns of
+//                 A (lane = row: 16 values from the swizzled tile, split, two
+//                 tcgen05.st), then an eighth of the weight tile's lo parts
+//                 into the lo tile (same swizzled positions); then
+//                 the TMEM stores are waited for and the shared-memory writes
+//                 fenced to the async proxy before the stage is released to
+//                 the MMA issuer
+//
+// Tensor memory (512 columns): the two accumulators (BN columns each), then
+// per stage A hi (32 columns: one per K element, lane = row) and A lo.
 // ===========================================================================
 constexpr int kTfBK = 32;            // 32 fp32 = 128 B = one swizzle row
 constexpr int kTfConvWarps = 8;
@@ -37,10 +58,46 @@ struct TfCfg {
     static constexpr uint32_t kABytes = kTcBM * kTfBK * 4;
     static constexpr uint32_t kBBytes = BN * kTfBK * 4;
     static constexpr uint32_t kLoadBytes = kABytes + kBBytes;        // what TMA brings per stage
-    static constexpr uint32_t kStageBytes = 2 * kLoadBytes;          // + the lo tiles
-    static constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256 : 512;
+    static constexpr uint32_t kStageBytes = kLoadBytes + kBBytes;    // + the weight lo tile
+    static constexpr uint32_t kAOpCol = 2 * BN;                      // first TMEM column of the A parts
+    static constexpr uint32_t kTmemCols = 512;
     static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
+    static_assert(2 * BN + STAGES * 2 * kTfBK <= 512, "accumulators and A operand parts fit in TMEM");
+    // TMEM column of stage s's A hi (part 0) or lo (part 1)
+    __host__ __device__ static constexpr uint32_t a_col(int s, int part) { return kAOpCol + uint32_t(s * 2 + part) * kTfBK; }
 };
+
+// D(tmem) (+)= A(tmem) * B(smem)^T, kind::tf32: A's 128 rows in the 128
+// lanes, its K elements in consecutive columns
+__device__ __forceinline__ void umma_tf32_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// this warp's lane quarter: lane i writes 16 consecutive 32-bit columns of
+// TMEM lane (quarter base + i)
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// What kind::tf32 reads of an fp32 operand: its top 19 bits (sign, exponent,
+// 10 mantissa bits), the low 13 mantissa bits cleared.  (Checked on B200: a
+// weight split as raw value plus v - tf32_trunc(v) gives the same error as
+// the explicit round-to-nearest split, 2.8e-5 against 2.7e-5 max-norm
+// relative on d = 768, ff = 3072; a rounding tensor core would leave an
+// error near 2^-11.)
+__device__ __forceinline__ float tf32_trunc(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
 
 __device__ __forceinline__ float tf32_round(float v) {
     // round to nearest on bit 13 (ties away from zero); inf / nan pass through
@@ -154,16 +211,17 @@ ffn_tc_f32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (!mbar_wait(&conv_bar[stage], phase, abort_p)) { ok = false; break; }
                     tc_fence_after();
                     const uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
-                    const uint64_t ahi = sdesc_kmajor_sw128(smem_u32(sa));
                     const uint64_t bhi = sdesc_kmajor_sw128(smem_u32(sa + Cfg::kABytes));
-                    const uint64_t alo = sdesc_kmajor_sw128(smem_u32(sa + Cfg::kLoadBytes));
-                    const uint64_t blo = sdesc_kmajor_sw128(smem_u32(sa + Cfg::kLoadBytes + Cfg::kABytes));
+                    const uint64_t blo = sdesc_kmajor_sw128(smem_u32(sa + Cfg::kLoadBytes));
+                    const uint32_t ahi = tmem_base + Cfg::a_col(stage, 0);
+                    const uint32_t alo = tmem_base + Cfg::a_col(stage, 1);
 #pragma unroll
-                    for (int kk = 0; kk < kTfBK / 8; ++kk) {   // K = 8 per tf32 MMA = 32 B
+                    for (int kk = 0; kk < kTfBK / 8; ++kk) {   // K = 8 per tf32 MMA: 32 B of B, 8 TMEM columns of A
                         const uint64_t o = uint64_t(2 * kk);
-                        umma_tf32(d_tmem, alo + o, bhi + o, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                        umma_tf32(d_tmem, ahi + o, blo + o, idesc, 1u);
-                        umma_tf32(d_tmem, ahi + o, bhi + o, idesc, 1u);
+                        const uint32_t c = uint32_t(8 * kk);
+                        umma_tf32_ts(d_tmem, alo + c, bhi + o, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        umma_tf32_ts(d_tmem, ahi + c, blo + o, idesc, 1u);
+                        umma_tf32_ts(d_tmem, ahi + c, bhi + o, idesc, 1u);
                     }
                     umma_commit(&empty_bar[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -179,27 +237,49 @@ ffn_tc_f32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     } else if (warp >= 2 + kTcEpiWarps) {
         // ---------------- converters (warps 10..17) ----------------
         const int ctid = threadIdx.x - (64 + 32 * kTcEpiWarps);   // 0..255
-        constexpr int kVec = int(Cfg::kLoadBytes / 16);           // float4s per stage
+        const int q = warp & 3;                                   // TMEM lane quarter
+        const int hh = (warp - (2 + kTcEpiWarps)) >> 2;           // half of A's 32 K columns
+        const int row = q * 32 + lane;                            // A row = TMEM lane
+        const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
+        constexpr int kBVec = int(Cfg::kBBytes / 16);             // float4s of the weight tile
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, abort_p))) { ok = false; break; }
-                float4* hi = reinterpret_cast<float4*>(smem + size_t(stage) * Cfg::kStageBytes);
-                float4* lo = reinterpret_cast<float4*>(smem + size_t(stage) * Cfg::kStageBytes + Cfg::kLoadBytes);
-#pragma unroll 4
-                for (int i = ctid; i < kVec; i += 32 * kTfConvWarps) {
-                    const float4 v = hi[i];
-                    float4 h, l;
-                    h.x = tf32_round(v.x); l.x = v.x - h.x;
-                    h.y = tf32_round(v.y); l.y = v.y - h.y;
-                    h.z = tf32_round(v.z); l.z = v.z - h.z;
-                    h.w = tf32_round(v.w); l.w = v.w - h.w;
-                    hi[i] = h;
-                    lo[i] = l;
+                uint8_t* st_base = smem + size_t(stage) * Cfg::kStageBytes;
+                // A: row `row`, 16-byte chunks 4*hh .. 4*hh+3 of its 128 bytes
+                // (128B swizzle: chunk c of row r sits at chunk c ^ (r & 7))
+                uint32_t ahi[16], alo[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int c = 4 * hh + j;
+                    const float4 v = *reinterpret_cast<const float4*>(st_base + size_t(row) * 128 +
+                                                                      size_t((c ^ (row & 7)) << 4));
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float h = tf32_round(vv[i]);
+                        ahi[j * 4 + i] = __float_as_uint(h);
+                        alo[j * 4 + i] = __float_as_uint(vv[i] - h);
+                    }
                 }
-                fence_proxy_async_smem();
+                tmem_st_32x32b_x16(lane_base + Cfg::a_col(stage, 0) + uint32_t(16 * hh), ahi);
+                tmem_st_32x32b_x16(lane_base + Cfg::a_col(stage, 1) + uint32_t(16 * hh), alo);
+                // the weight tile stays as loaded (its hi part is what the
+                // tensor cores read of it); its lo part into the stage's lo tile
+                const float4* bw = reinterpret_cast<const float4*>(st_base + Cfg::kABytes);
+                float4* blo = reinterpret_cast<float4*>(st_base + Cfg::kLoadBytes);
+#pragma unroll 4
+                for (int i = ctid; i < kBVec; i += 32 * kTfConvWarps) {
+                    const float4 v = bw[i];
+                    blo[i] = make_float4(v.x - tf32_trunc(v.x), v.y - tf32_trunc(v.y), v.z - tf32_trunc(v.z),
+                                         v.w - tf32_trunc(v.w));
+                }
+                tmem_st_wait();               // this warp's TMEM stores are done
+                fence_proxy_async_smem();     // the tensor cores see the shared-memory writes
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&conv_bar[stage]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }

@@ -733,8 +733,8 @@ int launch_tc2(const void* a, int a_cols, int a_rows, int routed_rows_ub, const 
     return L.finish(launch_err);
 }
 
-// fp32 on the tensor cores, three-pass TF32: 128 x 128 tiles, 3 stages
-constexpr int kTfBN = 128, kTfStages = 3;
+// fp32 on the tensor cores, three-pass TF32: 128 x 128 tiles, 4 stages
+constexpr int kTfBN = 128, kTfStages = 4;
 
 template <int MODE>
 int launch_tf32x3(const void* a, int a_cols, int a_rows, int routed_rows_ub, const void* w, int N, int E,
