@@ -13,11 +13,13 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_ffn_clock_record(dtype):
+# (T, E, k): about 225 rows per expert runs the single-CTA kernels; 2000
+# rows per expert runs bf16 fc2 on CTA pairs
+@pytest.mark.parametrize("dtype,T,E,k", [("bf16", 900, 8, 2), ("f32", 900, 8, 2), ("bf16", 8000, 4, 1)])
+def test_ffn_clock_record(dtype, T, E, k):
     dt = _lib.MOE_BF16 if dtype == "bf16" else _lib.MOE_F32
-    inp = wl.draw_custom(5, T=900, d=128, ff=256, E=8, dtype=dtype, router_std=0.5)
-    layer = MoELayer(MoEParams.from_arrays(inp, dt, DEV), 2, -1)
+    inp = wl.draw_custom(5, T=T, d=128, ff=256, E=E, dtype=dtype, router_std=0.5)
+    layer = MoELayer(MoEParams.from_arrays(inp, dt, DEV), k, -1)
     x = to_device(inp["x"], dt, DEV)
     ref = layer.forward(x).clone()
 
