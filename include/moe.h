@@ -457,8 +457,8 @@ MOE_API int moe_timing_read(double* ms_per_kernel, int64_t* launches_per_kernel)
  * 0) and fc2 (index 1) launch, the median over its CTAs of cycles per
  * microsecond (sm_mhz[2], MHz) and the time from the first CTA's start to
  * the last one's end (span_us[2]); 0 where no launch was recorded.  Either
- * array may be NULL.  Device-side cost while on: one load and four stores
- * per CTA. */
+ * array may be NULL.  Device-side cost: one load per CTA of each FFN
+ * launch, and four stores per CTA while on. */
 MOE_API int moe_ffn_clock_enable(int enable);
 MOE_API int moe_ffn_clock_read(double* sm_mhz, double* span_us);
 

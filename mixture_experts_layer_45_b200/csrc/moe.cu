@@ -1480,13 +1480,13 @@ int moe_ffn_clock_enable(int enable) {
 
 int moe_ffn_clock_read(double* sm_mhz, double* span_us) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
-    static unsigned long long rec[2][kClockCtas][4];
-    if (cudaMemcpyFromSymbol(rec, g_ffn_clock, sizeof(rec)) != cudaSuccess) return MOE_ERR_CUDA;
+    std::vector<unsigned long long> rec(size_t(2) * kClockCtas * 4);
+    if (cudaMemcpyFromSymbol(rec.data(), g_ffn_clock, sizeof(g_ffn_clock)) != cudaSuccess) return MOE_ERR_CUDA;
     for (int m = 0; m < 2; ++m) {
         std::vector<double> mhz;
         unsigned long long t_lo = ~0ull, t_hi = 0;
         for (int c = 0; c < kClockCtas; ++c) {
-            const unsigned long long* r = rec[m][c];
+            const unsigned long long* r = rec.data() + (size_t(m) * kClockCtas + c) * 4;
             if (r[1] == 0 || r[3] <= r[1]) continue;   // no launch, or one still running
             mhz.push_back(double(r[2] - r[0]) / double(r[3] - r[1]) * 1e3);
             t_lo = std::min(t_lo, r[1]);
