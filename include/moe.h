@@ -448,7 +448,7 @@ MOE_API int moe_timing_read(double* ms_per_kernel, int64_t* launches_per_kernel)
 /* SM clock of the grouped-FFN launches.  The power cap can hold the SM
  * clock well below its maximum within a millisecond, faster than an
  * outside clock sampler (nvidia-smi) follows it, so a tensor-bound launch
- * is judged by the clock it actually ran at.  moe_ffn_clock_enable(1)
+ * is read against the clock it actually ran at.  moe_ffn_clock_enable(1)
  * clears the record and makes every later fc1 / fc2 launch of the grouped
  * FFN note, in thread 0 of each CTA, the SM cycle counter and the global
  * nanosecond timer when the CTA starts its tiles and when it is done;
