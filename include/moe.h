@@ -407,7 +407,10 @@ MOE_API int moe_get_error(void* stream);
 /* Device GELU forms, for testing: y[i] = GELU(x[i]) (x, y device float[n]).
  * variant 0: 0.5 x (1 + erff(x / sqrt 2)), the fp32 path's form;
  * variant 1: the same with erf by Abramowitz & Stegun eq. 7.1.26 (|error|
- * <= 1.5e-7), the bf16 tensor-core epilogue's form. */
+ * <= 1.5e-7);
+ * variant 2: variant 1 evaluated two values at a time with the paired fp32
+ * instructions, the bf16 tensor-core epilogue's form (bit for bit variant
+ * 1).  Any other variant: MOE_ERR_INVALID_ARG. */
 MOE_API int moe_debug_gelu(const float* x, float* y, int n, int variant, void* stream);
 
 /* Failure-path check: launches one kernel whose bounded wait on a barrier

@@ -281,6 +281,63 @@ __device__ __forceinline__ void epi_bulk_wait_read() { asm volatile("cp.async.bu
 // the stores are complete
 __device__ __forceinline__ void epi_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Two fp32 values in 64 bits (x in the low half) for sm_100's paired fp32
+// instructions (add / mul / fma .rn.f32x2): each is the same IEEE operation
+// on both halves, so a paired evaluation gives bit for bit what two scalar
+// ones give, in half the instructions.
+__device__ __forceinline__ uint64_t f2_pack(float x, float y) {
+    return (uint64_t(__float_as_uint(y)) << 32) | __float_as_uint(x);
+}
+__device__ __forceinline__ float f2_x(uint64_t p) { return __uint_as_float(uint32_t(p)); }
+__device__ __forceinline__ float f2_y(uint64_t p) { return __uint_as_float(uint32_t(p >> 32)); }
+__device__ __forceinline__ uint64_t f2_splat(float v) { return f2_pack(v, v); }
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// gelu_as (Abramowitz & Stegun eq. 7.1.26 erf) on two values at once: the
+// same constants and the same operations in the same order, the FMA-pipe
+// ones paired, the reciprocal and the exponential per value; bit for bit
+// gelu_as of each half (1 - q is formed as fma(q, -1, 1), the same
+// correctly rounded value).
+__device__ __forceinline__ uint64_t gelu_as2(uint64_t v) {
+    const uint64_t a = v & 0x7FFFFFFF7FFFFFFFull;                       // |v|
+    const uint64_t d = fma2(f2_splat(0.2316418883f), a, f2_splat(1.0f));
+    const uint64_t t = f2_pack(rcp_approx(f2_x(d)), rcp_approx(f2_y(d)));
+    uint64_t poly = fma2(f2_splat(0.5307027145f), t, f2_splat(-0.7265760135f));
+    poly = fma2(poly, t, f2_splat(0.7107068705f));
+    poly = fma2(poly, t, f2_splat(-0.142248368f));
+    poly = fma2(poly, t, f2_splat(0.127414796f));
+    poly = mul2(poly, t);
+    const uint64_t e2 = mul2(mul2(f2_splat(-0.72134752044448169f), v), v);
+    const uint64_t q = mul2(poly, f2_pack(ex2_approx(f2_x(e2)), ex2_approx(f2_y(e2))));
+    const uint64_t w = fma2(q, f2_splat(-1.0f), f2_splat(1.0f));         // 1 - q
+    const uint64_t phi = f2_pack(f2_x(v) >= 0.f ? f2_x(w) : f2_x(q), f2_y(v) >= 0.f ? f2_y(w) : f2_y(q));
+    return mul2(v, phi);
+}
+
+// moe_debug_gelu variant 2: the paired form, y[i] for i in pairs
+__global__ void gelu2_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+    for (int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 2 * gridDim.x * blockDim.x) {
+        const float b = (i + 1 < n) ? x[i + 1] : 0.f;
+        const uint64_t r = gelu_as2(f2_pack(x[i], b));
+        y[i] = f2_x(r);
+        if (i + 1 < n) y[i + 1] = f2_y(r);
+    }
+}
+
 // One warp's share of a tile's epilogue.  The warp reads TMEM lane quarter
 // q (accumulator rows q*32 .. q*32+31, one per lane) and the 32-column
 // chunks sub, sub + EPIW/4, ... of the BN-column accumulator at `tacc`.  It
@@ -358,17 +415,16 @@ __device__ __forceinline__ void epilogue_tile_warp(uint32_t tacc, int q, int sub
                         // bias[nb + col .. +8): one 16-byte load (N % 8 == 0, 16-byte aligned rows)
                         const uint4 bw = __ldg(reinterpret_cast<const uint4*>(bb + nb + col));
                         const uint32_t bwv[4] = {bw.x, bw.y, bw.z, bw.w};
-                        float o[8];
+                        uint32_t o[4];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float bi = (i & 1) ? bf16_hi(bwv[i >> 1]) : bf16_lo(bwv[i >> 1]);
-                            const float cval = __uint_as_float(r[j][col + i]) + bi;
-                            o[i] = (MODE == kFc1Gelu) ? gelu_as(cval) : g * cval;
+                        for (int p = 0; p < 4; ++p) {
+                            // columns col + 2p, col + 2p + 1 as one pair
+                            const uint64_t acc = (uint64_t(r[j][col + 2 * p + 1]) << 32) | r[j][col + 2 * p];
+                            const uint64_t cval = add2(acc, f2_pack(bf16_lo(bwv[p]), bf16_hi(bwv[p])));
+                            const uint64_t y = (MODE == kFc1Gelu) ? gelu_as2(cval) : mul2(f2_splat(g), cval);
+                            o[p] = pack_bf16x2(f2_x(y), f2_y(y));
                         }
-                        u.x = pack_bf16x2(o[0], o[1]);
-                        u.y = pack_bf16x2(o[2], o[3]);
-                        u.z = pack_bf16x2(o[4], o[5]);
-                        u.w = pack_bf16x2(o[6], o[7]);
+                        u = make_uint4(o[0], o[1], o[2], o[3]);
                     }
                     st_shared_v4(stg + uint32_t(lane * kSegB + ((v ^ swz(lane)) << 4)), u);
                 }

@@ -1437,11 +1437,14 @@ int moe_get_error(void* stream) {
 }
 
 int moe_debug_gelu(const float* x, float* y, int n, int variant, void* stream) {
-    if (n < 0 || (variant != 0 && variant != 1)) return MOE_ERR_INVALID_ARG;
+    if (n < 0 || variant < 0 || variant > 2) return MOE_ERR_INVALID_ARG;
     if (n == 0) return MOE_OK;
     if (!x || !y) return MOE_ERR_INVALID_ARG;
-    gelu_probe_kernel<<<std::min(ceil_div(n, 256), 1024), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n,
-                                                                                                     variant);
+    if (variant == 2)
+        gelu2_probe_kernel<<<std::min(ceil_div(n, 512), 1024), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+    else
+        gelu_probe_kernel<<<std::min(ceil_div(n, 256), 1024), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n,
+                                                                                                         variant);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

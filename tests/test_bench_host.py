@@ -70,7 +70,7 @@ def test_committed_profiles_are_current():
 
 def test_traffic_is_read_for_the_bench_workload():
     w = wl.workload("large-top2")                  # the bench's default workload
-    assert bench.committed_traffic("ffn1", bench.workload_tag(w)) == 1526504608.0
+    assert bench.committed_traffic("ffn1", bench.workload_tag(w)) == 1527696240.0
     assert bench.committed_traffic("ffn1", "no-such-workload") is None
 
 

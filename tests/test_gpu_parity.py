@@ -264,14 +264,21 @@ def test_grouped_ffn_tile_edges(dtype, sizes, d, ff):
 
 
 def test_device_gelu_forms_match_erf():
-    """Both device GELU forms against CUDA's erff form and the float64 definition:
-    the A&S 7.1.26 erf is within its published bound (1.5e-7) plus fp32 rounding."""
-    xs = np.concatenate([np.linspace(-12, 12, 200001), [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0]]).astype(np.float32)
+    """The device GELU forms against CUDA's erff form and the float64 definition:
+    the A&S 7.1.26 erf is within its published bound (1.5e-7) plus fp32 rounding,
+    and the paired-instruction form the bf16 epilogue runs (variant 2) equals the
+    scalar one bit for bit, odd element count included."""
+    xs = np.concatenate([np.linspace(-12, 12, 200001),
+                         [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0, 3e-39, 0.5]]).astype(np.float32)
     x = torch.from_numpy(xs).to(DEV)
     y0 = torch.empty_like(x)
     y1 = torch.empty_like(x)
+    y2 = torch.empty_like(x)
     _lib.moe_debug_gelu(x, y0, x.numel(), 0)
     _lib.moe_debug_gelu(x, y1, x.numel(), 1)
+    _lib.moe_debug_gelu(x, y2, x.numel(), 2)
+    assert x.numel() % 2 == 1
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
     y0, y1 = y0.cpu().double().numpy(), y1.cpu().double().numpy()
     ref = moe_ref.gelu(xs.astype(np.float64))
     scale = np.maximum(np.abs(xs.astype(np.float64)), 1.0)
