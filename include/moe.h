@@ -36,7 +36,9 @@
  *   t's j-th choice (j = 0 is the largest gate).
  * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *   legacy default stream) and never synchronises the host, except
- *   moe_get_error and moe_timing_read.  Calls are CUDA-graph capturable.
+ *   moe_get_error, moe_timing_read, moe_ffn_clock_enable / _read and the
+ *   pipeline calls (each says so).  The layer calls are CUDA-graph
+ *   capturable.
  * - Errors: argument and shape errors are returned synchronously, before
  *   anything is launched (MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED,
  *   MOE_ERR_WORKSPACE).  A failed launch returns MOE_ERR_CUDA.  Errors that
