@@ -130,6 +130,18 @@ def test_no_launch_and_timing_read_without_gpu(lib):
     assert set(t) == set(_lib.KERNEL_NAMES) and all(v == (0.0, 0) for v in t.values())
 
 
+def test_ffn_clock_calls_fail_cleanly_without_gpu(lib):
+    """Without a device the clock record's calls report MOE_ERR_CUDA (they
+    touch device memory) and launch nothing."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert lib.moe_ffn_clock_enable(1) == _lib.MOE_ERR_CUDA
+    mhz = (ctypes.c_double * 2)()
+    assert lib.moe_ffn_clock_read(ctypes.cast(mhz, ctypes.c_void_p), None) == _lib.MOE_ERR_CUDA
+    assert _lib.moe_launch_count() == 0
+
+
 def test_shared_workspace_size_and_offsets(lib):
     T, d, ff, E, k = 4096, 768, 3072, 32, 1
     base = _lib.moe_workspace_size(T, d, ff, E, k, _lib.MOE_BF16)
